@@ -1,0 +1,189 @@
+/*
+ * usp.h -- C ABI of libusp.so: the per-rank hot path of USP (Ulysses + Ring)
+ * context-parallel attention on one NVIDIA B200 (sm_100a), with the P virtual
+ * ranks of a P_ulysses x P_ring mesh emulated on the one GPU.
+ *
+ * Sources (the pages on long_context_exact_tma):
+ *   - "Boosting Spec Eagle: USP for Long-Context Training": section "The
+ *     Solution" (Ulysses, Ring Attention, their USP hybrid; each ring device
+ *     holds a slice of the sequence and exchanges with its neighbours) and
+ *     "Implementation Details" (load balancing across the ring).
+ *   - DeepSpeed-Ulysses summary, section "Wie DeepSpeed-Ulysses funktioniert":
+ *     the input is split along the sequence; an all-to-all before attention
+ *     gives each GPU the whole sequence for a subset of heads; afterwards the
+ *     results are gathered and re-laid out.
+ *   - Blockwise Parallel Transformer (related-papers list of the LSS
+ *     Transformer page): attention computed block by block.
+ *   - LongNet slides, "Results": attention variants built on FlashAttention,
+ *     i.e. exact softmax attention evaluated tile by tile.
+ *
+ * Notation. P = P_u * P_r ranks; rank r = i * P_u + u (i: ring index, u:
+ * Ulysses index). c = S / (2P) tokens per zigzag chunk; rank r holds chunks r
+ * and 2P-1-r of the sequence. L = S / P_r tokens per head-sharded rank.
+ *
+ * Layouts (all row-major, last index contiguous):
+ *   global        [B][S][H][D]
+ *   rank-major    [P][B][2c][H][D]            (after the zigzag shard)
+ *   head-sharded  [P_r][P_u][B][L][H/P_u][D]  (after the seq->head all-to-all;
+ *                 the L tokens of rank (i,u) are, for u' = 0..P_u-1 in order,
+ *                 the 2c tokens of rank (i,u'))
+ *   LSE           head-sharded with D = 1: [P_r][P_u][B][L][Hq/P_u], fp32,
+ *                 natural log (global form [B][S][Hq]).
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   - Arguments are validated synchronously; on a bad argument nothing is
+ *     launched and a negative usp_status is returned (usp_last_error() then
+ *     holds a message). Work is enqueued asynchronously on `stream`.
+ *   - The library allocates no device memory: scratch comes from the caller's
+ *     workspace (usp_attn_workspace_size). The first 256 bytes of a workspace
+ *     hold a device status word that the attention kernels set when a bounded
+ *     wait gives up; usp_workspace_status() reads and clears it.
+ *   - Supported: D in {64, 128}; Hq % Hkv == 0; Hq % P_u == 0; Hkv % P_u == 0;
+ *     S % (2P) == 0. Other shapes return USP_ERR_UNSUPPORTED.
+ */
+#ifndef USP_H
+#define USP_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  USP_OK = 0,
+  USP_ERR_INVALID_ARG = -1, /* null/misaligned pointer, negative size, bad enum */
+  USP_ERR_UNSUPPORTED = -2, /* a shape outside the supported set */
+  USP_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
+  USP_ERR_TIMEOUT = -4,     /* a kernel's bounded wait gave up; outputs undefined */
+  USP_ERR_WORKSPACE = -5    /* workspace missing or smaller than required */
+} usp_status;
+
+typedef enum { USP_BF16 = 0, USP_F32 = 1 } usp_dtype;
+
+enum { USP_MODE_FUSED = 0, USP_MODE_STEPWISE = 1 };
+
+/* Library version (major*10000 + minor*100 + patch). */
+int usp_version(void);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* usp_last_error(void);
+
+/*
+ * Zigzag shard: global [B][S][H][D] -> rank-major [P][B][2c][H][D]; rank r
+ * receives chunks r and 2P-1-r (load balancing of the causal ring, "Boosting
+ * Spec Eagle", "Implementation Details"). A bit-exact copy of H*D-element token
+ * rows. usp_zigzag_unshard is its inverse. dtype selects 2- or 4-byte
+ * elements; D*elem_size must be a multiple of 4 bytes.
+ */
+int usp_zigzag_shard(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                     void* stream);
+int usp_zigzag_unshard(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                       void* stream);
+
+/*
+ * Ulysses all-to-all emulated as an on-device gather (DeepSpeed-Ulysses,
+ * "Wie DeepSpeed-Ulysses funktioniert"): rank-major [P][B][2c][H][D] ->
+ * head-sharded [P_r][P_u][B][L][H/P_u][D]. Rank (i,u) receives head group u of
+ * every rank (i,u') of its Ulysses group. usp_head2seq_permute is the inverse
+ * (the regather after attention). Bit-exact; 16-byte vector copies when the
+ * row of H/P_u heads is a multiple of 16 bytes. D may be 1 (the LSE layout).
+ */
+int usp_seq2head_permute(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                         void* stream);
+int usp_head2seq_permute(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                         void* stream);
+
+/*
+ * Bytes of workspace needed by usp_attn_fwd (bwd = 0, by mode) or
+ * usp_attn_bwd (bwd = 1). Returns 0 for an unsupported shape.
+ *   fused fwd   : 256 (status word)
+ *   stepwise fwd: 256 + P_r * B*S*Hq * (4*D + 4)  (fp32 partials of every ring step)
+ *   bwd         : 256 + B*S*Hq * (4*D + 4)        (fp32 dQ accumulator, Delta)
+ */
+size_t usp_attn_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, int mode,
+                               int bwd);
+
+/*
+ * Forward of exact softmax attention for every virtual rank, block by block
+ * over the ring's KV chunks (Ring Attention, "Boosting Spec Eagle", "The
+ * Solution"; blockwise attention, BPT), with the partial (O, LSE) pairs of the
+ * ring steps combined by log-sum-exp.
+ *   q            [P_r][P_u][B][L][Hq/P_u][D]  bf16 (head-sharded)
+ *   k, v         [P_r][P_u][B][L][Hkv/P_u][D] bf16
+ *   out          like q, bf16: O_i = sum_j softmax_j(scale * q_i.k_j) v_j
+ *   lse          [P_r][P_u][B][L][Hq/P_u] fp32, natural log
+ * Query head h of rank (i,u) attends kv head h / (Hq/Hkv) of the same rank
+ * group u; rank (i,u) at ring step t reads the KV of rank ((i-t) mod P_r, u).
+ * causal: key visible iff its original token position <= the query's.
+ * scale = 1/sqrt(D).
+ * mode USP_MODE_FUSED: one launch, ring steps merged online in the kernel.
+ * mode USP_MODE_STEPWISE: one launch per ring step writing fp32 partials into
+ * the workspace, then usp_lse_merge -- the ring algorithm step for step.
+ */
+int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
+                 int Hkv, int D, int causal, int P_u, int P_r, int mode, void* workspace, size_t ws_bytes,
+                 void* stream);
+
+/*
+ * Backward of usp_attn_fwd for every virtual rank. P is recomputed from the
+ * final merged LSE: P_ij = exp(scale q_i.k_j - LSE_i), dP = dO V^T,
+ * dS = P o (dP - Delta), Delta_i = sum_d dO_id O_id; dQ = scale dS K,
+ * dK = scale dS^T Q, dV = P^T dO, dK/dV summed over the q-heads of a GQA group.
+ *   q, out, dO   head-sharded bf16 (out is the forward output)
+ *   lse          the forward LSE
+ *   dQ           head-sharded bf16 (accumulated in fp32 in the workspace)
+ *   dK, dV       head-sharded fp32, [P_r][P_u][B][L][Hkv/P_u][D]
+ */
+int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dO,
+                 void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D, int causal, int P_u,
+                 int P_r, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Log-sum-exp merge of n_parts ring-step partials (the partial results each
+ * ring step produces, "Boosting Spec Eagle", "The Solution"):
+ *   LSE = m + log sum_t exp(LSE_t - m),  m = max_t LSE_t
+ *   O   = sum_t exp(LSE_t - LSE) O_t
+ * A partial with LSE_t = -inf (no visible key) contributes nothing; a row with
+ * every LSE_t = -inf yields O = 0, LSE = -inf.
+ *   o_parts    [n_parts][rows][D] fp32;  lse_parts [n_parts][rows] fp32
+ *   out        [rows][D], bf16 or fp32 (out_dtype);  lse_out [rows] fp32
+ * D must be a multiple of 4 (<= 256).
+ */
+int usp_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,
+                  int out_dtype, float* lse_out, void* stream);
+
+/*
+ * Backward preprocess: Delta_i = sum_d dO_id * O_id in fp32, for `rows` rows of
+ * D bf16 elements (any row-major layout, the same for both inputs).
+ */
+int usp_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D, void* stream);
+
+/*
+ * Synchronises `stream`, returns USP_ERR_TIMEOUT if a kernel that used this
+ * workspace recorded a timed-out wait since the last call (and clears the
+ * word), USP_OK otherwise. `site` (may be NULL) receives the recorded site code.
+ */
+int usp_workspace_status(void* workspace, int* site, void* stream);
+
+/*
+ * Limit of every bounded device wait launched by this thread from now on, in
+ * nanoseconds (default 2e9). A test hook: a very small limit makes waits give up.
+ */
+void usp_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing will ever complete, with limit `limit_ns`; the wait gives up,
+ * the kernel records its site and returns. Then usp_workspace_status on the
+ * same workspace reports USP_ERR_TIMEOUT.
+ */
+int usp_selftest_wait_timeout(void* workspace, size_t ws_bytes, unsigned long long limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* USP_H */

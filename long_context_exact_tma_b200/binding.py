@@ -1,0 +1,169 @@
+"""ctypes binding of libusp.so: one Python function per C entry point of
+include/usp.h, with the same name and argument order. Arguments may be torch
+tensors (their data pointers are passed) or integers (raw device pointers).
+Marshalling only: every step of the path runs in the library's kernels.
+
+Loading fails loudly (ImportError) when libusp.so has not been built; there is
+no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libusp.so")
+
+USP_OK = 0
+USP_ERR_INVALID_ARG = -1
+USP_ERR_UNSUPPORTED = -2
+USP_ERR_CUDA = -3
+USP_ERR_TIMEOUT = -4
+USP_ERR_WORKSPACE = -5
+USP_BF16 = 0
+USP_F32 = 1
+USP_MODE_FUSED = 0
+USP_MODE_STEPWISE = 1
+
+# name -> (restype, argtypes); mirrors include/usp.h
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_LL = ctypes.c_longlong
+_SZ = ctypes.c_size_t
+_LAYOUT = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
+SIGNATURES = {
+    "usp_version": (_I, []),
+    "usp_last_error": (ctypes.c_char_p, []),
+    "usp_zigzag_shard": (_I, _LAYOUT),
+    "usp_zigzag_unshard": (_I, _LAYOUT),
+    "usp_seq2head_permute": (_I, _LAYOUT),
+    "usp_head2seq_permute": (_I, _LAYOUT),
+    "usp_attn_workspace_size": (_SZ, [_I] * 10),
+    "usp_attn_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_P, _SZ, _P]),
+    "usp_attn_bwd": (_I, [_P] * 9 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_lse_merge": (_I, [_P, _P, _I, _LL, _I, _P, _I, _P, _P]),
+    "usp_bwd_preprocess": (_I, [_P, _P, _P, _LL, _I, _P]),
+    "usp_workspace_status": (_I, [_P, _P, _P]),
+    "usp_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "usp_selftest_wait_timeout": (_I, [_P, _SZ, ctypes.c_ulonglong, _P]),
+}
+
+_lib = None
+
+
+class UspError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"usp status {code}: {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_exact_tma_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(rc: int) -> int:
+    if rc != USP_OK:
+        raise UspError(rc, lib().usp_last_error().decode())
+    return rc
+
+
+def usp_version() -> int:
+    return lib().usp_version()
+
+
+def usp_last_error() -> str:
+    return lib().usp_last_error().decode()
+
+
+def _layout(name, src, dst, B, S, H, D, dtype, P_u, P_r, stream=None, check=True):
+    rc = getattr(lib(), name)(_ptr(src), _ptr(dst), B, S, H, D, dtype, P_u, P_r, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_zigzag_shard(src, dst, B, S, H, D, dtype, P_u, P_r, stream=None, check=True):
+    return _layout("usp_zigzag_shard", src, dst, B, S, H, D, dtype, P_u, P_r, stream, check)
+
+
+def usp_zigzag_unshard(src, dst, B, S, H, D, dtype, P_u, P_r, stream=None, check=True):
+    return _layout("usp_zigzag_unshard", src, dst, B, S, H, D, dtype, P_u, P_r, stream, check)
+
+
+def usp_seq2head_permute(src, dst, B, S, H, D, dtype, P_u, P_r, stream=None, check=True):
+    return _layout("usp_seq2head_permute", src, dst, B, S, H, D, dtype, P_u, P_r, stream, check)
+
+
+def usp_head2seq_permute(src, dst, B, S, H, D, dtype, P_u, P_r, stream=None, check=True):
+    return _layout("usp_head2seq_permute", src, dst, B, S, H, D, dtype, P_u, P_r, stream, check)
+
+
+def usp_attn_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, mode, bwd) -> int:
+    return int(lib().usp_attn_workspace_size(B, S, Hq, Hkv, D, int(causal), P_u, P_r, mode, int(bwd)))
+
+
+def usp_attn_fwd(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, P_u, P_r, mode, workspace, ws_bytes,
+                 stream=None, check=True):
+    rc = lib().usp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D, int(causal),
+                            P_u, P_r, mode, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_attn_bwd(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes,
+                 stream=None, check=True):
+    rc = lib().usp_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
+                            _ptr(dV), B, S, Hq, Hkv, D, int(causal), P_u, P_r, _ptr(workspace), ws_bytes,
+                            _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_lse_merge(o_parts, lse_parts, n_parts, rows, D, out, out_dtype, lse_out, stream=None, check=True):
+    rc = lib().usp_lse_merge(_ptr(o_parts), _ptr(lse_parts), n_parts, rows, D, _ptr(out), out_dtype,
+                             _ptr(lse_out), _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_bwd_preprocess(out, dO, delta, rows, D, stream=None, check=True):
+    rc = lib().usp_bwd_preprocess(_ptr(out), _ptr(dO), _ptr(delta), rows, D, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_workspace_status(workspace, stream=None):
+    """(status, site) of the device status word; clears it."""
+    site = ctypes.c_int(0)
+    rc = lib().usp_workspace_status(_ptr(workspace), ctypes.byref(site), _stream(stream))
+    return rc, site.value
+
+
+def usp_set_wait_limit_ns(ns: int) -> None:
+    lib().usp_set_wait_limit_ns(int(ns))
+
+
+def usp_selftest_wait_timeout(workspace, ws_bytes, limit_ns, stream=None, check=True):
+    rc = lib().usp_selftest_wait_timeout(_ptr(workspace), ws_bytes, int(limit_ns), _stream(stream))
+    return _check(rc) if check else rc

@@ -1,0 +1,292 @@
+// usp_api.cu -- the extern "C" entry points of libusp.so (declared in include/usp.h):
+// argument validation, workspace accounting, TMA tensor maps and kernel launches.
+#include <cudaTypedefs.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/usp.h"
+#include "usp_internal.h"
+
+using namespace usp;
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local unsigned long long g_wait_ns = 2000000000ull;
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(USP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_size(int dtype) { return dtype == USP_BF16 ? 2 : dtype == USP_F32 ? 4 : 0; }
+
+// Shapes of the layout calls: B*S*H*D elements, S % 2P == 0, H % P_u == 0.
+int check_layout(const void* src, const void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r) {
+  if (!src || !dst) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(src) || !aligned16(dst)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (B <= 0 || S <= 0 || H <= 0 || D <= 0 || P_u <= 0 || P_r <= 0)
+    return fail(USP_ERR_INVALID_ARG, "sizes must be positive");
+  const int es = elem_size(dtype);
+  if (es == 0) return fail(USP_ERR_INVALID_ARG, "dtype must be USP_BF16 or USP_F32");
+  if ((static_cast<long long>(D) * es) % 4 != 0) return fail(USP_ERR_UNSUPPORTED, "D * element size must be a multiple of 4");
+  const long long P = static_cast<long long>(P_u) * P_r;
+  if (S % (2 * P) != 0) return fail(USP_ERR_UNSUPPORTED, "S (%d) must be a multiple of 2*P (%lld)", S, 2 * P);
+  if (H % P_u != 0) return fail(USP_ERR_UNSUPPORTED, "H (%d) must be a multiple of P_u (%d)", H, P_u);
+  if (static_cast<long long>(B) * S * P_u >= (1LL << 31)) return fail(USP_ERR_UNSUPPORTED, "too many rows");
+  if (static_cast<long long>(H) * D * es >= (1LL << 31)) return fail(USP_ERR_UNSUPPORTED, "token row too large");
+  return USP_OK;
+}
+
+int run_layout(int map, const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+               void* stream) {
+  int rc = check_layout(src, dst, B, S, H, D, dtype, P_u, P_r);
+  if (rc != USP_OK) return rc;
+  LayoutArgs a{};
+  a.src = static_cast<const uint8_t*>(src);
+  a.dst = static_cast<uint8_t*>(dst);
+  a.map = map;
+  a.B = B; a.S = S; a.H = H; a.P_u = P_u; a.P_r = P_r;
+  a.row_bytes = static_cast<uint32_t>(D * elem_size(dtype));
+  cudaError_t e = launch_layout(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "layout kernel launch");
+}
+
+int check_geom(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, AttnGeom* g) {
+  if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || P_u <= 0 || P_r <= 0)
+    return fail(USP_ERR_INVALID_ARG, "sizes must be positive");
+  if (causal != 0 && causal != 1) return fail(USP_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (D != 64 && D != 128) return fail(USP_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
+  if (Hq % Hkv != 0) return fail(USP_ERR_UNSUPPORTED, "Hq %% Hkv != 0");
+  if (Hq % P_u != 0 || Hkv % P_u != 0) return fail(USP_ERR_UNSUPPORTED, "Hq and Hkv must be multiples of P_u");
+  const long long P = static_cast<long long>(P_u) * P_r;
+  if (S % (2 * P) != 0) return fail(USP_ERR_UNSUPPORTED, "S (%d) must be a multiple of 2*P (%lld)", S, 2 * P);
+  if (static_cast<long long>(B) * S * Hq >= (1LL << 31)) return fail(USP_ERR_UNSUPPORTED, "too many rows");
+  g->B = B; g->S = S; g->Hq = Hq; g->Hkv = Hkv; g->D = D; g->causal = causal; g->P_u = P_u; g->P_r = P_r;
+  g->P = static_cast<int>(P);
+  g->c = S / (2 * g->P);
+  g->L = S / P_r;
+  g->Hq_l = Hq / P_u;
+  g->Hkv_l = Hkv / P_u;
+  g->G = Hq / Hkv;
+  g->n_ranks = P_r * P_u;
+  return USP_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q{};
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Head-sharded bf16 tensor [n_rb][L][H_l][D] viewed as 4-D {D, H_l, L, n_rb};
+// box = 64 elements (128 B, one swizzle panel) x 1 head x 128 rows x 1.
+int make_tmap(CUtensorMap* m, const void* base, int D, int H_l, int L, int n_rb) {
+  auto fn = encode_fn();
+  if (!fn) return fail(USP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H_l), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(n_rb)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H_l) * D * 2,
+                           static_cast<cuuint64_t>(L) * H_l * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(USP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return USP_OK;
+}
+
+size_t rows_of(const AttnGeom& g) { return static_cast<size_t>(g.B) * g.S * g.Hq; }
+
+size_t fwd_ws(const AttnGeom& g, int mode) {
+  if (mode == USP_MODE_FUSED) return kStatusBytes;
+  return kStatusBytes + static_cast<size_t>(g.P_r) * rows_of(g) * (4 * static_cast<size_t>(g.D) + 4);
+}
+size_t bwd_ws(const AttnGeom& g) { return kStatusBytes + rows_of(g) * (4 * static_cast<size_t>(g.D) + 4); }
+
+}  // namespace
+
+extern "C" {
+
+int usp_version(void) { return 100; }
+
+const char* usp_last_error(void) { return g_err; }
+
+void usp_set_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns; }
+
+int usp_zigzag_shard(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                     void* stream) {
+  return run_layout(kZigzagShard, src, dst, B, S, H, D, dtype, P_u, P_r, stream);
+}
+int usp_zigzag_unshard(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                       void* stream) {
+  return run_layout(kZigzagUnshard, src, dst, B, S, H, D, dtype, P_u, P_r, stream);
+}
+int usp_seq2head_permute(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                         void* stream) {
+  return run_layout(kSeq2Head, src, dst, B, S, H, D, dtype, P_u, P_r, stream);
+}
+int usp_head2seq_permute(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
+                         void* stream) {
+  return run_layout(kHead2Seq, src, dst, B, S, H, D, dtype, P_u, P_r, stream);
+}
+
+size_t usp_attn_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, int mode,
+                               int bwd) {
+  AttnGeom g{};
+  if (check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g) != USP_OK) return 0;
+  if (bwd) return bwd_ws(g);
+  if (mode != USP_MODE_FUSED && mode != USP_MODE_STEPWISE) return 0;
+  return fwd_ws(g, mode);
+}
+
+int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
+                 int Hkv, int D, int causal, int P_u, int P_r, int mode, void* workspace, size_t ws_bytes,
+                 void* stream) {
+  AttnGeom g{};
+  int rc = check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
+  if (rc != USP_OK) return rc;
+  if (mode != USP_MODE_FUSED && mode != USP_MODE_STEPWISE) return fail(USP_ERR_INVALID_ARG, "bad mode %d", mode);
+  if (!q || !k || !v || !out || !lse) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t need = fwd_ws(g, mode);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return fail(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FwdLaunch L{};
+  L.g = g;
+  if ((rc = make_tmap(&L.tm_q, q, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L.tm_k, k, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L.tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  L.status = static_cast<int*>(workspace);
+  L.wait_ns = g_wait_ns;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  if (mode == USP_MODE_FUSED) {
+    L.out = out;
+    L.lse = lse;
+    L.step = -1;
+    e = launch_attn_fwd(L, st);
+    return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention forward launch");
+  }
+  const size_t rows = rows_of(g);
+  float* o_parts = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+  float* lse_parts = o_parts + static_cast<size_t>(P_r) * rows * D;
+  for (int t = 0; t < P_r; ++t) {
+    L.step = t;
+    L.o_part = o_parts + static_cast<size_t>(t) * rows * D;
+    L.lse_part = lse_parts + static_cast<size_t>(t) * rows;
+    e = launch_attn_fwd(L, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention forward (step) launch");
+  }
+  e = launch_lse_merge(o_parts, lse_parts, P_r, static_cast<long long>(rows), D, out, 0, lse, st);
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "merge launch");
+}
+
+int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dO,
+                 void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D, int causal, int P_u,
+                 int P_r, void* workspace, size_t ws_bytes, void* stream) {
+  AttnGeom g{};
+  int rc = check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
+  if (rc != USP_OK) return rc;
+  if (!q || !k || !v || !out || !lse || !dO || !dQ || !dK || !dV) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t need = bwd_ws(g);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return fail(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t rows = rows_of(g);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+  float* delta = dq_acc + rows * D;
+  BwdLaunch L{};
+  L.g = g;
+  if ((rc = make_tmap(&L.tm_q, q, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L.tm_k, k, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L.tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L.tm_do, dO, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  L.lse = lse;
+  L.delta = delta;
+  L.dq_acc = dq_acc;
+  L.dk = dK;
+  L.dv = dV;
+  L.status = static_cast<int*>(workspace);
+  L.wait_ns = g_wait_ns;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dq_acc, 0, rows * D * sizeof(float), st);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+  e = launch_bwd_preprocess(out, dO, delta, static_cast<long long>(rows), D, st);
+  if (e != cudaSuccess) return cuda_fail(e, "preprocess launch");
+  e = launch_attn_bwd(L, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");
+  e = launch_f32_to_bf16(dq_acc, dQ, static_cast<long long>(rows) * D, st);
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "dQ conversion launch");
+}
+
+int usp_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,
+                  int out_dtype, float* lse_out, void* stream) {
+  if (!o_parts || !lse_parts || !out || !lse_out) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(o_parts) || !aligned16(out)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (n_parts <= 0 || rows < 0 || D <= 0) return fail(USP_ERR_INVALID_ARG, "sizes must be positive");
+  if (D % 4 != 0 || D > 256) return fail(USP_ERR_UNSUPPORTED, "D must be a multiple of 4, at most 256");
+  if (out_dtype != USP_BF16 && out_dtype != USP_F32) return fail(USP_ERR_INVALID_ARG, "bad out_dtype");
+  cudaError_t e = launch_lse_merge(o_parts, lse_parts, n_parts, rows, D, out, out_dtype == USP_F32, lse_out,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "merge launch");
+}
+
+int usp_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D, void* stream) {
+  if (!out || !dO || !delta) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(out) || !aligned16(dO)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (rows < 0 || D <= 0) return fail(USP_ERR_INVALID_ARG, "sizes must be positive");
+  if (D % 4 != 0) return fail(USP_ERR_UNSUPPORTED, "D must be a multiple of 4");
+  cudaError_t e = launch_bwd_preprocess(out, dO, delta, rows, D, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "preprocess launch");
+}
+
+int usp_workspace_status(void* workspace, int* site, void* stream) {
+  if (!workspace) return fail(USP_ERR_INVALID_ARG, "null workspace");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (site) *site = word;
+  if (word != 0) return fail(USP_ERR_TIMEOUT, "a device wait timed out (site 0x%x)", word);
+  return USP_OK;
+}
+
+int usp_selftest_wait_timeout(void* workspace, size_t ws_bytes, unsigned long long limit_ns, void* stream) {
+  if (!workspace || ws_bytes < static_cast<size_t>(kStatusBytes))
+    return fail(USP_ERR_WORKSPACE, "workspace needs %d bytes", kStatusBytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = launch_wait_selftest(static_cast<int*>(workspace), limit_ns, st);
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "self-test launch");
+}
+
+}  // extern "C"

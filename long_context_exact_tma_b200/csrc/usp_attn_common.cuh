@@ -1,0 +1,111 @@
+// usp_attn_common.cuh -- geometry shared by the attention kernels: original
+// token positions of the zigzag / Ulysses layout and the classification of a
+// (query tile, key tile) pair for the causal mask.
+//
+// Zigzag reading ("Boosting Spec Eagle", "Implementation Details": load
+// balancing across the ring): 2P chunks of c tokens, rank r holds chunks r and
+// 2P-1-r. After the Ulysses all-to-all (DeepSpeed-Ulysses summary, "Wie
+// DeepSpeed-Ulysses funktioniert"), ring rank i holds, for u' = 0..P_u-1, the
+// 2c tokens of rank i*P_u + u' in order: local token tau lies in local chunk
+// kappa = tau / c, which is chunk (kappa odd ? 2P-1-r' : r') with r' = i*P_u + kappa/2.
+#pragma once
+
+#include <climits>
+
+#include "usp_internal.h"
+
+namespace usp {
+
+constexpr int kBM = 128;  // query rows per tile (UMMA M)
+constexpr int kBN = 128;  // keys per tile
+
+struct Geo {
+  int B, L, Hq_l, Hkv_l, G, P_u, P_r, P, c, causal, n_ranks, n_qtiles, n_ktiles;
+  float scale_log2;  // softmax scale * log2(e)
+  float scale;       // softmax scale
+};
+
+inline Geo make_geo(const AttnGeom& a) {
+  Geo g{};
+  g.B = a.B; g.L = a.L; g.Hq_l = a.Hq_l; g.Hkv_l = a.Hkv_l; g.G = a.G; g.P_u = a.P_u; g.P_r = a.P_r;
+  g.P = a.P; g.c = a.c; g.causal = a.causal; g.n_ranks = a.n_ranks;
+  g.n_qtiles = (a.L + kBM - 1) / kBM;
+  g.n_ktiles = (a.L + kBN - 1) / kBN;
+  g.scale = 1.0f / sqrtf(static_cast<float>(a.D));
+  g.scale_log2 = g.scale * 1.4426950408889634f;
+  return g;
+}
+
+// Original token position of local token tau of ring rank i (tau < L).
+__device__ __forceinline__ int token_pos(const Geo& g, int i, int tau) {
+  const int kappa = tau / g.c;
+  const int rp = i * g.P_u + (kappa >> 1);
+  const int chunk = (kappa & 1) ? (2 * g.P - 1 - rp) : rp;
+  return chunk * g.c + (tau - kappa * g.c);
+}
+
+// Smallest and largest original position among local tokens [t0, t1) of ring rank i.
+__device__ __forceinline__ void pos_range(const Geo& g, int i, int t0, int t1, int& pmin, int& pmax) {
+  if (t1 > g.L) t1 = g.L;
+  pmin = INT_MAX;
+  pmax = -1;
+  for (int kap = t0 / g.c; kap * g.c < t1; ++kap) {
+    const int a = max(t0, kap * g.c);
+    const int e = min(t1, (kap + 1) * g.c) - 1;
+    pmin = min(pmin, token_pos(g, i, a));
+    pmax = max(pmax, token_pos(g, i, e));
+  }
+}
+
+enum TileKind { kSkip = 0, kFull = 1, kMasked = 2 };
+
+// Kind of the pair (query tile with positions [qmin, qmax], key tile n of ring rank j).
+__device__ __forceinline__ int classify_tile(const Geo& g, int qmin, int qmax, int j, int n) {
+  const int k0 = n * kBN;
+  const bool ragged = k0 + kBN > g.L;
+  if (!g.causal) return ragged ? kMasked : kFull;
+  int kmin, kmax;
+  pos_range(g, j, k0, k0 + kBN, kmin, kmax);
+  if (qmax < kmin) return kSkip;
+  if (qmin >= kmax && !ragged) return kFull;
+  return kMasked;
+}
+
+// Enumerates, in ring order, the non-skipped key tiles a query tile of ring
+// rank i attends: steps t in [t_begin, t_end), owner j = (i - t) mod P_r,
+// key tiles n = 0 .. n_ktiles-1 of rank j. Every role of a CTA walks the same
+// sequence.
+struct KvWalk {
+  int t, n, j, kind;
+  bool valid;
+};
+
+__device__ __forceinline__ void kv_walk_settle(const Geo& g, int i, int qmin, int qmax, int t_end, KvWalk& w) {
+  while (w.t < t_end) {
+    w.j = (i - w.t + g.P_r) % g.P_r;
+    while (w.n < g.n_ktiles) {
+      w.kind = classify_tile(g, qmin, qmax, w.j, w.n);
+      if (w.kind != kSkip) {
+        w.valid = true;
+        return;
+      }
+      ++w.n;
+    }
+    ++w.t;
+    w.n = 0;
+  }
+  w.valid = false;
+}
+
+__device__ __forceinline__ KvWalk kv_walk_begin(const Geo& g, int i, int qmin, int qmax, int t_begin, int t_end) {
+  KvWalk w{t_begin, 0, 0, 0, false};
+  kv_walk_settle(g, i, qmin, qmax, t_end, w);
+  return w;
+}
+
+__device__ __forceinline__ void kv_walk_next(const Geo& g, int i, int qmin, int qmax, int t_end, KvWalk& w) {
+  ++w.n;
+  kv_walk_settle(g, i, qmin, qmax, t_end, w);
+}
+
+}  // namespace usp

@@ -1,0 +1,166 @@
+// usp_elementwise.cu -- HBM-bound kernels around the attention kernels:
+//   * log-sum-exp merge of ring-step partials (per ring step each rank holds a
+//     partial (O_t, LSE_t) of its queries; "Boosting Spec Eagle", "The Solution",
+//     Ring Attention),
+//   * backward preprocess Delta_i = sum_d dO_id O_id,
+//   * fp32 -> bf16 conversion of the dQ accumulator,
+//   * the bounded-wait self-test kernel.
+#include <math.h>
+
+#include "usp_internal.h"
+#include "usp_ptx.cuh"
+
+namespace usp {
+namespace {
+
+// One warp per row; lane l handles elements 4l, 4l+1, 4l+2, 4l+3 (+128 per pass).
+template <bool kOutF32>
+__global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ o_parts,
+                                                        const float* __restrict__ lse_parts, int n_parts,
+                                                        long long rows, int D, void* __restrict__ out,
+                                                        float* __restrict__ lse_out) {
+  const int lane = threadIdx.x & 31;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += n_warps) {
+    float m = -INFINITY;
+    for (int t = 0; t < n_parts; ++t) m = fmaxf(m, __ldg(lse_parts + static_cast<long long>(t) * rows + r));
+    float lse = -INFINITY;
+    if (m != -INFINITY) {
+      float acc = 0.f;
+      for (int t = 0; t < n_parts; ++t) acc += expf(__ldg(lse_parts + static_cast<long long>(t) * rows + r) - m);
+      lse = m + logf(acc);
+    }
+    for (int d4 = lane; d4 * 4 < D; d4 += 32) {
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (lse != -INFINITY) {
+        for (int t = 0; t < n_parts; ++t) {
+          const float lt = __ldg(lse_parts + static_cast<long long>(t) * rows + r);
+          if (lt == -INFINITY) continue;
+          const float w = expf(lt - lse);
+          const float4 p = __ldcs(reinterpret_cast<const float4*>(o_parts + (static_cast<long long>(t) * rows + r) * D) + d4);
+          o.x += w * p.x;
+          o.y += w * p.y;
+          o.z += w * p.z;
+          o.w += w * p.w;
+        }
+      }
+      if (kOutF32) {
+        reinterpret_cast<float4*>(static_cast<float*>(out) + r * D)[d4] = o;
+      } else {
+        uint2 packed;
+        packed.x = pack_bf16x2(o.x, o.y);
+        packed.y = pack_bf16x2(o.z, o.w);
+        reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + r * D)[d4] = packed;
+      }
+    }
+    if (lane == 0) lse_out[r] = lse;
+  }
+}
+
+// One warp per row; 4 bf16 (8 bytes) per lane per pass.
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ out,
+                                                             const __nv_bfloat16* __restrict__ dO,
+                                                             float* __restrict__ delta, long long rows, int D) {
+  const int lane = threadIdx.x & 31;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += n_warps) {
+    float acc = 0.f;
+    for (int d4 = lane; d4 * 4 < D; d4 += 32) {
+      const uint2 a = __ldcs(reinterpret_cast<const uint2*>(out + r * D) + d4);
+      const uint2 b = __ldcs(reinterpret_cast<const uint2*>(dO + r * D) + d4);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float2 fa = __bfloat1622float2(a2[k]);
+        const float2 fb = __bfloat1622float2(b2[k]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) delta[r] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
+                                                          long long n4) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    const float4 v = __ldcs(src + i);
+    uint2 p;
+    p.x = pack_bf16x2(v.x, v.y);
+    p.y = pack_bf16x2(v.z, v.w);
+    __stcs(dst + i, p);
+  }
+}
+
+// Waits on an mbarrier that nothing completes; the bounded wait must give up.
+__global__ void wait_selftest_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  WaitCtl w{&abort_flag, status, limit_ns};
+  if (threadIdx.x == 0) {
+    if (!mbar_wait(&bar, 0, w, 0x7E57)) {
+      // expected path: the site code is in *status
+    }
+  }
+  __syncthreads();
+}
+
+unsigned grid_for(long long units_per_block, long long units) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long blocks = (units + units_per_block - 1) / units_per_block;
+  const long long cap = static_cast<long long>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return static_cast<unsigned>(blocks);
+}
+
+}  // namespace
+
+cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D,
+                             void* out, int out_f32, float* lse_out, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = grid_for(8, rows);
+  if (out_f32)
+    lse_merge_kernel<true><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, n_parts, rows, D, out, lse_out);
+  else
+    lse_merge_kernel<false><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, n_parts, rows, D, out, lse_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D,
+                                  cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  bwd_preprocess_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
+                                                               static_cast<const __nv_bfloat16*>(dO), delta,
+                                                               rows, D);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const long long n4 = n / 4;  // callers pass multiples of 4 (D is 64 or 128)
+  f32_to_bf16_kernel<<<grid_for(256, n4), 256, 0, stream>>>(reinterpret_cast<const float4*>(src),
+                                                            static_cast<uint2*>(dst), n4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace usp

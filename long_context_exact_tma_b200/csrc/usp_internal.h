@@ -1,0 +1,64 @@
+// usp_internal.h -- launch interfaces shared by the .cu files of libusp.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace usp {
+
+constexpr int kStatusBytes = 256;  // workspace header: device status word + padding
+
+// Layout maps of the gather kernel (see usp_layout.cu).
+enum LayoutMap { kZigzagShard = 0, kZigzagUnshard = 1, kSeq2Head = 2, kHead2Seq = 3 };
+
+struct LayoutArgs {
+  const uint8_t* src;
+  uint8_t* dst;
+  int map;
+  uint32_t B, S, H, P_u, P_r;  // tokens, heads, mesh
+  uint32_t row_bytes;          // bytes of one head row (D * element size)
+};
+cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t stream);
+
+cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D,
+                             void* out, int out_f32, float* lse_out, cudaStream_t stream);
+cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D,
+                                  cudaStream_t stream);
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t stream);
+cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
+
+// Geometry of one attention problem in the head-sharded layout.
+struct AttnGeom {
+  int B, S, Hq, Hkv, D, causal, P_u, P_r;
+  int P, c, L, Hq_l, Hkv_l, G;  // derived
+  int n_ranks;                  // P_r * P_u head-sharded ranks
+};
+
+struct FwdLaunch {
+  AttnGeom g;
+  CUtensorMap tm_q, tm_k, tm_v;
+  void* out;          // bf16 head-sharded (fused mode)
+  float* lse;         // fp32 [ranks][B][L][Hq_l] (fused mode)
+  float* o_part;      // fp32 partial O of one ring step (stepwise mode)
+  float* lse_part;    // fp32 partial LSE of one ring step (stepwise mode)
+  int step;           // ring step (stepwise) or -1 (fused)
+  int* status;
+  unsigned long long wait_ns;
+};
+cudaError_t launch_attn_fwd(const FwdLaunch& a, cudaStream_t stream);
+
+struct BwdLaunch {
+  AttnGeom g;
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  const float* lse;    // [ranks][B][L][Hq_l]
+  const float* delta;  // same layout
+  float* dq_acc;       // fp32, q layout
+  float* dk;           // fp32, k layout
+  float* dv;           // fp32, v layout
+  int* status;
+  unsigned long long wait_ns;
+};
+cudaError_t launch_attn_bwd(const BwdLaunch& a, cudaStream_t stream);
+
+}  // namespace usp

@@ -1,0 +1,128 @@
+"""The C ABI loads, exports every symbol include/usp.h declares, and rejects bad
+arguments with the documented status codes before launching anything.
+
+Only invalid arguments are passed here (rejected during validation), so these
+tests need no GPU and never hand a fake pointer to a kernel.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_exact_tma_b200 import binding as B_
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "usp.h")
+
+FAKE = 1 << 20  # 16-byte aligned, never dereferenced (validation fails first)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(usp_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B_.lib()
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B_.SIGNATURES), "binding must mirror the header"
+
+
+def test_version_and_empty_error():
+    assert B_.usp_version() >= 100
+    assert isinstance(B_.usp_last_error(), str)
+
+
+def test_workspace_size_queries():
+    ws = B_.usp_attn_workspace_size
+    assert ws(1, 256, 2, 2, 64, 1, 2, 2, 0, 0) == 256
+    rows = 1 * 256 * 2
+    assert ws(1, 256, 2, 2, 64, 1, 2, 2, 1, 0) == 256 + 2 * rows * (4 * 64 + 4)
+    assert ws(1, 256, 2, 2, 64, 1, 2, 2, 0, 1) == 256 + rows * (4 * 64 + 4)
+    assert ws(1, 256, 2, 2, 96, 1, 2, 2, 0, 0) == 0      # D unsupported
+    assert ws(1, 250, 2, 2, 64, 1, 2, 2, 0, 0) == 0      # S % 2P != 0
+    assert ws(1, 256, 3, 2, 64, 1, 1, 1, 0, 0) == 0      # Hq % Hkv != 0
+    assert ws(1, 256, 2, 1, 64, 1, 2, 1, 0, 0) == 0      # Hkv % P_u != 0
+    assert ws(1, 256, 2, 2, 64, 1, 1, 1, 7, 0) == 0      # bad mode
+
+
+def _fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, S=256, Hq=2, Hkv=2, D=64, causal=1, P_u=2,
+             P_r=2, mode=0, ws=FAKE, ws_bytes=256)
+    a.update(kw)
+    return B_.lib().usp_attn_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["S"], a["Hq"], a["Hkv"],
+                                 a["D"], a["causal"], a["P_u"], a["P_r"], a["mode"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), B_.USP_ERR_UNSUPPORTED),
+    (dict(D=256), B_.USP_ERR_UNSUPPORTED),
+    (dict(Hq=3), B_.USP_ERR_UNSUPPORTED),
+    (dict(Hkv=1), B_.USP_ERR_UNSUPPORTED),
+    (dict(S=250), B_.USP_ERR_UNSUPPORTED),
+    (dict(S=0), B_.USP_ERR_INVALID_ARG),
+    (dict(B=-1), B_.USP_ERR_INVALID_ARG),
+    (dict(causal=2), B_.USP_ERR_INVALID_ARG),
+    (dict(mode=5), B_.USP_ERR_INVALID_ARG),
+    (dict(q=None), B_.USP_ERR_INVALID_ARG),
+    (dict(lse=None), B_.USP_ERR_INVALID_ARG),
+    (dict(k=FAKE + 8), B_.USP_ERR_INVALID_ARG),
+    (dict(ws=None), B_.USP_ERR_WORKSPACE),
+    (dict(ws_bytes=255), B_.USP_ERR_WORKSPACE),
+    (dict(mode=1, ws_bytes=4096), B_.USP_ERR_WORKSPACE),
+])
+def test_fwd_rejects_bad_arguments(kw, code):
+    assert _fwd(**kw) == code
+    assert B_.usp_last_error() != ""
+
+
+def test_bwd_rejects_bad_arguments():
+    L = B_.lib()
+    args = [FAKE] * 9 + [1, 256, 2, 2, 64, 1, 2, 2, FAKE, 256, None]
+    assert L.usp_attn_bwd(*args) == B_.USP_ERR_WORKSPACE  # needs rows*(4D+4) bytes
+    bad = list(args)
+    bad[13] = 48  # D
+    assert L.usp_attn_bwd(*bad) == B_.USP_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[6] = None  # dQ
+    assert L.usp_attn_bwd(*bad) == B_.USP_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["usp_zigzag_shard", "usp_zigzag_unshard", "usp_seq2head_permute",
+                                  "usp_head2seq_permute"])
+def test_layout_rejects_bad_arguments(name):
+    fn = getattr(B_.lib(), name)
+    assert fn(FAKE, FAKE, 1, 250, 4, 64, 0, 2, 2, None) == B_.USP_ERR_UNSUPPORTED   # S % 2P
+    assert fn(FAKE, FAKE, 1, 256, 3, 64, 0, 2, 2, None) == B_.USP_ERR_UNSUPPORTED   # H % P_u
+    assert fn(FAKE, FAKE, 1, 256, 4, 1, 0, 2, 2, None) == B_.USP_ERR_UNSUPPORTED    # D*2 % 4
+    assert fn(FAKE, FAKE, 1, 256, 4, 64, 7, 2, 2, None) == B_.USP_ERR_INVALID_ARG   # dtype
+    assert fn(None, FAKE, 1, 256, 4, 64, 0, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+    assert fn(FAKE + 4, FAKE, 1, 256, 4, 64, 0, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+    assert fn(FAKE, FAKE, 0, 256, 4, 64, 0, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+
+
+def test_merge_and_preprocess_reject_bad_arguments():
+    L = B_.lib()
+    assert L.usp_lse_merge(FAKE, FAKE, 0, 10, 64, FAKE, 0, FAKE, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_lse_merge(FAKE, FAKE, 2, 10, 66, FAKE, 0, FAKE, None) == B_.USP_ERR_UNSUPPORTED
+    assert L.usp_lse_merge(FAKE, FAKE, 2, 10, 64, FAKE, 3, FAKE, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_lse_merge(None, FAKE, 2, 10, 64, FAKE, 0, FAKE, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_bwd_preprocess(FAKE, FAKE, None, 10, 64, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_bwd_preprocess(FAKE, FAKE, FAKE, 10, 6, None) == B_.USP_ERR_UNSUPPORTED
+    assert L.usp_workspace_status(None, None, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_selftest_wait_timeout(FAKE, 16, 1000, None) == B_.USP_ERR_WORKSPACE
+
+
+def test_product_package_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "long_context_exact_tma_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "usp_oracle" not in text and "liboracle" not in text, f
