@@ -101,7 +101,8 @@ int usp_head2seq_permute(const void* src, void* dst, int B, int S, int H, int D,
  * usp_attn_bwd (bwd = 1). Returns 0 for an unsupported shape.
  *   fused fwd   : 256 (status word)
  *   stepwise fwd: 256 + P_r * B*S*Hq * (4*D + 4)  (fp32 partials of every ring step)
- *   bwd         : 256 + B*S*Hq * (4*D + 4)        (fp32 dQ accumulator, Delta)
+ *   bwd         : 256 + B*S*Hq*4*D + 2 * 4 * B*P_u*P_r*(Hq/P_u)*Lp, Lp = S/P_r rounded up
+ *                 to a multiple of 128 (fp32 dQ accumulator; LSE*log2(e) and Delta per head)
  */
 size_t usp_attn_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, int mode,
                                int bwd);

@@ -122,7 +122,12 @@ size_t fwd_ws(const AttnGeom& g, int mode) {
   if (mode == USP_MODE_FUSED) return kStatusBytes;
   return kStatusBytes + static_cast<size_t>(g.P_r) * rows_of(g) * (4 * static_cast<size_t>(g.D) + 4);
 }
-size_t bwd_ws(const AttnGeom& g) { return kStatusBytes + rows_of(g) * (4 * static_cast<size_t>(g.D) + 4); }
+int padded_L(const AttnGeom& g) { return (g.L + 127) / 128 * 128; }
+// [status][dQ fp32 accumulator: rows*D][LSE*log2e per head: n_rb*Hq_l*Lp][Delta per head: same]
+size_t bwd_ws(const AttnGeom& g) {
+  const size_t per_head = static_cast<size_t>(g.n_ranks) * g.B * g.Hq_l * padded_L(g);
+  return kStatusBytes + rows_of(g) * 4 * static_cast<size_t>(g.D) + 2 * per_head * 4;
+}
 
 }  // namespace
 
@@ -219,16 +224,20 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
     return fail(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t rows = rows_of(g);
+  const int Lp = padded_L(g);
+  const size_t per_head = static_cast<size_t>(g.n_ranks) * B * g.Hq_l * Lp;
   float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
-  float* delta = dq_acc + rows * D;
+  float* lse2 = dq_acc + rows * D;
+  float* delta = lse2 + per_head;
   BwdLaunch L{};
   L.g = g;
   if ((rc = make_tmap(&L.tm_q, q, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   if ((rc = make_tmap(&L.tm_k, k, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   if ((rc = make_tmap(&L.tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   if ((rc = make_tmap(&L.tm_do, dO, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
-  L.lse = lse;
+  L.lse2 = lse2;
   L.delta = delta;
+  L.Lp = Lp;
   L.dq_acc = dq_acc;
   L.dk = dK;
   L.dv = dV;
@@ -237,7 +246,7 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(dq_acc, 0, rows * D * sizeof(float), st);
   if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
-  e = launch_bwd_preprocess(out, dO, delta, static_cast<long long>(rows), D, st);
+  e = launch_bwd_prep_rows(out, dO, lse, delta, lse2, g.n_ranks * B, g.L, g.Hq_l, D, Lp, st);
   if (e != cudaSuccess) return cuda_fail(e, "preprocess launch");
   e = launch_attn_bwd(L, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");

@@ -236,7 +236,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const int tau_q = q0 + row;
     const int pos_q = tau_q < g.L ? token_pos(g, i, tau_q) : INT_MAX;
     const bool aligned = (g.c % kBN) == 0;
-    float m_use = -INFINITY, l_run = 0.f;
+    // l_run: sum of the fp32 weights (for LSE); lb_run: sum of the bf16-rounded
+    // weights the PV UMMA consumes (normalises O, so O stays a convex combination
+    // of V rows even when one key dominates).
+    float m_use = -INFINITY, l_run = 0.f, lb_run = 0.f;
     KvWalk kw = kv_walk_begin(g, i, qmin, qmax, t_begin, t_end);
     int it = 0;
     bool ok = true;
@@ -300,6 +303,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         rs += s[c];
       }
       l_run = l_run * alpha + rs;
+      lb_run *= alpha;
       if (it >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (it - 1) & 1, w, kSiteO));
         if (!ok) break;
@@ -319,6 +323,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         }
       }
       // P (bf16) into the two 64-key swizzled panels, row = query row.
+      float rsb = 0.f;
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
         uint4 v;
@@ -326,8 +331,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         v.y = pack_bf16x2(s[ch * 8 + 2], s[ch * 8 + 3]);
         v.z = pack_bf16x2(s[ch * 8 + 4], s[ch * 8 + 5]);
         v.w = pack_bf16x2(s[ch * 8 + 6], s[ch * 8 + 7]);
+        rsb += bf16x2_sum(v.x) + bf16x2_sum(v.y) + bf16x2_sum(v.z) + bf16x2_sum(v.w);
         *reinterpret_cast<uint4*>(sP + (ch >> 3) * C::kPanelBytes + sw128_offset(row, ch & 7)) = v;
       }
+      lb_run += rsb;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->p_full);
@@ -338,7 +345,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       tc_fence_after();
       const bool store = tau_q < g.L;
       const size_t row_idx = (static_cast<size_t>(rank * g.B + b) * g.L + (store ? tau_q : 0)) * g.Hq_l + h;
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv_l = lb_run > 0.f ? 1.f / lb_run : 0.f;
       const float lse_val = l_run > 0.f ? (m_use + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {

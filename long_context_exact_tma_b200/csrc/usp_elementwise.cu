@@ -86,6 +86,42 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
   }
 }
 
+// Delta and LSE*log2(e) of every row, written per head: row (rb, tau, h) of the
+// head-sharded layout goes to [rb*Hl + h][tau] of a [n_rb*Hl][Lp] table.
+__global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16* __restrict__ out,
+                                                            const __nv_bfloat16* __restrict__ dO,
+                                                            const float* __restrict__ lse,
+                                                            float* __restrict__ delta_t, float* __restrict__ lse2_t,
+                                                            long long rows, int L, int Hl, int D, int Lp) {
+  const int lane = threadIdx.x & 31;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += n_warps) {
+    float acc = 0.f;
+    for (int d4 = lane; d4 * 4 < D; d4 += 32) {
+      const uint2 x = __ldcs(reinterpret_cast<const uint2*>(out + r * D) + d4);
+      const uint2 y = __ldcs(reinterpret_cast<const uint2*>(dO + r * D) + d4);
+      const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+      const __nv_bfloat162* y2 = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float2 fx = __bfloat1622float2(x2[k]);
+        const float2 fy = __bfloat1622float2(y2[k]);
+        acc = fmaf(fx.x, fy.x, acc);
+        acc = fmaf(fx.y, fy.y, acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const long long h = r % Hl, rt = r / Hl, tau = rt % L, rb = rt / L;
+      const long long dst = (rb * Hl + h) * Lp + tau;
+      delta_t[dst] = acc;
+      lse2_t[dst] = lse[r] * 1.4426950408889634f;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
                                                           long long n4) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -147,6 +183,16 @@ cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta,
   bwd_preprocess_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
                                                                static_cast<const __nv_bfloat16*>(dO), delta,
                                                                rows, D);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* lse, float* delta_t, float* lse2_t,
+                                 int n_rb, int L, int Hl, int D, int Lp, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(n_rb) * L * Hl;
+  if (rows == 0) return cudaSuccess;
+  bwd_prep_rows_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
+                                                              static_cast<const __nv_bfloat16*>(dO), lse, delta_t,
+                                                              lse2_t, rows, L, Hl, D, Lp);
   return cudaGetLastError();
 }
 

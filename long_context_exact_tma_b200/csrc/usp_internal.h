@@ -48,11 +48,17 @@ struct FwdLaunch {
 };
 cudaError_t launch_attn_fwd(const FwdLaunch& a, cudaStream_t stream);
 
+// Backward preprocess into the per-head layout the backward kernel streams:
+// delta_t/lse2_t [n_ranks*B*Hq_l][Lp] (Lp = L rounded up to 128), lse2 = LSE*log2(e).
+cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* lse, float* delta_t, float* lse2_t,
+                                 int n_rb, int L, int Hl, int D, int Lp, cudaStream_t stream);
+
 struct BwdLaunch {
   AttnGeom g;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
-  const float* lse;    // [ranks][B][L][Hq_l]
-  const float* delta;  // same layout
+  const float* lse2;   // [n_ranks*B*Hq_l][Lp]
+  const float* delta;  // [n_ranks*B*Hq_l][Lp]
+  int Lp;
   float* dq_acc;       // fp32, q layout
   float* dk;           // fp32, k layout
   float* dv;           // fp32, v layout

@@ -217,6 +217,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Sum of the two bf16 values packed in w, in fp32 (exact widening).
+__device__ __forceinline__ float bf16x2_sum(uint32_t w) {
+  return __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte
 // swizzled tile whose 8-row atoms are 1024-byte aligned.
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {

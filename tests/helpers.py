@@ -79,11 +79,22 @@ def compare_fwd(o_gpu, lse_gpu, tensors, spec, rows=None):
     l_g = lse_gpu.float().numpy()[idx[:, 0], idx[:, 2], idx[:, 1]].astype(np.float64)
     err = np.abs(o_g - o_ref)
     lerr = np.abs(l_g - lse_ref)
-    return dict(o_max=float(err.max()), o_mean=float(err.mean()), lse_max=float(lerr.max()))
+    # O is delivered in bf16: its final rounding alone may move a value by half a
+    # bf16 ulp of the reference (2^-9 relative), which exceeds 1e-2 once |O| > 2.6.
+    # The max-abs bound applies to the error beyond that rounding.
+    excess = np.maximum(err - half_ulp_bf16(o_ref), 0.0)
+    return dict(o_max=float(err.max()), o_max_excess=float(excess.max()), o_mean=float(err.mean()),
+                lse_max=float(lerr.max()))
+
+
+def half_ulp_bf16(x):
+    """Half the bf16 spacing at |x| (bf16 keeps 8 significant bits)."""
+    ax = np.maximum(np.abs(np.asarray(x, np.float64)), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(ax)) - 8)
 
 
 def assert_fwd_ok(stats):
-    assert stats["o_max"] <= O_MAX_ABS, stats
+    assert stats["o_max_excess"] <= O_MAX_ABS, stats
     assert stats["o_mean"] <= O_MEAN_ABS, stats
     assert stats["lse_max"] <= LSE_MAX_ABS, stats
 
