@@ -1,0 +1,412 @@
+"""Benchmark of the USP attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+
+One step = one pass of the whole per-rank hot path over one batch, with the
+inputs already sharded the way the ranks hold them (zigzag, rank-major):
+  seq->head all-to-all of Q, K, V  ->  attention forward (ring steps merged
+  in-kernel)  ->  head->seq of O  ->  seq->head of dO  ->  attention backward
+  (preprocess, blockwise dQ/dK/dV)  ->  head->seq of dQ, dK, dV.
+Every step runs in libusp.so kernels through the C ABI. The metric is the
+algorithmic attention FLOPs of forward + backward (fwd = 4*B*Hq*S^2*D, x1/2
+when causal; bwd = 2.5 x fwd) per second of step time, for the whole job.
+
+Default workload: the S=16384 causal configuration (B=1, H=32, D=128, ring of
+8 zigzag chunks), forward and backward. --config picks another workload.
+With --gpus N (under torchrun) every rank runs its own independent batch
+(weak scaling; no collective on the data path), timing is the max over ranks.
+--impl reference times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from usp_inputs import WORKLOADS, workload  # noqa: E402
+
+METRIC = "attention TFLOP/s fwd+bwd at S=16K-256K; % of bf16 dense tensor peak"
+UNIT = "TFLOP/s"
+LAUNCHES_PER_STEP = 12  # 3 seq2head + fwd + head2seq(O) + seq2head(dO) + prep + bwd + dQ convert + 3 head2seq
+
+
+def flops_fwd(w) -> float:
+    return 4.0 * w["B"] * w["Hq"] * w["S"] * w["S"] * w["D"] * (0.5 if w["causal"] else 1.0)
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        return summarize_clock_lines(self.lines)
+
+
+def summarize_clock_lines(lines):
+    """Median SM clock, max clock and the throttle reasons seen in nvidia-smi CSV lines."""
+    sm, mx, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 7:
+            continue
+        try:
+            sm.append(float(parts[0]))
+            mx.append(float(parts[1]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[3:7]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+def setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Largest value over the ranks (timing only; the data path has no collective)."""
+    if world == 1:
+        return x
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------- our implementation
+class Step:
+    """Buffers and the launch sequence of one step of the hot path on one GPU."""
+
+    def __init__(self, w, dev, seed_offset=0):
+        from long_context_exact_tma_b200 import api
+        from long_context_exact_tma_b200 import binding as B_
+        self.api, self.B_ = api, B_
+        self.w = w
+        B, S, Hq, Hkv, D = w["B"], w["S"], w["Hq"], w["Hkv"], w["D"]
+        P_u, P_r = w["P_u"], w["P_r"]
+        P = P_u * P_r
+        spec = dict(w)
+        spec["seed"] = w["seed"] + seed_offset
+        t = workload(spec, device=dev, which=("q", "k", "v", "do"))
+        # inputs as the ranks hold them: zigzag-sharded, rank-major
+        self.rm = {n: api.zigzag_shard(t[n], P_u, P_r) for n in ("q", "k", "v", "do")}
+        del t
+        L = S // P_r
+        bf = torch.bfloat16
+        self.hs = {"q": torch.empty((P_r, P_u, B, L, Hq // P_u, D), dtype=bf, device=dev),
+                   "k": torch.empty((P_r, P_u, B, L, Hkv // P_u, D), dtype=bf, device=dev),
+                   "v": torch.empty((P_r, P_u, B, L, Hkv // P_u, D), dtype=bf, device=dev),
+                   "do": torch.empty((P_r, P_u, B, L, Hq // P_u, D), dtype=bf, device=dev)}
+        self.out = torch.empty_like(self.hs["q"])
+        self.lse = torch.empty(self.hs["q"].shape[:-1], dtype=torch.float32, device=dev)
+        self.dq = torch.empty_like(self.hs["q"])
+        self.dk = torch.empty(self.hs["k"].shape, dtype=torch.float32, device=dev)
+        self.dv = torch.empty(self.hs["v"].shape, dtype=torch.float32, device=dev)
+        self.o_rm = torch.empty((P, B, S // P, Hq, D), dtype=bf, device=dev)
+        self.dq_rm = torch.empty_like(self.o_rm)
+        self.dk_rm = torch.empty((P, B, S // P, Hkv, D), dtype=torch.float32, device=dev)
+        self.dv_rm = torch.empty_like(self.dk_rm)
+        self.ws_f = api.workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, w["causal"], P_u, P_r, 0, 0), dev)
+        self.ws_b = api.workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, w["causal"], P_u, P_r, 0, 1), dev)
+        self.stream = torch.cuda.current_stream()
+
+    def run(self, ev=None):
+        """One step; ev = (start, end) event pairs per timed call, or None."""
+        api, w = self.api, self.w
+        P_u, P_r, causal = w["P_u"], w["P_r"], w["causal"]
+        st = self.stream
+        for n in ("q", "k", "v"):
+            api.seq2head(self.rm[n], P_u, P_r, out=self.hs[n])
+        if ev:
+            ev["fwd"][0].record(st)
+        api.attn_fwd(self.hs["q"], self.hs["k"], self.hs["v"], causal, P_u, P_r, ws=self.ws_f, out=self.out,
+                     lse=self.lse)
+        if ev:
+            ev["fwd"][1].record(st)
+        api.head2seq(self.out, P_u, P_r, out=self.o_rm)
+        api.seq2head(self.rm["do"], P_u, P_r, out=self.hs["do"])
+        if ev:
+            ev["bwd"][0].record(st)
+        api.attn_bwd(self.hs["q"], self.hs["k"], self.hs["v"], self.out, self.lse, self.hs["do"], causal, P_u, P_r,
+                     ws=self.ws_b, dq=self.dq, dk=self.dk, dv=self.dv)
+        if ev:
+            ev["bwd"][1].record(st)
+        api.head2seq(self.dq, P_u, P_r, out=self.dq_rm)
+        api.head2seq(self.dk, P_u, P_r, out=self.dk_rm)
+        api.head2seq(self.dv, P_u, P_r, out=self.dv_rm)
+
+    def check_status(self):
+        for ws in (self.ws_f, self.ws_b):
+            rc, site = self.B_.usp_workspace_status(ws)
+            if rc != 0:
+                raise RuntimeError(f"device wait timed out (site {site:#x})")
+
+    def host_io(self):
+        """Pinned host buffers for the end-to-end measurement."""
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
+        self.h_in = {n: pin(self.rm[n]) for n in self.rm}
+        for n in self.rm:
+            self.h_in[n].copy_(self.rm[n])
+        self.h_out = [pin(self.o_rm), pin(self.dq_rm), pin(self.dk_rm), pin(self.dv_rm)]
+        h2d = sum(t.numel() * t.element_size() for t in self.h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+        return h2d, d2h
+
+    def run_e2e(self):
+        for n in self.rm:
+            self.rm[n].copy_(self.h_in[n], non_blocking=True)
+        self.run()
+        for h, d in zip(self.h_out, (self.o_rm, self.dq_rm, self.dk_rm, self.dv_rm)):
+            h.copy_(d, non_blocking=True)
+
+
+def cpu_baseline_sample(w, seconds=10.0, seed=0):
+    """Time the fp64 oracle (forward + dQ rows) on a bounded sample of the workload.
+
+    Returns (tflops, n_rows, elapsed, threads). Each sampled query row is credited
+    with the algorithmic FLOPs the oracle performs for it: 8*D per visible key
+    (QK^T and PV of the forward, dP and dQ of the backward).
+    """
+    import numpy as np
+
+    import oracle
+    t = workload(dict(w), device="cuda", which=("q", "k", "v", "do"))
+    tc = {n: t[n].cpu() for n in ("q", "k", "v", "do")}
+    del t
+    rng = np.random.default_rng(seed)
+    B, S, Hq, D = w["B"], w["S"], w["Hq"], w["D"]
+
+    def rows_of(n):
+        return [(int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(S))) for _ in range(n)]
+
+    def vis(rows):
+        return sum((i + 1) if w["causal"] else S for _, _, i in rows)
+
+    probe = rows_of(32)
+    t0 = time.perf_counter()
+    oracle.attn_dq_rows(tc["q"], tc["k"], tc["v"], tc["do"], w["causal"], probe)
+    per_row = max((time.perf_counter() - t0) / len(probe), 1e-6)
+    n = int(min(max(32, seconds / per_row), 200000))
+    rows = rows_of(n)
+    t0 = time.perf_counter()
+    oracle.attn_dq_rows(tc["q"], tc["k"], tc["v"], tc["do"], w["causal"], rows)
+    el = time.perf_counter() - t0
+    fl = 8.0 * D * vis(rows)
+    return fl / el / 1e12, n, el, oracle.max_threads()
+
+
+def bench_ours(args, w, world, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    step = Step(w, dev, seed_offset=1000 * rank)
+    peak_tf, peak_hbm, peak_src = read_peaks()
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    step.check_status()
+    ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] for k in ("fwd", "bwd")}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(local) as clk:
+        start.record()
+        for s in range(args.steps):
+            step.run({k: ev[k][s] for k in ev})
+        end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    step.check_status()
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world)
+    f_fwd = flops_fwd(w)
+    f_step = 3.5 * f_fwd
+    value = world * args.steps * f_step / (ms / 1e3) / 1e12
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["fwd"])
+    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["bwd"])
+    # end to end: host buffers in, host buffers out, through the same C ABI calls
+    h2d, d2h = step.host_io()
+    for _ in range(2):
+        step.run_e2e()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record()
+    for _ in range(args.steps):
+        step.run_e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = world * args.steps * f_step / (e2e_ms / 1e3) / 1e12
+    if rank != 0:
+        return None
+    bwd_tf = 2.5 * f_fwd / (bwd_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 + Box-Muller N(0,1), rounded to bf16)",
+        "config": {"workload": w["name"], "B": w["B"], "S": w["S"], "Hq": w["Hq"], "Hkv": w["Hkv"],
+                   "D": w["D"], "causal": bool(w["causal"]), "P_ulysses": w["P_u"], "P_ring": w["P_r"],
+                   "global_batch": w["B"] * world, "seq_len": w["S"],
+                   "parallelism": f"{world} independent replicas x (USP {w['P_u']}x{w['P_r']} virtual ranks)",
+                   "l2": "inputs larger than L2 (Q, K, V, dO 134 MB each)"},
+        "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
+        "fwd_tflops": round(f_fwd / (fwd_ms / 1e3) / 1e12, 2),
+        "bwd_tflops": round(bwd_tf, 2),
+        "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel<128> (usp_attn_bwd call)",
+                     "achieved": round(bwd_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(bwd_tf / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "traffic": None},
+        "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tf, n, el, thr = cpu_baseline_sample(w, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(tf, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
+                                "sample": f"fp64 oracle forward + dQ on {n} seeded query rows of {w['name']} "
+                                          f"({el:.1f} s), credited 8*D FLOPs per visible key"}
+    return line
+
+
+def bench_reference(args, w, world, rank):
+    """The oracle as the reference arm: each step a bounded sample, timed on the host cores."""
+    if rank != 0:
+        return None
+    samples = []
+    for _ in range(args.warmup):
+        cpu_baseline_sample(w, seconds=args.ref_seconds, seed=7)
+    tot_fl, tot_s, rows, thr = 0.0, 0.0, 0, 1
+    for s in range(args.steps):
+        tf, n, el, thr = cpu_baseline_sample(w, seconds=args.ref_seconds, seed=100 + s)
+        samples.append(tf)
+        tot_fl += tf * 1e12 * el
+        tot_s += el
+        rows += n
+    value = tot_fl / tot_s / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w["name"], "B": w["B"], "S": w["S"], "Hq": w["Hq"], "Hkv": w["Hkv"],
+                   "D": w["D"], "causal": bool(w["causal"]), "P_ulysses": w["P_u"], "P_ring": w["P_r"],
+                   "global_batch": w["B"], "seq_len": w["S"]},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"{rows} seeded query rows over {args.steps} steps (forward + dQ rows)"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--config", type=int, default=2, help="workload number (1-5), default the S=16K one")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=5.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: warmup raised to the minimum of 3", file=sys.stderr)
+        args.warmup = 3
+    w = dict(WORKLOADS[args.config])
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; other ranks have nothing to do
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        line = bench_reference(args, w, int(os.environ.get("WORLD_SIZE", "1")), 0)
+        print(json.dumps(line), flush=True)
+        return
+    world, rank, local = setup_dist(args)
+    try:
+        line = bench_ours(args, w, world, rank, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
