@@ -143,6 +143,39 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
                  int P_r, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Bytes of the static device scratch behind usp_attn_bwd_noalloc (32 MiB).
+ */
+#define USP_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * usp_attn_bwd without a workspace argument. The paper has no counterpart:
+ * this is a convenience of this library for callers that cannot allocate
+ * device memory for a workspace, such as code running while a framework's
+ * caching allocator or a pool reserved at start-up owns the device memory
+ * (a cudaMalloc behind its back can fail or fragment it), or serving loops
+ * that must not allocate after initialisation (cudaMalloc can synchronise the
+ * device).
+ *
+ * Arguments and results are those of usp_attn_bwd. The scratch (status word,
+ * fp32 dQ accumulator, per-head LSE and Delta tables) is a file-scope static
+ * __device__ array of USP_NOALLOC_SCRATCH_BYTES bytes, which every GPU that
+ * loads this part of the library holds until the process exits. A problem
+ * whose usp_attn_workspace_size(..., bwd=1) exceeds that size is rejected with
+ * USP_ERR_WORKSPACE before anything is launched. The call allocates nothing:
+ * no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, which may load the library's device code); make that
+ * first call before any stream capture. Every call shares the one array and
+ * clears the parts that must start at zero; calls whose work overlaps on the
+ * GPU (other streams, other threads) race on it and must be serialised by the
+ * caller.
+ */
+int usp_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                         const void* dO, void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D,
+                         int causal, int P_u, int P_r, void* stream);
+
+/*
  * Log-sum-exp merge of n_parts ring-step partials (the partial results each
  * ring step produces, "Boosting Spec Eagle", "The Solution"):
  *   LSE = m + log sum_t exp(LSE_t - m),  m = max_t LSE_t

@@ -131,6 +131,17 @@ size_t bwd_ws(const AttnGeom& g) {
 
 }  // namespace
 
+namespace usp {
+// Records `msg` as this thread's last error and returns `code` (for entry points in other files).
+int record_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+}  // namespace usp
+
 extern "C" {
 
 int usp_version(void) { return 100; }

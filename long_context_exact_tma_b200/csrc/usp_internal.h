@@ -9,6 +9,9 @@ namespace usp {
 
 constexpr int kStatusBytes = 256;  // workspace header: device status word + padding
 
+// Sets the calling thread's usp_last_error() message; returns `code`.
+int record_error(int code, const char* fmt, ...);
+
 // Layout maps of the gather kernel (see usp_layout.cu).
 enum LayoutMap { kZigzagShard = 0, kZigzagUnshard = 1, kSeq2Head = 2, kHead2Seq = 3 };
 

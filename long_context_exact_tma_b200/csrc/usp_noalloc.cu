@@ -1,0 +1,56 @@
+// usp_noalloc.cu -- usp_attn_bwd_noalloc: the attention backward for callers
+// that cannot allocate a workspace. Its scratch is a static device array of
+// this file; the call runs the regular usp_attn_bwd path on that array.
+#include <stddef.h>
+
+#include <mutex>
+
+#include "../../include/usp.h"
+#include "usp_internal.h"
+
+namespace {
+
+// The scratch itself. Host code must not use this name as an address: on the
+// host it is only a stand-in for the device symbol, so the device address is
+// looked up with cudaGetSymbolAddress once per device (below).
+__device__ __align__(256) unsigned char g_bwd_scratch[USP_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" int usp_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                                    const void* dO, void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv,
+                                    int D, int causal, int P_u, int P_r, void* stream) {
+  const size_t need = usp_attn_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, USP_MODE_FUSED, 1);
+  if (need == 0)  // a shape the backward does not support: the regular entry point reports why
+    return usp_attn_bwd(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, nullptr, 0, stream);
+  if (need > USP_NOALLOC_SCRATCH_BYTES)
+    return usp::record_error(USP_ERR_WORKSPACE,
+                             "usp_attn_bwd_noalloc: this problem needs %zu bytes of scratch but the static scratch "
+                             "holds %zu; call usp_attn_bwd with a workspace instead",
+                             need, static_cast<size_t>(USP_NOALLOC_SCRATCH_BYTES));
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return usp::record_error(USP_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return usp::record_error(USP_ERR_UNSUPPORTED, "usp_attn_bwd_noalloc: device index %d >= %d", dev, kMaxDevices);
+  void* scratch = nullptr;
+  {
+    // Set-up, once per device, with that device current.
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+      if (e != cudaSuccess || p == nullptr)
+        return usp::record_error(USP_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+      g_scratch_addr[dev] = p;
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  // usp_attn_bwd clears the status word and the dQ accumulator before its kernels run.
+  return usp_attn_bwd(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, scratch,
+                      USP_NOALLOC_SCRATCH_BYTES, stream);
+}
