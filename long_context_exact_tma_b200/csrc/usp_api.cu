@@ -116,6 +116,24 @@ int make_tmap(CUtensorMap* m, const void* base, int D, int H_l, int L, int n_rb)
   return USP_OK;
 }
 
+// fp32 dQ accumulator [n_rb][L][H_l][D] as 4-D {D, H_l, L, n_rb}; box = 32 fp32 (128 B) x 1 x 32 rows x 1,
+// 128-byte swizzle (the staging layout of the backward's reduce-add).
+int make_tmap_dq(CUtensorMap* m, const void* base, int D, int H_l, int L, int n_rb) {
+  auto fn = encode_fn();
+  if (!fn) return fail(USP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H_l), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(n_rb)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(H_l) * D * 4,
+                           static_cast<cuuint64_t>(L) * H_l * D * 4};
+  cuuint32_t box[4] = {32, 1, 32, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(USP_ERR_CUDA, "cuTensorMapEncodeTiled (dQ) failed (%d)", static_cast<int>(r));
+  return USP_OK;
+}
+
 size_t rows_of(const AttnGeom& g) { return static_cast<size_t>(g.B) * g.S * g.Hq; }
 
 size_t fwd_ws(const AttnGeom& g, int mode) {
@@ -246,6 +264,7 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   if ((rc = make_tmap(&L.tm_k, k, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   if ((rc = make_tmap(&L.tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   if ((rc = make_tmap(&L.tm_do, dO, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap_dq(&L.tm_dq, dq_acc, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   L.lse2 = lse2;
   L.delta = delta;
   L.Lp = Lp;

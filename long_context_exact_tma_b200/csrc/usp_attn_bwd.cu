@@ -8,21 +8,25 @@
 // with dK/dV summed over the q-heads of a GQA group and over every ring rank's
 // queries (in the ring algorithm dK/dV travel around the ring with K/V).
 //
-// CTA = one 128-key tile of one kv-head of one head-sharded rank (i.e. the
-// ring's KV chunk owner). It loops over the q-heads of the group, the ring
-// ranks whose queries see the tile, and their 128-row query tiles:
-//   warp 0      TMA: K, V once; per step Q, dO tiles and the 128 LSE/Delta values.
-//   warp 1      TMEM allocator + UMMA issuer:
-//                 S^T  = K Q^T        -> TMEM [0,128)      (M = keys, N = queries)
-//                 dP^T = V dO^T       -> TMEM [128,256)
-//                 dV  += P^T dO       -> TMEM [256,256+D)  (A = P^T from shared memory)
-//                 dK  += dS^T Q       -> TMEM [384,384+D)  (A = dS^T from shared memory)
-//                 dQt  = dS K         -> TMEM [0, D)       (A = dS, MN-major view of dS^T)
-//   warps 2..5  thread = key row: P^T and dS^T rows from S^T/dP^T (tcgen05.ld),
-//               written bf16 into 128B-swizzled shared memory; then thread =
-//               query row: the dQ tile is read from TMEM and added to the fp32
-//               dQ accumulator in global memory with vector atomics. At the end
-//               dK and dV rows (fp32) are written out.
+// CTA = one 128-key tile of one kv-head of one head-sharded rank (the ring's KV
+// chunk owner); it walks the q-heads of the group, the ring ranks whose queries
+// see the tile and their 128-row query tiles ("steps"). 320 threads:
+//   warp 0      TMA: K, V once; per step Q, dO (2 stages) and 128 LSE/Delta values.
+//   warp 1      TMEM allocator + UMMA issuer, per step k:
+//                 S^T  = K Q^T      -> TMEM [0,128)     (M = keys, N = queries)
+//                 dP^T = V dO^T     -> TMEM [128,256)
+//                 dV  += P^T dO     -> TMEM [256,256+D) (A = P^T read from TMEM)
+//                 dK  += dS^T Q     -> TMEM [384,384+D) (A = dS^T from shared memory)
+//                 dQt  = dS K       -> TMEM [128,128+D) (A = dS: MN-major view of dS^T)
+//               S^T of step k+1 is issued once step k's UMMAs have completed and
+//               dP^T of step k+1 once the dQ tile of step k has been read out.
+//   warps 2..9  two warpgroups; warpgroup c owns query columns [64c, 64c+64).
+//               Thread = key row: P^T (bf16, packed back into TMEM over the S^T
+//               columns it has read) and dS^T (bf16, 128B-swizzled shared memory).
+//               Then thread = query row: the dQ tile is read from TMEM, staged in
+//               the step's (now free) Q/dO buffers and added to the fp32 dQ
+//               accumulator with TMA bulk reduce-add (cp.reduce.async.bulk.tensor).
+//               At the end dK and dV rows (fp32) are written out.
 // Every wait is bounded (usp_ptx.cuh).
 #include <math.h>
 
@@ -33,25 +37,28 @@
 namespace usp {
 namespace {
 
-constexpr int kThreadsBwd = 192;
+constexpr int kThreadsBwd = 320;
+constexpr int kComputeThreads = 256;
 constexpr uint32_t kTmemColsBwd = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+constexpr uint32_t kColDQ = kColDP;  // the dQ tile reuses the dP^T columns
 
 template <int D>
 struct BwdCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = 128 * 128;
   static constexpr int kTileBytes = kPanels * kPanelBytes;
-  static constexpr int kStages = D == 128 ? 1 : 2;
+  static constexpr int kStages = 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;
   static constexpr int kOffDO = kOffQ + kStages * kTileBytes;
-  static constexpr int kOffPt = kOffDO + kStages * kTileBytes;  // P^T: 128 keys x 128 queries bf16
-  static constexpr int kOffDSt = kOffPt + 2 * kPanelBytes;      // dS^T
-  static constexpr int kOffRow = kOffDSt + 2 * kPanelBytes;     // per stage: LSE*log2e [128], Delta [128]
+  static constexpr int kOffDSt = kOffDO + kStages * kTileBytes;  // dS^T: 128 keys x 128 queries bf16
+  static constexpr int kOffRow = kOffDSt + 2 * kPanelBytes;      // per stage: LSE*log2e [128], Delta [128]
   static constexpr int kOffBar = kOffRow + kStages * 1024;
-  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+  // No alignment slack: the kernel requires (and checks) a 1024-byte aligned dynamic shared memory base.
+  static constexpr int kSmemBytes = kOffBar + 256;
+  static constexpr int kBoxesPerWarp = D / 64;  // 32x32 fp32 dQ boxes one compute warp stages per step
 };
 
 struct BwdArgs {
@@ -59,7 +66,6 @@ struct BwdArgs {
   const float* lse2;   // [n_ranks*B*Hq_l][Lp]: LSE * log2(e)
   const float* delta;  // [n_ranks*B*Hq_l][Lp]
   int Lp;
-  float* dq_acc;       // fp32 [n_ranks][B][L][Hq_l][D]
   float* dk;           // fp32 [n_ranks][B][L][Hkv_l][D]
   float* dv;
   int* status;
@@ -76,7 +82,7 @@ struct BwdBars {
 
 enum : int {
   kSiteBKv = 0x201, kSiteBQdEmpty = 0x202, kSiteBQd = 0x211, kSiteBDqFree = 0x212, kSiteBP = 0x213,
-  kSiteBSt = 0x221, kSiteBDq = 0x222, kSiteBQdC = 0x223
+  kSiteBDqOwn = 0x214, kSiteBSt = 0x221, kSiteBDq = 0x222, kSiteBQdC = 0x223, kSiteBAlign = 0x2FF
 };
 
 // Query steps of one key tile: q-head hh of the group, ring rank i, query tile m.
@@ -127,43 +133,43 @@ __device__ __forceinline__ void qwalk_next(const Geo& g, int j, int kmin, int km
   qwalk_settle(g, j, kmin, kmax, w);
 }
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdArgs a) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_addr(smem_raw) & 1023u) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicCAS(a.status, 0, kSiteBAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::kOffBar);
+  static_assert(sizeof(BwdBars) <= 256, "barrier block");
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sDO = smem + C::kOffDO;
-  uint8_t* sPt = smem + C::kOffPt;
   uint8_t* sDSt = smem + C::kOffDSt;
   float* sRow = reinterpret_cast<float*>(smem + C::kOffRow);
 
   const Geo& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // Work item: CTAs of one (b, Ulysses rank, kv-head) run together; inside it,
+  // key tiles in increasing original position (the causally heaviest first).
+  const int n_kt = g.P_r * g.n_ktiles;
   int wi = blockIdx.x;
+  const int order = wi % n_kt;
+  wi /= n_kt;
   const int gl = wi % g.Hkv_l;
   wi /= g.Hkv_l;
-  const int b = wi % g.B;
-  wi /= g.B;
-  const int jrank = wi % g.n_ranks;
-  wi /= g.n_ranks;
-  const int n = wi;
-  const int j = jrank / g.P_u, u = jrank % g.P_u;
+  const int u = wi % g.P_u;
+  const int b = wi / g.P_u;
+  int j, n;
+  tile_in_position_order(g, order, j, n);
+  const int jrank = j * g.P_u + u;
   const int k0 = n * kBN;
   int kmin, kmax;
   pos_range(g, j, k0, k0 + kBN, kmin, kmax);
@@ -173,12 +179,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->qd_full[s], 1);
-      mbar_init(&bars->qd_empty[s], 1);
+      mbar_init(&bars->qd_empty[s], kComputeThreads / 32);
     }
     mbar_init(&bars->st_full, 1);
-    mbar_init(&bars->p_full, 128);
+    mbar_init(&bars->p_full, kComputeThreads);
     mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_free, 128);
+    mbar_init(&bars->dq_free, kComputeThreads);
     mbar_init(&bars->drain, 1);
     fence_mbar_init();
   }
@@ -221,8 +227,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
                       qrb);
         }
         const size_t rowbase = (static_cast<size_t>(qrb) * g.Hq_l + h) * a.Lp + q0;
-        bulk_load(sRow + s * 256, a.lse2 + rowbase, 512, &bars->qd_full[s]);
-        bulk_load(sRow + s * 256 + 128, a.delta + rowbase, 512, &bars->qd_full[s]);
+        bulk_load_1d(sRow + s * 256, a.lse2 + rowbase, 512, &bars->qd_full[s]);
+        bulk_load_1d(sRow + s * 256 + 128, a.delta + rowbase, 512, &bars->qd_full[s]);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         mbar_wait_drain(&bars->kv_full, 0, a.wait_ns);
@@ -238,49 +244,75 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       constexpr uint32_t kIdKM = idesc_bf16_f32(128, D, 0, 1);    // A K-major, B MN-major
       constexpr uint32_t kIdMM = idesc_bf16_f32(128, D, 1, 1);    // both MN-major
       const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ), aDO = smem_addr(sDO);
-      const uint32_t aPt = smem_addr(sPt), aDSt = smem_addr(sDSt);
-      bool ok = mbar_wait(&bars->kv_full, 0, w, kSiteBKv);
-      bool issued_any = false;
-      int it = 0;
-      for (QWalk qw = qwalk_begin(g, j, kmin, kmax); ok && qw.valid; qwalk_next(g, j, kmin, kmax, qw), ++it) {
-        const int s = it % C::kStages;
-        if (!mbar_wait(&bars->qd_full[s], (it / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
-        if (it >= 1 && !mbar_wait(&bars->dq_free, (it - 1) & 1, w, kSiteBDqFree)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qb = aQ + s * C::kTileBytes, db = aDO + s * C::kTileBytes;
+      const uint32_t aDSt = smem_addr(sDSt);
+      auto issue_s = [&](int s) {  // S^T = K Q^T
+        const uint32_t qb = aQ + s * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
           umma_bf16(tmem + kColS, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), kIdSS,
                     kk > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dp = [&](int s) {  // dP^T = V dO^T
+        const uint32_t db = aDO + s * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
           umma_bf16(tmem + kColDP, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(db + off, 16, 1024), kIdSS,
                     kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->st_full);
-        issued_any = true;
-        if (!mbar_wait(&bars->p_full, it & 1, w, kSiteBP)) { ok = false; break; }
+      };
+      bool ok = mbar_wait(&bars->kv_full, 0, w, kSiteBKv);
+      bool issued_any = false;
+      int k = 0;
+      QWalk qw = qwalk_begin(g, j, kmin, kmax);
+      if (ok && qw.valid) {
+        ok = mbar_wait(&bars->qd_full[0], 0, w, kSiteBQd);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          issue_dp(0);
+          umma_commit(&bars->st_full);
+          issued_any = true;
+        }
+      }
+      for (; ok && qw.valid; ++k) {
+        const int s = k % C::kStages;
+        if (!mbar_wait(&bars->p_full, k & 1, w, kSiteBP)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t qb = aQ + s * C::kTileBytes, db = aDO + s * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk) {  // K = 128 queries
-          const uint32_t aoff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+          // P^T lives in TMEM: warpgroup c packed its 64 queries at columns 64c .. 64c+31
+          const uint32_t pcol = kColS + (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
           const uint32_t boff = kk * 16 * 128;
-          umma_bf16(tmem + kColDV, sdesc_sw128(aPt + aoff, 16, 1024),
-                    sdesc_sw128(db + boff, C::kPanelBytes, 1024), kIdKM, (it > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16(tmem + kColDK, sdesc_sw128(aDSt + aoff, 16, 1024),
-                    sdesc_sw128(qb + boff, C::kPanelBytes, 1024), kIdKM, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem + kColDV, tmem + pcol, sdesc_sw128(db + boff, C::kPanelBytes, 1024), kIdKM,
+                           (k > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t aoff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+          umma_bf16(tmem + kColDK, sdesc_sw128(aDSt + aoff, 16, 1024), sdesc_sw128(qb + boff, C::kPanelBytes, 1024),
+                    kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {  // K = 128 keys
           const uint32_t off = kk * 16 * 128;
-          umma_bf16(tmem + kColS, sdesc_sw128(aDSt + off, C::kPanelBytes, 1024),
+          umma_bf16(tmem + kColDQ, sdesc_sw128(aDSt + off, C::kPanelBytes, 1024),
                     sdesc_sw128(aK + off, C::kPanelBytes, 1024), kIdMM, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars->dq_full);
-        umma_commit(&bars->qd_empty[s]);
+        qwalk_next(g, j, kmin, kmax, qw);
+        if (qw.valid) {
+          const int s1 = (k + 1) % C::kStages;
+          if (!mbar_wait(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
+          // S^T of the next step overwrites the columns P^T is read from: wait for this step's UMMAs.
+          if (!mbar_wait(&bars->dq_full, k & 1, w, kSiteBDqOwn)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(s1);
+          if (!mbar_wait(&bars->dq_free, k & 1, w, kSiteBDqFree)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(s1);
+          umma_commit(&bars->st_full);
+        }
       }
       if (!ok && issued_any) {
         umma_commit(&bars->drain);
@@ -290,30 +322,33 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ compute warps
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;  // key row of S^T / dP^T / dK / dV; query row of the dQ tile
+    const int cw = warp - 2;       // 0..7
+    const int wg = cw >> 2;        // warpgroup: query columns [64 wg, 64 wg + 64)
+    const int wq = warp & 3;       // TMEM lane quarter
+    const int row = wq * 32 + lane;  // key row of S^T/dP^T/dK/dV; query row of the dQ tile
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const int tau_k = k0 + row;
     const int pos_k = tau_k < g.L ? token_pos(g, j, tau_k) : INT_MAX;  // padding keys see no query
     const bool aligned = (g.c % kBM) == 0;
+    const int cbase = wg * 64;
     bool ok = true;
-    int it = 0;
-    for (QWalk qw = qwalk_begin(g, j, kmin, kmax); qw.valid; qwalk_next(g, j, kmin, kmax, qw), ++it) {
-      const int s = it % C::kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, it & 1, w, kSiteBSt));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[s], (it / C::kStages) & 1, w, kSiteBQdC));
+    int k = 0;
+    for (QWalk qw = qwalk_begin(g, j, kmin, kmax); qw.valid; qwalk_next(g, j, kmin, kmax, qw), ++k) {
+      const int s = k % C::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, k & 1, w, kSiteBSt));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[s], (k / C::kStages) & 1, w, kSiteBQdC));
       if (!ok) break;
       tc_fence_after();
       const float* lse2 = sRow + s * 256;
       const float* dl = lse2 + 128;
       const int q0 = qw.m * kBM;
       const bool masked = qw.kind == kMasked;
-      // Visible query columns: col >= lo (causal, aligned) and col < qvalid.
       int lo = 0;
       const int qvalid = g.L - q0;
       if (masked && aligned && g.causal) lo = pos_k == INT_MAX ? INT_MAX : pos_k - token_pos(g, qw.i, q0);
 #pragma unroll
-      for (int c0 = 0; c0 < kBM; c0 += 32) {
+      for (int half = 0; half < 2; ++half) {
+        const int c0 = cbase + half * 32;
         uint32_t rs[32], rp[32];
         tmem_ld32(trow + kColS + c0, rs);
         tmem_ld32(trow + kColDP + c0, rp);
@@ -341,50 +376,75 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
           dk[c >> 1] = pack_bf16x2(dv[0], dv[1]);
         }
+        // P^T back into TMEM (columns already read by this thread), 2 bf16 per column
+        tmem_st16(trow + kColS + cbase + half * 16, pk);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int ch = (c0 >> 3) + q;  // 16-byte chunk index along the 128 queries
           const uint32_t off = (ch >> 3) * C::kPanelBytes + sw128_offset(row, ch & 7);
-          *reinterpret_cast<uint4*>(sPt + off) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           *reinterpret_cast<uint4*>(sDSt + off) = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
         }
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->p_full);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, it & 1, w, kSiteBDq));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, k & 1, w, kSiteBDq));
       if (!ok) break;
       tc_fence_after();
-      const int h = gl * g.G + qw.hh;
-      const int qrank = qw.i * g.P_u + u;
-      const bool add = q0 + row < g.L;
-      float* dq_row = a.dq_acc + ((static_cast<size_t>(qrank * g.B + b) * g.L + (add ? q0 + row : 0)) * g.Hq_l + h) * D;
+      // dQ tile: this thread's query row, columns [wg*D/2, wg*D/2 + D/2)
+      uint32_t rq[C::kBoxesPerWarp][32];
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(trow + kColS + c0, r);
-        tmem_ld_wait();
-        reg_fence32(r);
-        if (add) {
+      for (int q = 0; q < C::kBoxesPerWarp; ++q) tmem_ld32(trow + kColDQ + wg * (D / 2) + q * 32, rq[q]);
+      tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            atomicAdd(reinterpret_cast<float4*>(dq_row + c0) + q,
-                      make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                  __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])));
-        }
-      }
+      for (int q = 0; q < C::kBoxesPerWarp; ++q) reg_fence32(rq[q]);
       tc_fence_before();
       mbar_arrive(&bars->dq_free);
+      // stage 32x32 fp32 boxes in this step's Q/dO buffers (free: the step's UMMAs are done)
+      const int h = gl * g.G + qw.hh;
+      const int qrb = (qw.i * g.P_u + u) * g.B + b;
+      const int box_row = q0 + wq * 32;
+#pragma unroll
+      for (int q = 0; q < C::kBoxesPerWarp; ++q) {
+        const int box = (wg * C::kBoxesPerWarp + q) * 4 + wq;
+        uint8_t* base = box < D / 16 ? sQ + s * C::kTileBytes + box * 4096
+                                     : sDO + s * C::kTileBytes + (box - D / 16) * 4096;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(base + sw128_offset(lane, ch)) =
+              make_uint4(rq[q][4 * ch], rq[q][4 * ch + 1], rq[q][4 * ch + 2], rq[q][4 * ch + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (box_row < g.L) {
+#pragma unroll
+          for (int q = 0; q < C::kBoxesPerWarp; ++q) {
+            const int box = (wg * C::kBoxesPerWarp + q) * 4 + wq;
+            const uint8_t* base = box < D / 16 ? sQ + s * C::kTileBytes + box * 4096
+                                               : sDO + s * C::kTileBytes + (box - D / 16) * 4096;
+            tma_reduce_add_4d(&tm_dq, base, wg * (D / 2) + q * 32, h, box_row, qrb);
+          }
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        mbar_arrive(&bars->qd_empty[s]);
+      }
+      __syncwarp();
     }
+    if (lane == 0) bulk_wait_group0();  // this warp's reduce-adds have landed in global memory
+    __syncwarp();
     // ------------------------------------------------------------ dK, dV epilogue
     if (ok) {
       tc_fence_after();
       const bool store = tau_k < g.L;
       const size_t kr = (static_cast<size_t>(jrank * g.B + b) * g.L + (store ? tau_k : 0)) * g.Hkv_l + gl;
+      // warpgroup wg writes columns [wg*D/2, wg*D/2 + D/2)
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
         uint32_t rk[32], rv[32];
-        if (it >= 1) {
+        if (k >= 1) {
           tmem_ld32(trow + kColDK + c0, rk);
           tmem_ld32(trow + kColDV + c0, rv);
           tmem_ld_wait();
@@ -429,16 +489,15 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   a.lse2 = L.lse2;
   a.delta = L.delta;
   a.Lp = L.Lp;
-  a.dq_acc = L.dq_acc;
   a.dk = L.dk;
   a.dv = L.dv;
   a.status = L.status;
   a.wait_ns = L.wait_ns;
-  const long long blocks = static_cast<long long>(a.g.n_ktiles) * a.g.n_ranks * a.g.B * a.g.Hkv_l;
+  const long long blocks = static_cast<long long>(a.g.n_ktiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hkv_l;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  attn_bwd_kernel<D><<<static_cast<unsigned>(blocks), kThreadsBwd, C::kSmemBytes, stream>>>(L.tm_q, L.tm_k, L.tm_v,
-                                                                                           L.tm_do, a);
+  attn_bwd_kernel<D><<<static_cast<unsigned>(blocks), kThreadsBwd, C::kSmemBytes, stream>>>(
+      L.tm_q, L.tm_k, L.tm_v, L.tm_do, L.tm_dq, a);
   return cudaGetLastError();
 }
 

@@ -57,6 +57,23 @@ __device__ __forceinline__ void pos_range(const Geo& g, int i, int t0, int t1, i
   }
 }
 
+// The o-th 128-token tile of the whole sequence (all ring ranks) in increasing
+// original position: returns its ring rank i and local tile index n. When a
+// chunk is not a whole number of tiles the plain (rank, tile) order is used.
+__device__ __forceinline__ void tile_in_position_order(const Geo& g, int o, int& i, int& n) {
+  if (g.c % kBN == 0) {
+    const int tpc = g.c / kBN;  // tiles per chunk
+    const int chunk = o / tpc, within = o % tpc;
+    const bool late = chunk >= g.P;
+    const int r = late ? 2 * g.P - 1 - chunk : chunk;
+    i = r / g.P_u;
+    n = (2 * (r % g.P_u) + (late ? 1 : 0)) * tpc + within;
+  } else {
+    i = o / g.n_ktiles;
+    n = o % g.n_ktiles;
+  }
+}
+
 enum TileKind { kSkip = 0, kFull = 1, kMasked = 2 };
 
 // Kind of the pair (query tile with positions [qmin, qmax], key tile n of ring rank j).

@@ -93,16 +93,20 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   const Geo& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Work item: heaviest (latest) query tiles first.
+  // Work item: CTAs of one (b, Ulysses rank, head) run together so that its K/V
+  // stay in L2; inside it, query tiles in decreasing original position (the
+  // causally heaviest first).
+  const int n_qt = g.P_r * g.n_qtiles;
   int wi = blockIdx.x;
+  const int order = n_qt - 1 - wi % n_qt;
+  wi /= n_qt;
   const int h = wi % g.Hq_l;
   wi /= g.Hq_l;
-  const int b = wi % g.B;
-  wi /= g.B;
-  const int rank = wi % g.n_ranks;
-  wi /= g.n_ranks;
-  const int m = g.n_qtiles - 1 - wi;
-  const int i = rank / g.P_u, u = rank % g.P_u;
+  const int u = wi % g.P_u;
+  const int b = wi / g.P_u;
+  int i, m;
+  tile_in_position_order(g, order, i, m);
+  const int rank = i * g.P_u + u;
   const int kvh = h / g.G;
   const int q0 = m * kBM;
   const int t_begin = a.step < 0 ? 0 : a.step;

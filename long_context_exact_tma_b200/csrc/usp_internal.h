@@ -59,6 +59,7 @@ cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* l
 struct BwdLaunch {
   AttnGeom g;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  CUtensorMap tm_dq;   // fp32 dQ accumulator, box 32 x 1 x 32 rows (TMA reduce-add target)
   const float* lse2;   // [n_ranks*B*Hq_l][Lp]
   const float* delta;  // [n_ranks*B*Hq_l][Lp]
   int Lp;
