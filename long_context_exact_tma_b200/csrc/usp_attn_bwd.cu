@@ -75,14 +75,17 @@ struct BwdArgs {
 struct BwdBars {
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
-  uint64_t st_full, p_full, dq_full, dq_free, drain;
+  uint64_t st_full, p_full, p_used, dq_full, dq_free, drain;
+  // Step descriptors published by the producer with qd_full of that step:
+  // {q-head in group (-1 = no more steps), ring rank i, query tile m, tile kind}.
+  int step[4][4];
   uint32_t tmem_base;
   int abort_flag;
 };
 
 enum : int {
   kSiteBKv = 0x201, kSiteBQdEmpty = 0x202, kSiteBQd = 0x211, kSiteBDqFree = 0x212, kSiteBP = 0x213,
-  kSiteBDqOwn = 0x214, kSiteBSt = 0x221, kSiteBDq = 0x222, kSiteBQdC = 0x223, kSiteBAlign = 0x2FF
+  kSiteBPUsed = 0x214, kSiteBSt = 0x221, kSiteBDq = 0x222, kSiteBQdC = 0x223, kSiteBAlign = 0x2FF
 };
 
 // Query steps of one key tile: q-head hh of the group, ring rank i, query tile m.
@@ -183,6 +186,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->p_full, kComputeThreads);
+    mbar_init(&bars->p_used, 1);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_free, kComputeThreads);
     mbar_init(&bars->drain, 1);
@@ -212,11 +216,22 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         tma_load_4d(&tm_v, &bars->kv_full, sV + p * C::kPanelBytes, p * 64, gl, k0, krb);
       }
       int issued = 0;
-      for (QWalk qw = qwalk_begin(g, j, kmin, kmax); qw.valid; qwalk_next(g, j, kmin, kmax, qw), ++issued) {
+      QWalk qw = qwalk_begin(g, j, kmin, kmax);
+      while (true) {
         const int s = issued % C::kStages;
         if (issued >= C::kStages &&
             !mbar_wait(&bars->qd_empty[s], ((issued / C::kStages) - 1) & 1, w, kSiteBQdEmpty))
           break;
+        int* slot = bars->step[issued & 3];
+        if (!qw.valid) {  // publish the end of the walk on this stage's barrier
+          slot[0] = -1;
+          mbar_arrive(&bars->qd_full[s]);
+          break;
+        }
+        slot[0] = qw.hh;
+        slot[1] = qw.i;
+        slot[2] = qw.m;
+        slot[3] = qw.kind;
         const int h = gl * g.G + qw.hh;
         const int qrb = (qw.i * g.P_u + u) * g.B + b;
         const int q0 = qw.m * kBM;
@@ -229,6 +244,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const size_t rowbase = (static_cast<size_t>(qrb) * g.Hq_l + h) * a.Lp + q0;
         bulk_load_1d(sRow + s * 256, a.lse2 + rowbase, 512, &bars->qd_full[s]);
         bulk_load_1d(sRow + s * 256 + 128, a.delta + rowbase, 512, &bars->qd_full[s]);
+        ++issued;
+        qwalk_next(g, j, kmin, kmax, qw);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         mbar_wait_drain(&bars->kv_full, 0, a.wait_ns);
@@ -265,11 +282,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       };
       bool ok = mbar_wait(&bars->kv_full, 0, w, kSiteBKv);
       bool issued_any = false;
+      bool have = false;
       int k = 0;
-      QWalk qw = qwalk_begin(g, j, kmin, kmax);
-      if (ok && qw.valid) {
-        ok = mbar_wait(&bars->qd_full[0], 0, w, kSiteBQd);
-        if (ok) {
+      if (ok) ok = mbar_wait(&bars->qd_full[0], 0, w, kSiteBQd);
+      if (ok) {
+        have = bars->step[0][0] >= 0;
+        if (have) {
           tc_fence_after();
           issue_s(0);
           issue_dp(0);
@@ -277,42 +295,44 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           issued_any = true;
         }
       }
-      for (; ok && qw.valid; ++k) {
+      for (; ok && have; ++k) {
         const int s = k % C::kStages;
         if (!mbar_wait(&bars->p_full, k & 1, w, kSiteBP)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qb = aQ + s * C::kTileBytes, db = aDO + s * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk) {  // K = 128 queries
+        for (int kk = 0; kk < kBM / 16; ++kk) {  // dV += P^T dO, K = 128 queries
           // P^T lives in TMEM: warpgroup c packed its 64 queries at columns 64c .. 64c+31
           const uint32_t pcol = kColS + (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
-          const uint32_t boff = kk * 16 * 128;
-          umma_bf16_tmem_a(tmem + kColDV, tmem + pcol, sdesc_sw128(db + boff, C::kPanelBytes, 1024), kIdKM,
-                           (k > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem + kColDV, tmem + pcol, sdesc_sw128(db + kk * 16 * 128, C::kPanelBytes, 1024),
+                           kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->p_used);  // P^T (in the S^T columns) has been read once this lands
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk) {  // dK += dS^T Q, K = 128 queries
           const uint32_t aoff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_bf16(tmem + kColDK, sdesc_sw128(aDSt + aoff, 16, 1024), sdesc_sw128(qb + boff, C::kPanelBytes, 1024),
-                    kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(tmem + kColDK, sdesc_sw128(aDSt + aoff, 16, 1024),
+                    sdesc_sw128(qb + kk * 16 * 128, C::kPanelBytes, 1024), kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
         }
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {  // K = 128 keys
+        for (int kk = 0; kk < kBN / 16; ++kk) {  // dQt = dS K, K = 128 keys
           const uint32_t off = kk * 16 * 128;
           umma_bf16(tmem + kColDQ, sdesc_sw128(aDSt + off, C::kPanelBytes, 1024),
                     sdesc_sw128(aK + off, C::kPanelBytes, 1024), kIdMM, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars->dq_full);
-        qwalk_next(g, j, kmin, kmax, qw);
-        if (qw.valid) {
-          const int s1 = (k + 1) % C::kStages;
-          if (!mbar_wait(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
-          // S^T of the next step overwrites the columns P^T is read from: wait for this step's UMMAs.
-          if (!mbar_wait(&bars->dq_full, k & 1, w, kSiteBDqOwn)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(s1);
-          if (!mbar_wait(&bars->dq_free, k & 1, w, kSiteBDqFree)) { ok = false; break; }
-          tc_fence_after();
-          issue_dp(s1);
-          umma_commit(&bars->st_full);
-        }
+        const int s1 = (k + 1) % C::kStages;
+        if (!mbar_wait(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
+        have = bars->step[(k + 1) & 3][0] >= 0;
+        if (!have) break;
+        // S^T of the next step overwrites the columns P^T is read from: wait for the dV UMMAs only.
+        if (!mbar_wait(&bars->p_used, k & 1, w, kSiteBPUsed)) { ok = false; break; }
+        tc_fence_after();
+        issue_s(s1);
+        if (!mbar_wait(&bars->dq_free, k & 1, w, kSiteBDqFree)) { ok = false; break; }
+        tc_fence_after();
+        issue_dp(s1);
+        umma_commit(&bars->st_full);
       }
       if (!ok && issued_any) {
         umma_commit(&bars->drain);
@@ -333,19 +353,24 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     const int cbase = wg * 64;
     bool ok = true;
     int k = 0;
-    for (QWalk qw = qwalk_begin(g, j, kmin, kmax); qw.valid; qwalk_next(g, j, kmin, kmax, qw), ++k) {
+    for (;; ++k) {
       const int s = k % C::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[s], (k / C::kStages) & 1, w, kSiteBQdC));
+      if (!ok) break;
+      const int* slot = bars->step[k & 3];
+      const int st_hh = slot[0];
+      if (st_hh < 0) break;
+      const int st_i = slot[1], st_m = slot[2], st_kind = slot[3];
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, k & 1, w, kSiteBSt));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->qd_full[s], (k / C::kStages) & 1, w, kSiteBQdC));
       if (!ok) break;
       tc_fence_after();
       const float* lse2 = sRow + s * 256;
       const float* dl = lse2 + 128;
-      const int q0 = qw.m * kBM;
-      const bool masked = qw.kind == kMasked;
+      const int q0 = st_m * kBM;
+      const bool masked = st_kind == kMasked;
       int lo = 0;
       const int qvalid = g.L - q0;
-      if (masked && aligned && g.causal) lo = pos_k == INT_MAX ? INT_MAX : pos_k - token_pos(g, qw.i, q0);
+      if (masked && aligned && g.causal) lo = pos_k == INT_MAX ? INT_MAX : pos_k - token_pos(g, st_i, q0);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int c0 = cbase + half * 32;
@@ -367,7 +392,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
               if (aligned || !g.causal)
                 vis = col >= lo && col < qvalid;
               else
-                vis = col < qvalid && pos_k <= token_pos(g, qw.i, q0 + col);
+                vis = col < qvalid && pos_k <= token_pos(g, st_i, q0 + col);
             }
             const float p = vis ? ex2_approx(fmaf(__uint_as_float(rs[c + e]), g.scale_log2, -lse2[col])) : 0.f;
             pv[e] = p;
@@ -402,8 +427,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       tc_fence_before();
       mbar_arrive(&bars->dq_free);
       // stage 32x32 fp32 boxes in this step's Q/dO buffers (free: the step's UMMAs are done)
-      const int h = gl * g.G + qw.hh;
-      const int qrb = (qw.i * g.P_u + u) * g.B + b;
+      const int h = gl * g.G + st_hh;
+      const int qrb = (st_i * g.P_u + u) * g.B + b;
       const int box_row = q0 + wq * 32;
 #pragma unroll
       for (int q = 0; q < C::kBoxesPerWarp; ++q) {

@@ -67,6 +67,9 @@ struct FwdBars {
   uint64_t k_full[3], v_full[3], kv_empty[3];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, o_done, drain;
+  // Key-tile descriptors published by the producer with k_full of that tile:
+  // {1, or -1 = no more tiles; ring rank j of the key owner; key tile n; tile kind}.
+  int step[4][4];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -74,7 +77,7 @@ struct FwdBars {
 // Wait-site codes recorded in the status word: 0x100 | role << 4 | which.
 enum : int {
   kSiteQ = 0x101, kSiteKvEmpty = 0x102, kSiteK = 0x111, kSiteSFree = 0x112, kSiteP = 0x113, kSiteV = 0x114,
-  kSiteS = 0x121, kSiteO = 0x122
+  kSiteS = 0x121, kSiteO = 0x122, kSiteKs = 0x123
 };
 
 template <int D>
@@ -147,19 +150,31 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     if (lane == 0) {
       KvWalk kw = kv_walk_begin(g, i, qmin, qmax, t_begin, t_end);
       int issued = 0;
-      if (kw.valid) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        const int qrb = rank * g.B + b;
-        mbar_expect_tx(&bars->q_full, C::kTileBytes);
-        for (int p = 0; p < C::kPanels; ++p)
-          tma_load_4d(&tm_q, &bars->q_full, sQ + p * C::kPanelBytes, p * 64, h, q0, qrb);
-        for (; kw.valid; kv_walk_next(g, i, qmin, qmax, t_end, kw), ++issued) {
+      const bool any = kw.valid;
+      {
+        if (any) {
+          tma_prefetch_desc(&tm_q);
+          tma_prefetch_desc(&tm_k);
+          tma_prefetch_desc(&tm_v);
+          mbar_expect_tx(&bars->q_full, C::kTileBytes);
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_4d(&tm_q, &bars->q_full, sQ + p * C::kPanelBytes, p * 64, h, q0, rank * g.B + b);
+        }
+        while (true) {
           const int s = issued % C::kStages;
           if (issued >= C::kStages &&
               !mbar_wait(&bars->kv_empty[s], ((issued / C::kStages) - 1) & 1, w, kSiteKvEmpty))
             break;
+          int* slot = bars->step[issued & 3];
+          if (!kw.valid) {  // publish the end of the walk on this stage's barrier
+            slot[0] = -1;
+            mbar_arrive(&bars->k_full[s]);
+            break;
+          }
+          slot[0] = 1;
+          slot[1] = kw.j;
+          slot[2] = kw.n;
+          slot[3] = kw.kind;
           const int krb = (kw.j * g.P_u + u) * g.B + b;
           mbar_expect_tx(&bars->k_full[s], C::kTileBytes);
           for (int p = 0; p < C::kPanels; ++p)
@@ -169,10 +184,12 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           for (int p = 0; p < C::kPanels; ++p)
             tma_load_4d(&tm_v, &bars->v_full[s], sV + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
                         kw.n * kBN, krb);
+          ++issued;
+          kv_walk_next(g, i, qmin, qmax, t_end, kw);
         }
         if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
           // Let every copy this thread started land before the CTA exits.
-          mbar_wait_drain(&bars->q_full, 0, a.wait_ns);
+          if (any) mbar_wait_drain(&bars->q_full, 0, a.wait_ns);
           for (int it = issued - C::kStages < 0 ? 0 : issued - C::kStages; it < issued; ++it) {
             mbar_wait_drain(&bars->k_full[it % C::kStages], (it / C::kStages) & 1, a.wait_ns);
             mbar_wait_drain(&bars->v_full[it % C::kStages], (it / C::kStages) & 1, a.wait_ns);
@@ -187,7 +204,6 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, 0, 1);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aP = smem_addr(sP);
-      KvWalk kw = kv_walk_begin(g, i, qmin, qmax, t_begin, t_end);
       bool ok = true;
       int it = 0;
       bool issued_any = false;
@@ -207,11 +223,16 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         umma_commit(&bars->kv_empty[s]);
         return true;
       };
-      if (kw.valid) ok = mbar_wait(&bars->q_full, 0, w, kSiteQ);
-      for (; ok && kw.valid; kv_walk_next(g, i, qmin, qmax, t_end, kw), ++it) {
+      ok = mbar_wait(&bars->k_full[0], 0, w, kSiteK);
+      bool have = ok && bars->step[0][0] >= 0;
+      if (have) ok = mbar_wait(&bars->q_full, 0, w, kSiteQ);
+      for (; ok && have; ++it) {
         const int s = it % C::kStages;
         const int sb = it & 1;
-        if (!mbar_wait(&bars->k_full[s], (it / C::kStages) & 1, w, kSiteK)) { ok = false; break; }
+        if (it > 0) {
+          if (!mbar_wait(&bars->k_full[s], (it / C::kStages) & 1, w, kSiteK)) { ok = false; break; }
+          if (bars->step[it & 3][0] < 0) break;
+        }
         if (it >= 2 && !mbar_wait(&bars->s_free[sb], ((it >> 1) - 1) & 1, w, kSiteSFree)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kbase = aK + s * C::kTileBytes;
@@ -244,11 +265,15 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     // weights the PV UMMA consumes (normalises O, so O stays a convex combination
     // of V rows even when one key dominates).
     float m_use = -INFINITY, l_run = 0.f, lb_run = 0.f;
-    KvWalk kw = kv_walk_begin(g, i, qmin, qmax, t_begin, t_end);
     int it = 0;
     bool ok = true;
-    for (; kw.valid; kv_walk_next(g, i, qmin, qmax, t_end, kw), ++it) {
+    for (;; ++it) {
       const int sb = it & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->k_full[it % C::kStages], (it / C::kStages) & 1, w, kSiteKs));
+      if (!ok) break;
+      const int* slot = bars->step[it & 3];
+      if (slot[0] < 0) break;
+      const int kj = slot[1], kn = slot[2], kkind = slot[3];
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (it >> 1) & 1, w, kSiteS));
       if (!ok) break;
       tc_fence_after();
@@ -272,19 +297,19 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         s[64 + c] = __uint_as_float(r2[c]);
         s[96 + c] = __uint_as_float(r3[c]);
       }
-      if (kw.kind == kMasked) {
-        const int k0 = kw.n * kBN;
+      if (kkind == kMasked) {
+        const int k0 = kn * kBN;
         const int kvalid = g.L - k0;  // keys at or past this column are padding
         if (aligned) {
           // the whole key tile lies in one chunk: positions are base + column
-          const int lim = g.causal ? pos_q - token_pos(g, kw.j, k0) : INT_MAX;
+          const int lim = g.causal ? pos_q - token_pos(g, kj, k0) : INT_MAX;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c > lim || c >= kvalid) s[c] = -INFINITY;
         } else {
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
-            const bool vis = c < kvalid && (!g.causal || token_pos(g, kw.j, k0 + c) <= pos_q);
+            const bool vis = c < kvalid && (!g.causal || token_pos(g, kj, k0 + c) <= pos_q);
             if (!vis) s[c] = -INFINITY;
           }
         }
