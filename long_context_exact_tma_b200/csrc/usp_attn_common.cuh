@@ -49,6 +49,7 @@ __device__ __forceinline__ void pos_range(const Geo& g, int i, int t0, int t1, i
   if (t1 > g.L) t1 = g.L;
   pmin = INT_MAX;
   pmax = -1;
+  if (t0 >= t1) return;  // the range lies wholly in the padding past L
   for (int kap = t0 / g.c; kap * g.c < t1; ++kap) {
     const int a = max(t0, kap * g.c);
     const int e = min(t1, (kap + 1) * g.c) - 1;
