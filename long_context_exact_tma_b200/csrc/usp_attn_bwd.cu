@@ -98,8 +98,8 @@ __device__ __forceinline__ int classify_q(const Geo& g, int i, int m, int kmin, 
   const int q0 = m * kBM;
   int qmin, qmax;
   pos_range(g, i, q0, q0 + kBM, qmin, qmax);
+  // Padded query columns need no mask: their LSE is +inf, so P = 0 there.
   if (g.causal && qmax < kmin) return kSkip;
-  if (q0 + kBM > g.L) return kMasked;  // padded query columns must be masked
   if (!g.causal || qmin >= kmax) return kFull;
   return kMasked;
 }
@@ -367,10 +367,35 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const float* lse2 = sRow + s * 256;
       const float* dl = lse2 + 128;
       const int q0 = st_m * kBM;
-      const bool masked = st_kind == kMasked;
-      int lo = 0;
-      const int qvalid = g.L - q0;
-      if (masked && aligned && g.causal) lo = pos_k == INT_MAX ? INT_MAX : pos_k - token_pos(g, st_i, q0);
+      if (st_kind == kMasked) {
+        // causal: rewrite S^T of this key row to -inf where the query does not see
+        // the key, so the main pass carries no masking (P = 0 there)
+        const int lo = pos_k == INT_MAX ? kBM : pos_k - token_pos(g, st_i, q0);  // aligned: cols >= lo see it
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          const int c0 = cbase + half * 32;
+          uint32_t vis;  // bit c: query column c0 + c sees this key
+          if (aligned) {
+            const int nb = min(max(lo - c0, 0), 32);  // leading invisible columns
+            vis = nb >= 32 ? 0u : (0xFFFFFFFFu << nb);
+          } else {
+            vis = 0u;
+            for (int c = 0; c < 32; ++c) {
+              const int tq = q0 + c0 + c;
+              if (tq < g.L && pos_k <= token_pos(g, st_i, tq)) vis |= 1u << c;
+            }
+          }
+          uint32_t r[32];
+          tmem_ld32(trow + kColS + c0, r);
+          tmem_ld_wait();
+          reg_fence32(r);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (!((vis >> c) & 1u)) r[c] = 0xFF800000u;  // -inf
+          tmem_st32(trow + kColS + c0, r);
+        }
+        tmem_st_wait();
+      }
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int c0 = cbase + half * 32;
@@ -387,14 +412,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int col = c0 + c + e;
-            bool vis = true;
-            if (masked) {
-              if (aligned || !g.causal)
-                vis = col >= lo && col < qvalid;
-              else
-                vis = col < qvalid && pos_k <= token_pos(g, st_i, q0 + col);
-            }
-            const float p = vis ? ex2_approx(fmaf(__uint_as_float(rs[c + e]), g.scale_log2, -lse2[col])) : 0.f;
+            const float p = ex2_approx(fmaf(__uint_as_float(rs[c + e]), g.scale_log2, -lse2[col]));  // -inf -> 0
             pv[e] = p;
             dv[e] = p * (__uint_as_float(rp[c + e]) - dl[col]) * g.scale;
           }

@@ -120,6 +120,18 @@ __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16*
       lse2_t[dst] = lse[r] * 1.4426950408889634f;
     }
   }
+  // Padding rows [L, Lp) of every head: LSE = +inf and Delta = 0, so a padded
+  // query contributes exactly zero (P = exp2(s - inf) = 0) whatever the workspace held.
+  const long long pad = Lp - L;
+  if (pad > 0) {
+    const long long n_pad = (rows / L) * pad;  // heads * padding rows
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < n_pad; x += stride) {
+      const long long dst = (x / pad) * Lp + L + x % pad;
+      delta_t[dst] = 0.f;
+      lse2_t[dst] = INFINITY;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,

@@ -98,3 +98,22 @@ def test_bwd_full_size_sampled(cuda, cfg):
         dk_g = dk.double().numpy()[ci[:, 0], ci[:, 2], ci[:, 1]]
         dv_g = dv.double().numpy()[ci[:, 0], ci[:, 2], ci[:, 1]]
         assert rel_l2(dk_g, dk_ref) <= GRAD_REL_L2 and rel_l2(dv_g, dv_ref) <= GRAD_REL_L2
+
+
+def test_bwd_ignores_stale_workspace_contents(cuda):
+    """A workspace full of NaN bytes (a reused scratch) gives the same gradients as
+    a fresh one, on a ragged causal case whose padded query rows read it."""
+    from long_context_exact_tma_b200 import binding as B_
+    spec = make_spec(S=600, Hq=4, Hkv=2, D=128, P_u=1, P_r=3, seed=308)
+    t = inputs(spec, which=("q", "k", "v", "do"))
+    P_u, P_r = spec["P_u"], spec["P_r"]
+    q, k, v, do = (head_shard_cpu(t[n], spec).to(cuda) for n in ("q", "k", "v", "do"))
+    out, lse = api.attn_fwd(q, k, v, True, P_u, P_r)
+    clean = api.attn_bwd(q, k, v, out, lse, do, True, P_u, P_r)
+    need = B_.usp_attn_workspace_size(1, 600, 4, 2, 128, 1, P_u, P_r, 0, 1)
+    dirty_ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=cuda)
+    dirty = api.attn_bwd(q, k, v, out, lse, do, True, P_u, P_r, ws=dirty_ws)
+    torch.cuda.synchronize()
+    for a_, b_ in zip(clean, dirty):
+        assert torch.isfinite(b_.float()).all()
+        assert rel_l2(b_.double().cpu().numpy(), a_.double().cpu().numpy()) <= 1e-5
