@@ -330,17 +330,31 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         }
         tmem_st_wait();
       }
-      // pass 1: row max, 32 columns at a time
-      float mx = -INFINITY;
+      // The whole S row in registers: one round trip to TMEM.
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      tmem_ld32(trow + cS + 0, r0);
+      tmem_ld32(trow + cS + 32, r1);
+      tmem_ld32(trow + cS + 64, r2);
+      tmem_ld32(trow + cS + 96, r3);
+      tmem_ld_wait();
+      reg_fence32(r0);
+      reg_fence32(r1);
+      reg_fence32(r2);
+      reg_fence32(r3);
+      // row max with 8 independent partial maxima (short dependency chains)
+      float pm[8];
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(trow + cS + c0, r);
-        tmem_ld_wait();
-        reg_fence32(r);
+      for (int q = 0; q < 8; ++q) pm[q] = fmax3(__uint_as_float(r0[q]), __uint_as_float(r1[q]), __uint_as_float(r2[q]));
 #pragma unroll
-        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+      for (int c = 8; c < 32; c += 8) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) pm[q] = fmax3(pm[q], __uint_as_float(r0[c + q]), __uint_as_float(r1[c + q]));
+#pragma unroll
+        for (int q = 0; q < 8; ++q) pm[q] = fmax3(pm[q], __uint_as_float(r2[c + q]), __uint_as_float(r3[c + q]));
       }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) pm[q] = fmaxf(pm[q], __uint_as_float(r3[q]));
+      const float mx = fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], fmax3(pm[5], pm[6], pm[7])));
       const float m_tile = mx * g.scale_log2;
       const bool bump = m_tile > m_use + kRescaleThresh;
       float alpha = 1.f;
@@ -348,6 +362,34 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         alpha = ex2_approx(m_use - m_tile);
         m_use = m_tile;
       }
+      const float m_safe = m_use == -INFINITY ? 0.f : m_use;
+      // P = exp2(S*scale*log2e - m) as bf16 into the first 64 columns of S_t, two
+      // keys per column (-inf scores give 0).
+      // independent packed accumulators for the fp32 and the bf16-rounded sums
+      float2 acc[4], accb[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = accb[q] = make_float2(0.f, 0.f);
+      const float2 sl2 = make_float2(g.scale_log2, g.scale_log2);
+      const float2 nm = make_float2(-m_safe, -m_safe);
+      auto emit = [&](const uint32_t (&r)[32], uint32_t col) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2, nm);
+          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], pv);
+          pk[c >> 1] = pack_bf16x2(pv.x, pv.y);
+          accb[(c >> 1) & 3] = fadd2(accb[(c >> 1) & 3], bf16x2_unpack(pk[c >> 1]));
+        }
+        tmem_st16(trow + cS + col, pk);
+      };
+      emit(r0, 0);
+      emit(r1, 16);
+      emit(r2, 32);
+      emit(r3, 48);
+      const float rs = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) + (acc[3].x + acc[3].y);
+      const float rsb =
+          (accb[0].x + accb[0].y) + (accb[1].x + accb[1].y) + (accb[2].x + accb[2].y) + (accb[3].x + accb[3].y);
       // The PV UMMA of the previous tile has completed (S_t is only issued after
       // it), so O_t can be rescaled in place.
       if (it > 0 && __any_sync(0xffffffffu, bump)) {
@@ -361,30 +403,6 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
           tmem_st32(trow + cO + c0, o);
         }
-      }
-      const float m_safe = m_use == -INFINITY ? 0.f : m_use;
-      // pass 2: P = exp2(S*scale*log2e - m) as bf16 into the first 64 columns of S_t
-      // (two keys per column; chunk c0 lands on columns this thread has already read)
-      float rs = 0.f, rsb = 0.f;
-#pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(trow + cS + c0, r);
-        tmem_ld_wait();
-        reg_fence32(r);
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            pv[e] = ex2_approx(fmaf(__uint_as_float(r[c + e]), g.scale_log2, -m_safe));  // -inf -> 0
-            rs += pv[e];
-          }
-          pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-          rsb += bf16x2_sum(pk[c >> 1]);
-        }
-        tmem_st16(trow + cS + c0 / 2, pk);
       }
       l_run = l_run * alpha + rs;
       lb_run = lb_run * alpha + rsb;
