@@ -1,6 +1,7 @@
 // usp_api.cu -- the extern "C" entry points of libusp.so (declared in include/usp.h):
 // argument validation, workspace accounting, TMA tensor maps and kernel launches.
 #include <cudaTypedefs.h>
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -280,7 +281,7 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   if (e != cudaSuccess) return cuda_fail(e, "preprocess launch");
   e = launch_attn_bwd(L, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");
-  e = launch_f32_to_bf16(dq_acc, dQ, static_cast<long long>(rows) * D, st);
+  e = launch_f32_to_bf16(dq_acc, dQ, static_cast<long long>(rows) * D, 1.0f / sqrtf(static_cast<float>(D)), st);
   return e == cudaSuccess ? USP_OK : cuda_fail(e, "dQ conversion launch");
 }
 

@@ -4,7 +4,8 @@
 // give no formula, these are the derivatives of softmax attention): with P
 // recomputed from the forward's final merged LSE,
 //   P_ij = exp(scale q_i.k_j - LSE_i),   dP = dO V^T,   Delta_i = sum_d dO_id O_id,
-//   dS = scale * P o (dP - Delta),        dQ = dS K,   dK = dS^T Q,   dV = P^T dO,
+//   dS = scale * P o (dP - Delta),        dQ = dS K,   dK = dS^T Q,   dV = P^T dO
+// (the scale is applied once, to dK in the epilogue and to dQ in its conversion),
 // with dK/dV summed over the q-heads of a GQA group and over every ring rank's
 // queries (in the ring algorithm dK/dV travel around the ring with K/V).
 //
@@ -63,8 +64,8 @@ struct BwdCfg {
 
 struct BwdArgs {
   Geo g;
-  const float* lse2;   // [n_ranks*B*Hq_l][Lp]: LSE * log2(e)
-  const float* delta;  // [n_ranks*B*Hq_l][Lp]
+  const float* lse2;   // [n_ranks*B*Hq_l][Lp]: -LSE * log2(e)
+  const float* delta;  // [n_ranks*B*Hq_l][Lp]: -Delta
   int Lp;
   float* dk;           // fp32 [n_ranks][B][L][Hkv_l][D]
   float* dv;
@@ -364,8 +365,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, k & 1, w, kSiteBSt));
       if (!ok) break;
       tc_fence_after();
-      const float* lse2 = sRow + s * 256;
-      const float* dl = lse2 + 128;
+      const float* nlse2 = sRow + s * 256;  // -LSE*log2(e) of the 128 query rows
+      const float* ndl = nlse2 + 128;         // -Delta of the 128 query rows
       const int q0 = st_m * kBM;
       if (st_kind == kMasked) {
         // causal: rewrite S^T of this key row to -inf where the query does not see
@@ -406,18 +407,18 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         reg_fence32(rs);
         reg_fence32(rp);
         uint32_t pk[16], dk[16];
+        const float2 sl2 = make_float2(g.scale_log2, g.scale_log2);
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = c0 + c + e;
-            const float p = ex2_approx(fmaf(__uint_as_float(rs[c + e]), g.scale_log2, -lse2[col]));  // -inf -> 0
-            pv[e] = p;
-            dv[e] = p * (__uint_as_float(rp[c + e]) - dl[col]) * g.scale;
-          }
-          pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-          dk[c >> 1] = pack_bf16x2(dv[0], dv[1]);
+          // nlse2 = -LSE*log2(e) and ndl = -Delta of the two query columns (smem broadcast)
+          const float2 nl = *reinterpret_cast<const float2*>(nlse2 + c0 + c);
+          const float2 nd = *reinterpret_cast<const float2*>(ndl + c0 + c);
+          const float2 x = ffma2(make_float2(__uint_as_float(rs[c]), __uint_as_float(rs[c + 1])), sl2, nl);
+          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));  // -inf -> 0
+          // dS (without the softmax scale, which is applied to dK and dQ at the end)
+          const float2 ds = fmul2(pv, fadd2(make_float2(__uint_as_float(rp[c]), __uint_as_float(rp[c + 1])), nd));
+          pk[c >> 1] = pack_bf16x2(pv.x, pv.y);
+          dk[c >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         // P^T back into TMEM (columns already read by this thread), 2 bf16 per column
         tmem_st16(trow + kColS + cbase + half * 16, pk);
@@ -502,8 +503,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           float4* dvp = reinterpret_cast<float4*>(a.dv + kr * D + c0);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            dkp[q] = make_float4(__uint_as_float(rk[4 * q]), __uint_as_float(rk[4 * q + 1]),
-                                 __uint_as_float(rk[4 * q + 2]), __uint_as_float(rk[4 * q + 3]));
+            dkp[q] = make_float4(__uint_as_float(rk[4 * q]) * g.scale, __uint_as_float(rk[4 * q + 1]) * g.scale,
+                                 __uint_as_float(rk[4 * q + 2]) * g.scale, __uint_as_float(rk[4 * q + 3]) * g.scale);
             dvp[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
                                  __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
           }

@@ -86,8 +86,9 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
   }
 }
 
-// Delta and LSE*log2(e) of every row, written per head: row (rb, tau, h) of the
-// head-sharded layout goes to [rb*Hl + h][tau] of a [n_rb*Hl][Lp] table.
+// -Delta and -LSE*log2(e) of every row (the negated forms the backward adds),
+// written per head: row (rb, tau, h) of the head-sharded layout goes to
+// [rb*Hl + h][tau] of a [n_rb*Hl][Lp] table.
 __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16* __restrict__ out,
                                                             const __nv_bfloat16* __restrict__ dO,
                                                             const float* __restrict__ lse,
@@ -116,8 +117,8 @@ __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16*
     if (lane == 0) {
       const long long h = r % Hl, rt = r / Hl, tau = rt % L, rb = rt / L;
       const long long dst = (rb * Hl + h) * Lp + tau;
-      delta_t[dst] = acc;
-      lse2_t[dst] = lse[r] * 1.4426950408889634f;
+      delta_t[dst] = -acc;
+      lse2_t[dst] = -lse[r] * 1.4426950408889634f;
     }
   }
   // Padding rows [L, Lp) of every head: LSE = +inf and Delta = 0, so a padded
@@ -129,19 +130,19 @@ __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16*
     for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < n_pad; x += stride) {
       const long long dst = (x / pad) * Lp + L + x % pad;
       delta_t[dst] = 0.f;
-      lse2_t[dst] = INFINITY;
+      lse2_t[dst] = -INFINITY;
     }
   }
 }
 
 __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
-                                                          long long n4) {
+                                                          long long n4, float scale) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
     const float4 v = __ldcs(src + i);
     uint2 p;
-    p.x = pack_bf16x2(v.x, v.y);
-    p.y = pack_bf16x2(v.z, v.w);
+    p.x = pack_bf16x2(v.x * scale, v.y * scale);
+    p.y = pack_bf16x2(v.z * scale, v.w * scale);
     __stcs(dst + i, p);
   }
 }
@@ -208,11 +209,11 @@ cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* l
   return cudaGetLastError();
 }
 
-cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t stream) {
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, float scale, cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
   const long long n4 = n / 4;  // callers pass multiples of 4 (D is 64 or 128)
   f32_to_bf16_kernel<<<grid_for(256, n4), 256, 0, stream>>>(reinterpret_cast<const float4*>(src),
-                                                            static_cast<uint2*>(dst), n4);
+                                                            static_cast<uint2*>(dst), n4, scale);
   return cudaGetLastError();
 }
 

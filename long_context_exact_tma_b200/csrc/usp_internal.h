@@ -28,7 +28,8 @@ cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n
                              void* out, int out_f32, float* lse_out, cudaStream_t stream);
 cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D,
                                   cudaStream_t stream);
-cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t stream);
+// dst = bf16(src * scale), n a multiple of 4.
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, float scale, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
 
 // Geometry of one attention problem in the head-sharded layout.
@@ -52,7 +53,8 @@ struct FwdLaunch {
 cudaError_t launch_attn_fwd(const FwdLaunch& a, cudaStream_t stream);
 
 // Backward preprocess into the per-head layout the backward kernel streams:
-// delta_t/lse2_t [n_ranks*B*Hq_l][Lp] (Lp = L rounded up to 128), lse2 = LSE*log2(e).
+// delta_t/lse2_t [n_ranks*B*Hq_l][Lp] (Lp = L rounded up to 128), holding -Delta
+// and -LSE*log2(e); padding rows hold 0 and -inf.
 cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* lse, float* delta_t, float* lse2_t,
                                  int n_rb, int L, int Hl, int D, int Lp, cudaStream_t stream);
 
