@@ -101,8 +101,8 @@ int usp_head2seq_permute(const void* src, void* dst, int B, int S, int H, int D,
  * usp_attn_bwd (bwd = 1). Returns 0 for an unsupported shape.
  *   fused fwd   : 256 (status word)
  *   stepwise fwd: 256 + P_r * B*S*Hq * (4*D + 4)  (fp32 partials of every ring step)
- *   bwd         : 256 + B*S*Hq*4*D + 2 * 4 * B*P_u*P_r*(Hq/P_u)*Lp, Lp = S/P_r rounded up
- *                 to a multiple of 128 (fp32 dQ accumulator; LSE*log2(e) and Delta per head)
+ *   bwd         : 256 + 2 * 4 * B*P_u*P_r*(Hq/P_u)*Lp, Lp = S/P_r rounded up to a
+ *                 multiple of 128 (-LSE*log2(e) and -Delta per head and row)
  */
 size_t usp_attn_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, int mode,
                                int bwd);
@@ -135,7 +135,8 @@ int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
  * dK = scale dS^T Q, dV = P^T dO, dK/dV summed over the q-heads of a GQA group.
  *   q, out, dO   head-sharded bf16 (out is the forward output)
  *   lse          the forward LSE
- *   dQ           head-sharded bf16 (accumulated in fp32 in the workspace)
+ *   dQ           head-sharded bf16 (accumulated in fp32 in TMEM by a query-major
+ *                kernel; dK/dV come from a key-major kernel)
  *   dK, dV       head-sharded fp32, [P_r][P_u][B][L][Hkv/P_u][D]
  */
 int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dO,

@@ -117,24 +117,6 @@ int make_tmap(CUtensorMap* m, const void* base, int D, int H_l, int L, int n_rb)
   return USP_OK;
 }
 
-// fp32 dQ accumulator [n_rb][L][H_l][D] as 4-D {D, H_l, L, n_rb}; box = 32 fp32 (128 B) x 1 x 32 rows x 1,
-// 128-byte swizzle (the staging layout of the backward's reduce-add).
-int make_tmap_dq(CUtensorMap* m, const void* base, int D, int H_l, int L, int n_rb) {
-  auto fn = encode_fn();
-  if (!fn) return fail(USP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H_l), static_cast<cuuint64_t>(L),
-                        static_cast<cuuint64_t>(n_rb)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(H_l) * D * 4,
-                           static_cast<cuuint64_t>(L) * H_l * D * 4};
-  cuuint32_t box[4] = {32, 1, 32, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(USP_ERR_CUDA, "cuTensorMapEncodeTiled (dQ) failed (%d)", static_cast<int>(r));
-  return USP_OK;
-}
-
 size_t rows_of(const AttnGeom& g) { return static_cast<size_t>(g.B) * g.S * g.Hq; }
 
 size_t fwd_ws(const AttnGeom& g, int mode) {
@@ -142,10 +124,10 @@ size_t fwd_ws(const AttnGeom& g, int mode) {
   return kStatusBytes + static_cast<size_t>(g.P_r) * rows_of(g) * (4 * static_cast<size_t>(g.D) + 4);
 }
 int padded_L(const AttnGeom& g) { return (g.L + 127) / 128 * 128; }
-// [status][dQ fp32 accumulator: rows*D][LSE*log2e per head: n_rb*Hq_l*Lp][Delta per head: same]
+// [status][-LSE*log2e per head: n_rb*Hq_l*Lp][-Delta per head: same]
 size_t bwd_ws(const AttnGeom& g) {
   const size_t per_head = static_cast<size_t>(g.n_ranks) * g.B * g.Hq_l * padded_L(g);
-  return kStatusBytes + rows_of(g) * 4 * static_cast<size_t>(g.D) + 2 * per_head * 4;
+  return kStatusBytes + 2 * per_head * 4;
 }
 
 }  // namespace
@@ -253,11 +235,9 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   if (!workspace || ws_bytes < need || !aligned16(workspace))
     return fail(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t rows = rows_of(g);
   const int Lp = padded_L(g);
   const size_t per_head = static_cast<size_t>(g.n_ranks) * B * g.Hq_l * Lp;
-  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
-  float* lse2 = dq_acc + rows * D;
+  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
   float* delta = lse2 + per_head;
   BwdLaunch L{};
   L.g = g;
@@ -265,24 +245,22 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   if ((rc = make_tmap(&L.tm_k, k, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   if ((rc = make_tmap(&L.tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   if ((rc = make_tmap(&L.tm_do, dO, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
-  if ((rc = make_tmap_dq(&L.tm_dq, dq_acc, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   L.lse2 = lse2;
   L.delta = delta;
   L.Lp = Lp;
-  L.dq_acc = dq_acc;
+  L.dq = dQ;
   L.dk = dK;
   L.dv = dV;
   L.status = static_cast<int*>(workspace);
   L.wait_ns = g_wait_ns;
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dq_acc, 0, rows * D * sizeof(float), st);
   if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
   e = launch_bwd_prep_rows(out, dO, lse, delta, lse2, g.n_ranks * B, g.L, g.Hq_l, D, Lp, st);
   if (e != cudaSuccess) return cuda_fail(e, "preprocess launch");
   e = launch_attn_bwd(L, st);
-  if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");
-  e = launch_f32_to_bf16(dq_acc, dQ, static_cast<long long>(rows) * D, 1.0f / sqrtf(static_cast<float>(D)), st);
-  return e == cudaSuccess ? USP_OK : cuda_fail(e, "dQ conversion launch");
+  if (e != cudaSuccess) return cuda_fail(e, "attention backward (dK, dV) launch");
+  e = launch_attn_bwd_dq(L, st);
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention backward (dQ) launch");
 }
 
 int usp_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,

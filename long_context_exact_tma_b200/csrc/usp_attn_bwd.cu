@@ -1,33 +1,30 @@
-// usp_attn_bwd.cu -- backward of the blockwise USP attention on sm_100a.
+// usp_attn_bwd.cu -- backward of the blockwise USP attention on sm_100a: the
+// key-major half (dK, dV). The query-major half (dQ) is usp_attn_bwd_dq.cu.
 //
 // What it computes (the gradient of the forward's exact attention; the pages
 // give no formula, these are the derivatives of softmax attention): with P
 // recomputed from the forward's final merged LSE,
 //   P_ij = exp(scale q_i.k_j - LSE_i),   dP = dO V^T,   Delta_i = sum_d dO_id O_id,
-//   dS = scale * P o (dP - Delta),        dQ = dS K,   dK = dS^T Q,   dV = P^T dO
-// (the scale is applied once, to dK in the epilogue and to dQ in its conversion),
+//   dS = P o (dP - Delta),   dK = scale dS^T Q,   dV = P^T dO,
 // with dK/dV summed over the q-heads of a GQA group and over every ring rank's
 // queries (in the ring algorithm dK/dV travel around the ring with K/V).
 //
 // CTA = one 128-key tile of one kv-head of one head-sharded rank (the ring's KV
 // chunk owner); it walks the q-heads of the group, the ring ranks whose queries
 // see the tile and their 128-row query tiles ("steps"). 320 threads:
-//   warp 0      TMA: K, V once; per step Q, dO (2 stages) and 128 LSE/Delta values.
+//   warp 0      TMA: K, V once; per step Q, dO (2 stages) and 128 LSE/Delta values;
+//               it alone walks the steps and publishes one descriptor per step.
 //   warp 1      TMEM allocator + UMMA issuer, per step k:
-//                 S^T  = K Q^T      -> TMEM [0,128)     (M = keys, N = queries)
-//                 dP^T = V dO^T     -> TMEM [128,256)
-//                 dV  += P^T dO     -> TMEM [256,256+D) (A = P^T read from TMEM)
-//                 dK  += dS^T Q     -> TMEM [384,384+D) (A = dS^T from shared memory)
-//                 dQt  = dS K       -> TMEM [128,128+D) (A = dS: MN-major view of dS^T)
-//               S^T of step k+1 is issued once step k's UMMAs have completed and
-//               dP^T of step k+1 once the dQ tile of step k has been read out.
+//                 S^T  = K Q^T     -> TMEM [0,128)     (M = keys, N = queries)
+//                 dP^T = V dO^T    -> TMEM [128,256)
+//                 dV  += P^T dO    -> TMEM [256,256+D) (A = P^T read from TMEM)
+//                 dK  += dS^T Q    -> TMEM [384,384+D) (A = dS^T read from TMEM)
+//               S^T / dP^T of step k+1 are issued as soon as the UMMAs that read
+//               P^T / dS^T from those columns have completed.
 //   warps 2..9  two warpgroups; warpgroup c owns query columns [64c, 64c+64).
-//               Thread = key row: P^T (bf16, packed back into TMEM over the S^T
-//               columns it has read) and dS^T (bf16, 128B-swizzled shared memory).
-//               Then thread = query row: the dQ tile is read from TMEM, staged in
-//               the step's (now free) Q/dO buffers and added to the fp32 dQ
-//               accumulator with TMA bulk reduce-add (cp.reduce.async.bulk.tensor).
-//               At the end dK and dV rows (fp32) are written out.
+//               Thread = key row: P^T and dS^T as bf16, packed back into TMEM
+//               over the S^T / dP^T columns they came from. At the end dK and dV
+//               rows (fp32) are written out.
 // Every wait is bounded (usp_ptx.cuh).
 #include <math.h>
 
@@ -42,7 +39,6 @@ constexpr int kThreadsBwd = 320;
 constexpr int kComputeThreads = 256;
 constexpr uint32_t kTmemColsBwd = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
-constexpr uint32_t kColDQ = kColDP;  // the dQ tile reuses the dP^T columns
 
 template <int D>
 struct BwdCfg {
@@ -54,12 +50,10 @@ struct BwdCfg {
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;
   static constexpr int kOffDO = kOffQ + kStages * kTileBytes;
-  static constexpr int kOffDSt = kOffDO + kStages * kTileBytes;  // dS^T: 128 keys x 128 queries bf16
-  static constexpr int kOffRow = kOffDSt + 2 * kPanelBytes;      // per stage: LSE*log2e [128], Delta [128]
+  static constexpr int kOffRow = kOffDO + kStages * kTileBytes;  // per stage: -LSE*log2e [128], -Delta [128]
   static constexpr int kOffBar = kOffRow + kStages * 1024;
   // No alignment slack: the kernel requires (and checks) a 1024-byte aligned dynamic shared memory base.
   static constexpr int kSmemBytes = kOffBar + 256;
-  static constexpr int kBoxesPerWarp = D / 64;  // 32x32 fp32 dQ boxes one compute warp stages per step
 };
 
 struct BwdArgs {
@@ -76,7 +70,7 @@ struct BwdArgs {
 struct BwdBars {
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
-  uint64_t st_full, p_full, p_used, dq_full, dq_free, drain;
+  uint64_t st_full, p_full, p_used, ds_used, drain;
   // Step descriptors published by the producer with qd_full of that step:
   // {q-head in group (-1 = no more steps), ring rank i, query tile m, tile kind}.
   int step[4][4];
@@ -85,8 +79,8 @@ struct BwdBars {
 };
 
 enum : int {
-  kSiteBKv = 0x201, kSiteBQdEmpty = 0x202, kSiteBQd = 0x211, kSiteBDqFree = 0x212, kSiteBP = 0x213,
-  kSiteBPUsed = 0x214, kSiteBSt = 0x221, kSiteBDq = 0x222, kSiteBQdC = 0x223, kSiteBAlign = 0x2FF
+  kSiteBKv = 0x201, kSiteBQdEmpty = 0x202, kSiteBQd = 0x211, kSiteBDsUsed = 0x212, kSiteBP = 0x213,
+  kSiteBPUsed = 0x214, kSiteBSt = 0x221, kSiteBQdC = 0x223, kSiteBEpi = 0x224, kSiteBAlign = 0x2FF
 };
 
 // Query steps of one key tile: q-head hh of the group, ring rank i, query tile m.
@@ -141,7 +135,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
+                    const BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_addr(smem_raw) & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -155,7 +149,6 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sDO = smem + C::kOffDO;
-  uint8_t* sDSt = smem + C::kOffDSt;
   float* sRow = reinterpret_cast<float*>(smem + C::kOffRow);
 
   const Geo& g = a.g;
@@ -183,13 +176,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars->qd_full[s], 1);
-      mbar_init(&bars->qd_empty[s], kComputeThreads / 32);
+      mbar_init(&bars->qd_empty[s], 1);
     }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->p_full, kComputeThreads);
     mbar_init(&bars->p_used, 1);
-    mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_free, kComputeThreads);
+    mbar_init(&bars->ds_used, 1);
     mbar_init(&bars->drain, 1);
     fence_mbar_init();
   }
@@ -260,9 +252,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     if (lane == 0) {
       constexpr uint32_t kIdSS = idesc_bf16_f32(128, 128, 0, 0);  // both K-major
       constexpr uint32_t kIdKM = idesc_bf16_f32(128, D, 0, 1);    // A K-major, B MN-major
-      constexpr uint32_t kIdMM = idesc_bf16_f32(128, D, 1, 1);    // both MN-major
       const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ), aDO = smem_addr(sDO);
-      const uint32_t aDSt = smem_addr(sDSt);
       auto issue_s = [&](int s) {  // S^T = K Q^T
         const uint32_t qb = aQ + s * C::kTileBytes;
 #pragma unroll
@@ -301,36 +291,32 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (!mbar_wait(&bars->p_full, k & 1, w, kSiteBP)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qb = aQ + s * C::kTileBytes, db = aDO + s * C::kTileBytes;
+        // P^T and dS^T live in TMEM: warpgroup c packed its 64 queries at columns 64c .. 64c+31
+        // of the S^T (P^T) and dP^T (dS^T) blocks.
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk) {  // dV += P^T dO, K = 128 queries
-          // P^T lives in TMEM: warpgroup c packed its 64 queries at columns 64c .. 64c+31
-          const uint32_t pcol = kColS + (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
-          umma_bf16_tmem_a(tmem + kColDV, tmem + pcol, sdesc_sw128(db + kk * 16 * 128, C::kPanelBytes, 1024),
+          const uint32_t pcol = (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
+          umma_bf16_tmem_a(tmem + kColDV, tmem + kColS + pcol, sdesc_sw128(db + kk * 16 * 128, C::kPanelBytes, 1024),
                            kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->p_used);  // P^T (in the S^T columns) has been read once this lands
+        umma_commit(&bars->p_used);
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk) {  // dK += dS^T Q, K = 128 queries
-          const uint32_t aoff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_bf16(tmem + kColDK, sdesc_sw128(aDSt + aoff, 16, 1024),
-                    sdesc_sw128(qb + kk * 16 * 128, C::kPanelBytes, 1024), kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t pcol = (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
+          umma_bf16_tmem_a(tmem + kColDK, tmem + kColDP + pcol, sdesc_sw128(qb + kk * 16 * 128, C::kPanelBytes, 1024),
+                           kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
         }
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {  // dQt = dS K, K = 128 keys
-          const uint32_t off = kk * 16 * 128;
-          umma_bf16(tmem + kColDQ, sdesc_sw128(aDSt + off, C::kPanelBytes, 1024),
-                    sdesc_sw128(aK + off, C::kPanelBytes, 1024), kIdMM, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars->dq_full);
+        umma_commit(&bars->ds_used);
+        umma_commit(&bars->qd_empty[s]);  // this step's Q/dO stage is free once these UMMAs land
         const int s1 = (k + 1) % C::kStages;
         if (!mbar_wait(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
         have = bars->step[(k + 1) & 3][0] >= 0;
         if (!have) break;
-        // S^T of the next step overwrites the columns P^T is read from: wait for the dV UMMAs only.
+        // the next S^T / dP^T overwrite the columns P^T / dS^T are read from
         if (!mbar_wait(&bars->p_used, k & 1, w, kSiteBPUsed)) { ok = false; break; }
         tc_fence_after();
         issue_s(s1);
-        if (!mbar_wait(&bars->dq_free, k & 1, w, kSiteBDqFree)) { ok = false; break; }
+        if (!mbar_wait(&bars->ds_used, k & 1, w, kSiteBDsUsed)) { ok = false; break; }
         tc_fence_after();
         issue_dp(s1);
         umma_commit(&bars->st_full);
@@ -420,66 +406,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           pk[c >> 1] = pack_bf16x2(pv.x, pv.y);
           dk[c >> 1] = pack_bf16x2(ds.x, ds.y);
         }
-        // P^T back into TMEM (columns already read by this thread), 2 bf16 per column
+        // P^T and dS^T back into TMEM over the S^T / dP^T columns this thread has read
         tmem_st16(trow + kColS + cbase + half * 16, pk);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = (c0 >> 3) + q;  // 16-byte chunk index along the 128 queries
-          const uint32_t off = (ch >> 3) * C::kPanelBytes + sw128_offset(row, ch & 7);
-          *reinterpret_cast<uint4*>(sDSt + off) = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
-        }
+        tmem_st16(trow + kColDP + cbase + half * 16, dk);
       }
       tmem_st_wait();
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->p_full);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, k & 1, w, kSiteBDq));
-      if (!ok) break;
-      tc_fence_after();
-      // dQ tile: this thread's query row, columns [wg*D/2, wg*D/2 + D/2)
-      uint32_t rq[C::kBoxesPerWarp][32];
-#pragma unroll
-      for (int q = 0; q < C::kBoxesPerWarp; ++q) tmem_ld32(trow + kColDQ + wg * (D / 2) + q * 32, rq[q]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < C::kBoxesPerWarp; ++q) reg_fence32(rq[q]);
-      tc_fence_before();
-      mbar_arrive(&bars->dq_free);
-      // stage 32x32 fp32 boxes in this step's Q/dO buffers (free: the step's UMMAs are done)
-      const int h = gl * g.G + st_hh;
-      const int qrb = (st_i * g.P_u + u) * g.B + b;
-      const int box_row = q0 + wq * 32;
-#pragma unroll
-      for (int q = 0; q < C::kBoxesPerWarp; ++q) {
-        const int box = (wg * C::kBoxesPerWarp + q) * 4 + wq;
-        uint8_t* base = box < D / 16 ? sQ + s * C::kTileBytes + box * 4096
-                                     : sDO + s * C::kTileBytes + (box - D / 16) * 4096;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(base + sw128_offset(lane, ch)) =
-              make_uint4(rq[q][4 * ch], rq[q][4 * ch + 1], rq[q][4 * ch + 2], rq[q][4 * ch + 3]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        if (box_row < g.L) {
-#pragma unroll
-          for (int q = 0; q < C::kBoxesPerWarp; ++q) {
-            const int box = (wg * C::kBoxesPerWarp + q) * 4 + wq;
-            const uint8_t* base = box < D / 16 ? sQ + s * C::kTileBytes + box * 4096
-                                               : sDO + s * C::kTileBytes + (box - D / 16) * 4096;
-            tma_reduce_add_4d(&tm_dq, base, wg * (D / 2) + q * 32, h, box_row, qrb);
-          }
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        mbar_arrive(&bars->qd_empty[s]);
-      }
-      __syncwarp();
     }
-    if (lane == 0) bulk_wait_group0();  // this warp's reduce-adds have landed in global memory
-    __syncwarp();
     // ------------------------------------------------------------ dK, dV epilogue
+    // the last step's dK/dV UMMAs (and every earlier one) have landed once its ds_used arrives
+    if (ok && k >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars->ds_used, (k - 1) & 1, w, kSiteBEpi));
     if (ok) {
       tc_fence_after();
       const bool store = tau_k < g.L;
@@ -541,7 +478,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   attn_bwd_kernel<D><<<static_cast<unsigned>(blocks), kThreadsBwd, C::kSmemBytes, stream>>>(
-      L.tm_q, L.tm_k, L.tm_v, L.tm_do, L.tm_dq, a);
+      L.tm_q, L.tm_k, L.tm_v, L.tm_do, a);
   return cudaGetLastError();
 }
 

@@ -61,16 +61,16 @@ cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* l
 struct BwdLaunch {
   AttnGeom g;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
-  CUtensorMap tm_dq;   // fp32 dQ accumulator, box 32 x 1 x 32 rows (TMA reduce-add target)
-  const float* lse2;   // [n_ranks*B*Hq_l][Lp]
-  const float* delta;  // [n_ranks*B*Hq_l][Lp]
+  const float* lse2;   // [n_ranks*B*Hq_l][Lp]: -LSE*log2(e), -inf on padding rows
+  const float* delta;  // [n_ranks*B*Hq_l][Lp]: -Delta, 0 on padding rows
   int Lp;
-  float* dq_acc;       // fp32, q layout
+  void* dq;            // bf16, q layout (written by the query-major kernel)
   float* dk;           // fp32, k layout
   float* dv;           // fp32, v layout
   int* status;
   unsigned long long wait_ns;
 };
-cudaError_t launch_attn_bwd(const BwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_attn_bwd(const BwdLaunch& a, cudaStream_t stream);     // dK, dV (key-major)
+cudaError_t launch_attn_bwd_dq(const BwdLaunch& a, cudaStream_t stream);  // dQ (query-major)
 
 }  // namespace usp

@@ -44,8 +44,8 @@ def test_workspace_size_queries():
     rows = 1 * 256 * 2
     assert ws(1, 256, 2, 2, 64, 1, 2, 2, 1, 0) == 256 + 2 * rows * (4 * 64 + 4)
     Lp = 128  # S/P_r = 128 already a multiple of 128
-    assert ws(1, 256, 2, 2, 64, 1, 2, 2, 0, 1) == 256 + rows * 4 * 64 + 2 * 4 * (4 * 1 * 1 * Lp)
-    assert ws(1, 600, 2, 2, 64, 1, 1, 1, 0, 1) == 256 + 1200 * 4 * 64 + 2 * 4 * (1 * 2 * 640)
+    assert ws(1, 256, 2, 2, 64, 1, 2, 2, 0, 1) == 256 + 2 * 4 * (4 * 1 * 1 * Lp)
+    assert ws(1, 600, 2, 2, 64, 1, 1, 1, 0, 1) == 256 + 2 * 4 * (1 * 2 * 640)
     assert ws(1, 256, 2, 2, 96, 1, 2, 2, 0, 0) == 0      # D unsupported
     assert ws(1, 250, 2, 2, 64, 1, 2, 2, 0, 0) == 0      # S % 2P != 0
     assert ws(1, 256, 3, 2, 64, 1, 1, 1, 0, 0) == 0      # Hq % Hkv != 0
@@ -86,7 +86,7 @@ def test_fwd_rejects_bad_arguments(kw, code):
 def test_bwd_rejects_bad_arguments():
     L = B_.lib()
     args = [FAKE] * 9 + [1, 256, 2, 2, 64, 1, 2, 2, FAKE, 256, None]
-    assert L.usp_attn_bwd(*args) == B_.USP_ERR_WORKSPACE  # needs rows*(4D+4) bytes
+    assert L.usp_attn_bwd(*args) == B_.USP_ERR_WORKSPACE  # needs the per-head LSE/Delta tables
     bad = list(args)
     bad[13] = 48  # D
     assert L.usp_attn_bwd(*bad) == B_.USP_ERR_UNSUPPORTED

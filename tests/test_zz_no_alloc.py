@@ -45,9 +45,13 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls(cuda):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda):
-    # B=1, S=65536, H=32, D=128 needs ~1 GiB of scratch, far beyond the static 32 MiB
+    # The call below passes placeholder buffers, so it must be rejected before any
+    # launch: check first that this shape's scratch really exceeds the static array.
+    B, S, H, D = 4, 262144, 32, 128
+    need = B_.usp_attn_workspace_size(B, S, H, H, D, 1, 1, 1, 0, 1)
+    assert need > (32 << 20), need
     big = torch.empty(16, dtype=torch.uint8, device=cuda)
-    rc = B_.usp_attn_bwd_noalloc(big, big, big, big, big, big, big, big, big, 1, 65536, 32, 32, 128, 1, 1, 1,
+    rc = B_.usp_attn_bwd_noalloc(big, big, big, big, big, big, big, big, big, B, S, H, H, D, 1, 1, 1,
                                  check=False)
     assert rc == B_.USP_ERR_WORKSPACE
     msg = B_.usp_last_error()
