@@ -3,7 +3,6 @@
 //     partial (O_t, LSE_t) of its queries; "Boosting Spec Eagle", "The Solution",
 //     Ring Attention),
 //   * backward preprocess Delta_i = sum_d dO_id O_id,
-//   * fp32 -> bf16 conversion of the dQ accumulator,
 //   * the bounded-wait self-test kernel.
 #include <math.h>
 
@@ -135,18 +134,6 @@ __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16*
   }
 }
 
-__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
-                                                          long long n4, float scale) {
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
-    const float4 v = __ldcs(src + i);
-    uint2 p;
-    p.x = pack_bf16x2(v.x * scale, v.y * scale);
-    p.y = pack_bf16x2(v.z * scale, v.w * scale);
-    __stcs(dst + i, p);
-  }
-}
-
 // Waits on an mbarrier that nothing completes; the bounded wait must give up.
 __global__ void wait_selftest_kernel(int* status, unsigned long long limit_ns) {
   __shared__ uint64_t bar;
@@ -206,14 +193,6 @@ cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* l
   bwd_prep_rows_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
                                                               static_cast<const __nv_bfloat16*>(dO), lse, delta_t,
                                                               lse2_t, rows, L, Hl, D, Lp);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, float scale, cudaStream_t stream) {
-  if (n == 0) return cudaSuccess;
-  const long long n4 = n / 4;  // callers pass multiples of 4 (D is 64 or 128)
-  f32_to_bf16_kernel<<<grid_for(256, n4), 256, 0, stream>>>(reinterpret_cast<const float4*>(src),
-                                                            static_cast<uint2*>(dst), n4, scale);
   return cudaGetLastError();
 }
 

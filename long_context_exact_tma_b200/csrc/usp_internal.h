@@ -28,8 +28,6 @@ cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n
                              void* out, int out_f32, float* lse_out, cudaStream_t stream);
 cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D,
                                   cudaStream_t stream);
-// dst = bf16(src * scale), n a multiple of 4.
-cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, float scale, cudaStream_t stream);
 cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
 
 // Geometry of one attention problem in the head-sharded layout.
