@@ -39,7 +39,7 @@ from usp_inputs import WORKLOADS, workload  # noqa: E402
 
 METRIC = "attention TFLOP/s fwd+bwd at S=16K-256K; % of bf16 dense tensor peak"
 UNIT = "TFLOP/s"
-LAUNCHES_PER_STEP = 12  # 3 seq2head + fwd + head2seq(O) + seq2head(dO) + prep + bwd + dQ convert + 3 head2seq
+LAUNCHES_PER_STEP = 12  # 3 seq2head + fwd + head2seq(O) + seq2head(dO) + prep + dK/dV + dQ + 3 head2seq
 
 
 def flops_fwd(w) -> float:
@@ -195,10 +195,21 @@ class Step:
             ev["fwd"][1].record(st)
         api.head2seq(self.out, P_u, P_r, out=self.o_rm)
         api.seq2head(self.rm["do"], P_u, P_r, out=self.hs["do"])
+        # backward = prepare + key-major dK/dV kernel + query-major dQ kernel (what
+        # usp_attn_bwd runs), called phase by phase so the dK/dV kernel is timed alone
+        geo = (w["B"], w["S"], w["Hq"], w["Hkv"], w["D"], causal, P_u, P_r)
+        B_, ws_b = self.B_, self.ws_b
         if ev:
             ev["bwd"][0].record(st)
-        api.attn_bwd(self.hs["q"], self.hs["k"], self.hs["v"], self.out, self.lse, self.hs["do"], causal, P_u, P_r,
-                     ws=self.ws_b, dq=self.dq, dk=self.dk, dv=self.dv)
+        B_.usp_attn_bwd_prepare(self.out, self.lse, self.hs["do"], *geo, ws_b, ws_b.numel(), st)
+        if ev:
+            ev["dkdv"][0].record(st)
+        B_.usp_attn_bwd_dkdv(self.hs["q"], self.hs["k"], self.hs["v"], self.hs["do"], self.dk, self.dv, *geo,
+                             ws_b, ws_b.numel(), st)
+        if ev:
+            ev["dkdv"][1].record(st)
+        B_.usp_attn_bwd_dq(self.hs["q"], self.hs["k"], self.hs["v"], self.hs["do"], self.dq, *geo,
+                           ws_b, ws_b.numel(), st)
         if ev:
             ev["bwd"][1].record(st)
         api.head2seq(self.dq, P_u, P_r, out=self.dq_rm)
@@ -275,7 +286,7 @@ def bench_ours(args, w, world, rank, local):
     torch.cuda.synchronize()
     step.check_status()
     ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)] for k in ("fwd", "bwd")}
+              for _ in range(args.steps)] for k in ("fwd", "bwd", "dkdv")}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     with ClockSampler(local) as clk:
@@ -293,6 +304,7 @@ def bench_ours(args, w, world, rank, local):
     value = world * args.steps * f_step / (ms / 1e3) / 1e12
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["fwd"])
     bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["bwd"])
+    dkdv_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["dkdv"])
     # end to end: host buffers in, host buffers out, through the same C ABI calls
     h2d, d2h = step.host_io()
     for _ in range(2):
@@ -310,6 +322,9 @@ def bench_ours(args, w, world, rank, local):
     if rank != 0:
         return None
     bwd_tf = 2.5 * f_fwd / (bwd_ms / 1e3) / 1e12
+    # dominant kernel: the key-major dK/dV kernel, whose algorithmic work is its four
+    # GEMMs per (key tile, query tile) pair (S^T, dP^T, dV, dK) = 2 x the forward FLOPs
+    dkdv_tf = 2.0 * f_fwd / (dkdv_ms / 1e3) / 1e12
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -331,10 +346,10 @@ def bench_ours(args, w, world, rank, local):
         "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
         "fwd_tflops": round(f_fwd / (fwd_ms / 1e3) / 1e12, 2),
         "bwd_tflops": round(bwd_tf, 2),
-        "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel<128> (usp_attn_bwd call)",
-                     "achieved": round(bwd_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": round(bwd_tf / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
-                     "traffic": None},
+        "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel (key-major dK/dV; usp_attn_bwd_dkdv call)",
+                     "achieved": round(dkdv_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(dkdv_tf / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "launch_ms": round(dkdv_ms, 4), "traffic": args.dkdv_traffic},
         "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
@@ -386,6 +401,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dkdv-traffic", type=float, default=None,
+                    help="DRAM bytes per dK/dV launch from an ncu capture of this exact kernel, if current")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warmup raised to the minimum of 3", file=sys.stderr)

@@ -144,6 +144,27 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
                  int P_r, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * The three phases of usp_attn_bwd, callable on their own (same arguments and
+ * layouts; the workspace is the one usp_attn_bwd takes):
+ *   usp_attn_bwd_prepare  clears the status word and fills the workspace with
+ *                         -Delta_i = -sum_d dO_id O_id and -LSE_i*log2(e) per head
+ *                         (padding rows: 0 and -inf);
+ *   usp_attn_bwd_dkdv     key-major kernel: dK = scale dS^T Q, dV = P^T dO, summed
+ *                         over the GQA group and every ring rank's queries;
+ *   usp_attn_bwd_dq       query-major kernel: dQ = scale dS K over every ring step,
+ *                         accumulated on chip and written once as bf16.
+ * dkdv and dq read only the prepared workspace and the inputs, so they may run in
+ * either order (or on two streams) after prepare.
+ */
+int usp_attn_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,
+                         int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream);
+int usp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, float* dK, float* dV, int B,
+                      int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes,
+                      void* stream);
+int usp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dQ, int B, int S, int Hq,
+                    int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Bytes of the static device scratch behind usp_attn_bwd_noalloc (32 MiB).
  */
 #define USP_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

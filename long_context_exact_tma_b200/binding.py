@@ -41,6 +41,9 @@ SIGNATURES = {
     "usp_attn_workspace_size": (_SZ, [_I] * 10),
     "usp_attn_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_P, _SZ, _P]),
     "usp_attn_bwd": (_I, [_P] * 9 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_attn_bwd_prepare": (_I, [_P, _P, _P] + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_attn_bwd_dkdv": (_I, [_P] * 6 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_attn_bwd_dq": (_I, [_P] * 5 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 8 + [_P]),
     "usp_lse_merge": (_I, [_P, _P, _I, _LL, _I, _P, _I, _P, _P]),
     "usp_bwd_preprocess": (_I, [_P, _P, _P, _LL, _I, _P]),
@@ -140,6 +143,27 @@ def usp_attn_bwd(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_
     rc = lib().usp_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
                             _ptr(dV), B, S, Hq, Hkv, D, int(causal), P_u, P_r, _ptr(workspace), ws_bytes,
                             _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_attn_bwd_prepare(out, lse, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream=None,
+                         check=True):
+    rc = lib().usp_attn_bwd_prepare(_ptr(out), _ptr(lse), _ptr(dO), B, S, Hq, Hkv, D, int(causal), P_u, P_r,
+                                    _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_attn_bwd_dkdv(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream=None,
+                      check=True):
+    rc = lib().usp_attn_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dK), _ptr(dV), B, S, Hq, Hkv, D,
+                                 int(causal), P_u, P_r, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_attn_bwd_dq(q, k, v, dO, dQ, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream=None,
+                    check=True):
+    rc = lib().usp_attn_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dQ), B, S, Hq, Hkv, D, int(causal),
+                               P_u, P_r, _ptr(workspace), ws_bytes, _stream(stream))
     return _check(rc) if check else rc
 
 

@@ -221,6 +221,84 @@ int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
   return e == cudaSuccess ? USP_OK : cuda_fail(e, "merge launch");
 }
 
+int usp_attn_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,
+                         int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream) {
+  AttnGeom g{};
+  int rc = check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
+  if (rc != USP_OK) return rc;
+  if (!out || !lse || !dO) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(out) || !aligned16(lse) || !aligned16(dO))
+    return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t need = bwd_ws(g);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return fail(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int Lp = padded_L(g);
+  const size_t per_head = static_cast<size_t>(g.n_ranks) * B * g.Hq_l * Lp;
+  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+  float* delta = lse2 + per_head;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+  e = launch_bwd_prep_rows(out, dO, lse, delta, lse2, g.n_ranks * B, g.L, g.Hq_l, D, Lp, st);
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "preprocess launch");
+}
+
+namespace {
+// Validation and TMA maps shared by the two backward kernels (workspace prepared
+// by usp_attn_bwd_prepare).
+int bwd_launch_setup(const void* q, const void* k, const void* v, const void* dO, int B, int S, int Hq, int Hkv,
+                     int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, BwdLaunch* L) {
+  AttnGeom g{};
+  int rc = check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
+  if (rc != USP_OK) return rc;
+  if (!q || !k || !v || !dO) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO))
+    return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t need = bwd_ws(g);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return fail(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  const int Lp = padded_L(g);
+  const size_t per_head = static_cast<size_t>(g.n_ranks) * B * g.Hq_l * Lp;
+  L->g = g;
+  if ((rc = make_tmap(&L->tm_q, q, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L->tm_k, k, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L->tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  if ((rc = make_tmap(&L->tm_do, dO, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
+  L->lse2 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + kStatusBytes);
+  L->delta = L->lse2 + per_head;
+  L->Lp = Lp;
+  L->status = static_cast<int*>(workspace);
+  L->wait_ns = g_wait_ns;
+  return USP_OK;
+}
+}  // namespace
+
+int usp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, float* dK, float* dV, int B,
+                      int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes,
+                      void* stream) {
+  if (!dK || !dV) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(dK) || !aligned16(dV)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  BwdLaunch L{};
+  const int rc = bwd_launch_setup(q, k, v, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, &L);
+  if (rc != USP_OK) return rc;
+  L.dk = dK;
+  L.dv = dV;
+  const cudaError_t e = launch_attn_bwd(L, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention backward (dK, dV) launch");
+}
+
+int usp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dQ, int B, int S, int Hq,
+                    int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream) {
+  if (!dQ) return fail(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(dQ)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  BwdLaunch L{};
+  const int rc = bwd_launch_setup(q, k, v, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, &L);
+  if (rc != USP_OK) return rc;
+  L.dq = dQ;
+  const cudaError_t e = launch_attn_bwd_dq(L, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention backward (dQ) launch");
+}
+
 int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dO,
                  void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D, int causal, int P_u,
                  int P_r, void* workspace, size_t ws_bytes, void* stream) {
@@ -231,36 +309,13 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dO) ||
       !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
     return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const size_t need = bwd_ws(g);
-  if (!workspace || ws_bytes < need || !aligned16(workspace))
-    return fail(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int Lp = padded_L(g);
-  const size_t per_head = static_cast<size_t>(g.n_ranks) * B * g.Hq_l * Lp;
-  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
-  float* delta = lse2 + per_head;
-  BwdLaunch L{};
-  L.g = g;
-  if ((rc = make_tmap(&L.tm_q, q, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
-  if ((rc = make_tmap(&L.tm_k, k, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
-  if ((rc = make_tmap(&L.tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
-  if ((rc = make_tmap(&L.tm_do, dO, D, g.Hq_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
-  L.lse2 = lse2;
-  L.delta = delta;
-  L.Lp = Lp;
-  L.dq = dQ;
-  L.dk = dK;
-  L.dv = dV;
-  L.status = static_cast<int*>(workspace);
-  L.wait_ns = g_wait_ns;
-  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
-  if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
-  e = launch_bwd_prep_rows(out, dO, lse, delta, lse2, g.n_ranks * B, g.L, g.Hq_l, D, Lp, st);
-  if (e != cudaSuccess) return cuda_fail(e, "preprocess launch");
-  e = launch_attn_bwd(L, st);
-  if (e != cudaSuccess) return cuda_fail(e, "attention backward (dK, dV) launch");
-  e = launch_attn_bwd_dq(L, st);
-  return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention backward (dQ) launch");
+  if ((rc = usp_attn_bwd_prepare(out, lse, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream)) !=
+      USP_OK)
+    return rc;
+  if ((rc = usp_attn_bwd_dkdv(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes,
+                              stream)) != USP_OK)
+    return rc;
+  return usp_attn_bwd_dq(q, k, v, dO, dQ, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream);
 }
 
 int usp_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,

@@ -117,3 +117,26 @@ def test_bwd_ignores_stale_workspace_contents(cuda):
     for a_, b_ in zip(clean, dirty):
         assert torch.isfinite(b_.float()).all()
         assert rel_l2(b_.double().cpu().numpy(), a_.double().cpu().numpy()) <= 1e-5
+
+
+def test_bwd_phases_compose_to_usp_attn_bwd(cuda):
+    """prepare, then the dQ kernel before the dK/dV kernel, gives bit for bit what
+    usp_attn_bwd gives (both kernels only read the prepared workspace)."""
+    from long_context_exact_tma_b200 import binding as B_
+    spec = make_spec(S=1536, Hq=8, Hkv=2, D=128, P_u=2, P_r=2, seed=309)
+    t = inputs(spec, which=("q", "k", "v", "do"))
+    P_u, P_r = spec["P_u"], spec["P_r"]
+    q, k, v, do = (head_shard_cpu(t[n], spec).to(cuda) for n in ("q", "k", "v", "do"))
+    out, lse = api.attn_fwd(q, k, v, True, P_u, P_r)
+    whole = api.attn_bwd(q, k, v, out, lse, do, True, P_u, P_r)
+    geo = (1, 1536, 8, 2, 128, 1, P_u, P_r)
+    need = B_.usp_attn_workspace_size(*geo, 0, 1)
+    ws = api.workspace(need, cuda)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(whole[1]), torch.empty_like(whole[2])
+    B_.usp_attn_bwd_prepare(out, lse, do, *geo, ws, need)
+    B_.usp_attn_bwd_dq(q, k, v, do, dq, *geo, ws, need)
+    B_.usp_attn_bwd_dkdv(q, k, v, do, dk, dv, *geo, ws, need)
+    torch.cuda.synchronize()
+    assert B_.usp_workspace_status(ws)[0] == 0
+    for a_, b_ in zip(whole, (dq, dk, dv)):
+        assert torch.equal(a_, b_)
