@@ -39,6 +39,30 @@ from usp_inputs import WORKLOADS, workload  # noqa: E402
 
 METRIC = "attention TFLOP/s fwd+bwd at S=16K-256K; % of bf16 dense tensor peak"
 UNIT = "TFLOP/s"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# dK/dV kernel on causal_fwd_s16k_ring8, from the ncu capture summarised in
+# profiles/attn_bwd_kernel_causal_fwd_s16k_ring8.md. Reported only while the
+# kernel's sources hash to what was captured (else the figure is stale: null).
+DKDV_TRAFFIC = {"workload": "causal_fwd_s16k_ring8", "bytes": None, "sources_sha256": None}
+DKDV_SOURCES = ("usp_attn_bwd.cu", "usp_attn_common.cuh", "usp_ptx.cuh", "usp_internal.h")
+
+
+def dkdv_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in DKDV_SOURCES:
+        with open(os.path.join(ROOT, "long_context_exact_tma_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def dkdv_traffic(workload_name: str):
+    rec = DKDV_TRAFFIC
+    if rec["bytes"] is None or workload_name != rec["workload"]:
+        return None
+    return rec["bytes"] if dkdv_sources_sha256() == rec["sources_sha256"] else None
+
+
 LAUNCHES_PER_STEP = 12  # 3 seq2head + fwd + head2seq(O) + seq2head(dO) + prep + dK/dV + dQ + 3 head2seq
 
 
@@ -70,7 +94,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
@@ -349,7 +373,7 @@ def bench_ours(args, w, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel (key-major dK/dV; usp_attn_bwd_dkdv call)",
                      "achieved": round(dkdv_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(dkdv_tf / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
-                     "launch_ms": round(dkdv_ms, 4), "traffic": args.dkdv_traffic},
+                     "launch_ms": round(dkdv_ms, 4), "traffic": dkdv_traffic(w["name"])},
         "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
@@ -394,15 +418,13 @@ def bench_reference(args, w, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--config", type=int, default=2, help="workload number (1-5), default the S=16K one")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--dkdv-traffic", type=float, default=None,
-                    help="DRAM bytes per dK/dV launch from an ncu capture of this exact kernel, if current")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warmup raised to the minimum of 3", file=sys.stderr)

@@ -61,21 +61,29 @@ struct WaitCtl {
 // Wait for the phase with parity `parity` of `bar` to complete. Returns false
 // when the CTA has aborted or when this wait ran past the limit (then it raises
 // the abort flag and records `site` in the status word).
+// The status word (a global load of several hundred cycles) and the timer are
+// read only every 32nd round, so that a phase completing is seen within one
+// try_wait and not after a global round trip.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w, int site) {
   const uint32_t a = smem_addr(bar);
   if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
+  uint64_t t0 = 0;
+  for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(a, parity)) return true;
     if (*w.abort_flag) return false;
-    if (*reinterpret_cast<volatile int*>(w.status) != 0) {  // another CTA already gave up
-      *w.abort_flag = 1;
-      return false;
-    }
-    if (global_timer_ns() - t0 > w.limit_ns) {
-      *w.abort_flag = 1;
-      atomicCAS(w.status, 0, site);
-      return false;
+    if ((n & 31u) == 0u) {
+      if (*reinterpret_cast<volatile int*>(w.status) != 0) {  // another CTA already gave up
+        *w.abort_flag = 1;
+        return false;
+      }
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > w.limit_ns) {
+        *w.abort_flag = 1;
+        atomicCAS(w.status, 0, site);
+        return false;
+      }
     }
   }
 }
