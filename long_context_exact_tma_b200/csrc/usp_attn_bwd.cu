@@ -16,15 +16,16 @@
 //               it alone walks the steps and publishes one descriptor per step.
 //   warp 1      TMEM allocator + UMMA issuer, per step k:
 //                 S^T  = K Q^T     -> TMEM [0,128)     (M = keys, N = queries)
-//                 dP^T = V dO^T    -> TMEM [128,256)
+//                 dP^T = V dO^T    -> TMEM [128,256)   (overlaps the P^T phase below)
 //                 dV  += P^T dO    -> TMEM [256,256+D) (A = P^T read from TMEM)
 //                 dK  += dS^T Q    -> TMEM [384,384+D) (A = dS^T read from TMEM)
 //               S^T / dP^T of step k+1 are issued as soon as the UMMAs that read
 //               P^T / dS^T from those columns have completed.
 //   warps 2..9  two warpgroups; warpgroup c owns query columns [64c, 64c+64).
-//               Thread = key row: P^T and dS^T as bf16, packed back into TMEM
-//               over the S^T / dP^T columns they came from. At the end dK and dV
-//               rows (fp32) are written out.
+//               Thread = key row, in two phases per step: P^T as bf16 over the S^T
+//               columns as soon as S^T lands (dV starts on it while dP^T is still
+//               in flight), then dS^T over the dP^T columns (dK starts on it). At
+//               the end dK and dV rows (fp32) are written out.
 // Every wait is bounded (usp_ptx.cuh).
 #include <math.h>
 
@@ -70,7 +71,7 @@ struct BwdArgs {
 struct BwdBars {
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
-  uint64_t st_full, p_full, p_used, ds_used, drain;
+  uint64_t s_full, dp_full, p_full, ds_full, p_used, ds_used, drain;
   // Step descriptors published by the producer with qd_full of that step:
   // {q-head in group (-1 = no more steps), ring rank i, query tile m, tile kind}.
   int step[4][4];
@@ -80,7 +81,8 @@ struct BwdBars {
 
 enum : int {
   kSiteBKv = 0x201, kSiteBQdEmpty = 0x202, kSiteBQd = 0x211, kSiteBDsUsed = 0x212, kSiteBP = 0x213,
-  kSiteBPUsed = 0x214, kSiteBSt = 0x221, kSiteBQdC = 0x223, kSiteBEpi = 0x224, kSiteBAlign = 0x2FF
+  kSiteBPUsed = 0x214, kSiteBDs = 0x215, kSiteBSt = 0x221, kSiteBDp = 0x222, kSiteBQdC = 0x223, kSiteBEpi = 0x224,
+  kSiteBAlign = 0x2FF
 };
 
 // Query steps of one key tile: q-head hh of the group, ring rank i, query tile m.
@@ -178,8 +180,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       mbar_init(&bars->qd_full[s], 1);
       mbar_init(&bars->qd_empty[s], 1);
     }
-    mbar_init(&bars->st_full, 1);
-    mbar_init(&bars->p_full, kComputeThreads);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->p_full, kComputeThreads / 32);  // one arrival per compute warp
+    mbar_init(&bars->ds_full, kComputeThreads / 32);
     mbar_init(&bars->p_used, 1);
     mbar_init(&bars->ds_used, 1);
     mbar_init(&bars->drain, 1);
@@ -281,8 +285,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (have) {
           tc_fence_after();
           issue_s(0);
+          umma_commit(&bars->s_full);
           issue_dp(0);
-          umma_commit(&bars->st_full);
+          umma_commit(&bars->dp_full);
           issued_any = true;
         }
       }
@@ -300,6 +305,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
                            kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->p_used);
+        if (!mbar_wait(&bars->ds_full, k & 1, w, kSiteBDs)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk) {  // dK += dS^T Q, K = 128 queries
           const uint32_t pcol = (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
@@ -316,10 +323,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (!mbar_wait(&bars->p_used, k & 1, w, kSiteBPUsed)) { ok = false; break; }
         tc_fence_after();
         issue_s(s1);
+        umma_commit(&bars->s_full);
         if (!mbar_wait(&bars->ds_used, k & 1, w, kSiteBDsUsed)) { ok = false; break; }
         tc_fence_after();
         issue_dp(s1);
-        umma_commit(&bars->st_full);
+        umma_commit(&bars->dp_full);
       }
       if (!ok && issued_any) {
         umma_commit(&bars->drain);
@@ -348,7 +356,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int st_hh = slot[0];
       if (st_hh < 0) break;
       const int st_i = slot[1], st_m = slot[2], st_kind = slot[3];
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->st_full, k & 1, w, kSiteBSt));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, k & 1, w, kSiteBSt));
       if (!ok) break;
       tc_fence_after();
       const float* nlse2 = sRow + s * 256;  // -LSE*log2(e) of the 128 query rows
@@ -383,36 +391,56 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         }
         tmem_st_wait();
       }
+      // Phase 1 (while the tensor core computes dP^T): P^T = exp2(s*scale*log2e - LSE*log2e)
+      // as bf16 over the S^T columns; the fp32 values stay in registers for dS.
+      float2 pr[32];
+      const float2 sl2 = make_float2(g.scale_log2, g.scale_log2);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int c0 = cbase + half * 32;
-        uint32_t rs[32], rp[32];
+        uint32_t rs[32];
         tmem_ld32(trow + kColS + c0, rs);
-        tmem_ld32(trow + kColDP + c0, rp);
         tmem_ld_wait();
         reg_fence32(rs);
-        reg_fence32(rp);
-        uint32_t pk[16], dk[16];
-        const float2 sl2 = make_float2(g.scale_log2, g.scale_log2);
+        uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          // nlse2 = -LSE*log2(e) and ndl = -Delta of the two query columns (smem broadcast)
-          const float2 nl = *reinterpret_cast<const float2*>(nlse2 + c0 + c);
-          const float2 nd = *reinterpret_cast<const float2*>(ndl + c0 + c);
+          const float2 nl = *reinterpret_cast<const float2*>(nlse2 + c0 + c);  // smem broadcast
           const float2 x = ffma2(make_float2(__uint_as_float(rs[c]), __uint_as_float(rs[c + 1])), sl2, nl);
           const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));  // -inf -> 0
-          // dS (without the softmax scale, which is applied to dK and dQ at the end)
-          const float2 ds = fmul2(pv, fadd2(make_float2(__uint_as_float(rp[c]), __uint_as_float(rp[c + 1])), nd));
+          pr[half * 16 + (c >> 1)] = pv;
           pk[c >> 1] = pack_bf16x2(pv.x, pv.y);
+        }
+        tmem_st16(trow + kColS + cbase + half * 16, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive_warp(&bars->p_full);
+      // Phase 2 (while the tensor core computes dV): dS^T = P^T o (dP^T - Delta) as
+      // bf16 over the dP^T columns (without the softmax scale, applied to dK at the end).
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->dp_full, k & 1, w, kSiteBDp));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int c0 = cbase + half * 32;
+        uint32_t rp[32];
+        tmem_ld32(trow + kColDP + c0, rp);
+        tmem_ld_wait();
+        reg_fence32(rp);
+        uint32_t dk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float2 nd = *reinterpret_cast<const float2*>(ndl + c0 + c);
+          const float2 ds = fmul2(pr[half * 16 + (c >> 1)],
+                                  fadd2(make_float2(__uint_as_float(rp[c]), __uint_as_float(rp[c + 1])), nd));
           dk[c >> 1] = pack_bf16x2(ds.x, ds.y);
         }
-        // P^T and dS^T back into TMEM over the S^T / dP^T columns this thread has read
-        tmem_st16(trow + kColS + cbase + half * 16, pk);
         tmem_st16(trow + kColDP + cbase + half * 16, dk);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      mbar_arrive_warp(&bars->ds_full);
     }
     // ------------------------------------------------------------ dK, dV epilogue
     // the last step's dK/dV UMMAs (and every earlier one) have landed once its ds_used arrives

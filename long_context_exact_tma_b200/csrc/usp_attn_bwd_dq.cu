@@ -136,8 +136,8 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       mbar_init(&bars->dq_done[s], 1);
     }
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->dp_free, kComputeDq);
-    mbar_init(&bars->ds_full, kComputeDq);
+    mbar_init(&bars->dp_free, kComputeDq / 32);  // one arrival per compute warp
+    mbar_init(&bars->ds_full, kComputeDq / 32);
     mbar_init(&bars->drain, 1);
     fence_mbar_init();
   }
@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
         reg_fence32(rp);
         if (half == 1) {  // every dP column of this thread has been read
           tc_fence_before();
-          mbar_arrive(&bars->dp_free);
+          mbar_arrive_warp(&bars->dp_free);
         }
         uint32_t dk[16];
 #pragma unroll
@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->ds_full);
+      mbar_arrive_warp(&bars->ds_full);
     }
     // ------------------------------------------------------------ epilogue: dQ rows
     if (ok && it >= 1)

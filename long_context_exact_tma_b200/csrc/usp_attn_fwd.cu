@@ -14,12 +14,13 @@
 // share every K/V tile (320 threads):
 //   warp 0      TMA producer: Q0, Q1 once, then K and V tiles into a kStages ring;
 //               it alone walks the key tiles and publishes one descriptor per tile.
-//   warp 1      TMEM allocator and UMMA issuer (one thread), per key tile:
-//                 S_t  = Q_t K^T  (t = 0, 1; M=128 N=128, fp32 in TMEM)
+//   warp 1      TMEM allocator and UMMA issuer (one thread), per key tile and
+//               query tile t = 0, 1 in turn:
 //                 O_t += P_t V    (M=128 N=D; A = P_t read from TMEM)
-//               S_t of the next tile is issued as soon as the PV UMMA that read
-//               P_t has completed, so the tensor core alternates between the two
-//               tiles while each softmax warpgroup works.
+//                 S_t  = Q_t K^T  of the next key tile (M=128 N=128, fp32 in TMEM;
+//                                 it overwrites P_t, so it waits for that PV)
+//               so the tensor core runs tile 1's PV and S while softmax 0 works
+//               and the other way round.
 //   warps 2..5  softmax of tile 0, warps 6..9 softmax of tile 1: thread = query
 //               row = TMEM lane. tcgen05.ld of S, mask by original positions,
 //               online max/sum in the exp2 domain with lazy rescaling of O (only
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t], 128);
+      mbar_init(&bars->p_full[t], 4);  // one arrival per softmax warp
       mbar_init(&bars->pv_done[t], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -227,34 +228,35 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, 0, 1);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+      auto issue_s = [&](int t, uint32_t kbase) {  // S_t = Q_t K^T
+        const uint32_t qbase = aQ + t * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+          umma_bf16(tmem + col_s(t), sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
+                    kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->s_full[t]);
+      };
       bool ok = mbar_wait(&bars->k_full[0], 0, w, kSiteK);
       const bool have = ok && bars->step[0][0] >= 0;
       bool issued_any = false;
       if (have) ok = mbar_wait(&bars->q_full, 0, w, kSiteQ);
+      if (ok && have) {
+        tc_fence_after();
+        issue_s(0, aK);
+        issue_s(1, aK);
+        issued_any = true;
+      }
+      // Per key tile `it`, per query tile t in turn: O_t += P_t V, then S_t of
+      // tile it+1 (which overwrites P_t, so it waits for that PV to land). The
+      // softmax of one query tile thus overlaps the other tile's PV and S.
       for (int it = 0; ok && have; ++it) {
         const int s = it % C::kStages;
-        if (it > 0) {
-          if (!mbar_wait(&bars->k_full[s], (it / C::kStages) & 1, w, kSiteK)) { ok = false; break; }
-          if (bars->step[it & 3][0] < 0) break;
-        }
-        const uint32_t kbase = aK + s * C::kTileBytes;
-        for (int t = 0; t < 2 && ok; ++t) {
-          // S_t overwrites the columns P_t was read from by the previous PV UMMA.
-          if (it > 0 && !mbar_wait(&bars->pv_done[t], (it - 1) & 1, w, kSitePvDone)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qbase = aQ + t * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-            umma_bf16(tmem + col_s(t), sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                      kIdescQK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&bars->s_full[t]);
-          issued_any = true;
-        }
-        if (!ok) break;
+        const int s1 = (it + 1) % C::kStages;
         if (!mbar_wait(&bars->v_full[s], (it / C::kStages) & 1, w, kSiteV)) { ok = false; break; }
         const uint32_t vbase = aV + s * C::kTileBytes;
+        bool next = false;
         for (int t = 0; t < 2 && ok; ++t) {
           if (!mbar_wait(&bars->p_full[t], it & 1, w, kSiteP)) { ok = false; break; }
           tc_fence_after();
@@ -264,9 +266,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
                              sdesc_sw128(vbase + kk * 16 * 128, C::kPanelBytes, 1024), kIdescPV,
                              (it > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&bars->pv_done[t]);
+          if (t == 1) umma_commit(&bars->kv_empty[s]);
+          if (t == 0) {
+            if (!mbar_wait(&bars->k_full[s1], ((it + 1) / C::kStages) & 1, w, kSiteK)) { ok = false; break; }
+            next = bars->step[(it + 1) & 3][0] >= 0;
+          }
+          if (next) {
+            if (!mbar_wait(&bars->pv_done[t], it & 1, w, kSitePvDone)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(t, aK + s1 * C::kTileBytes);
+          }
         }
-        if (!ok) break;
-        umma_commit(&bars->kv_empty[s]);
+        if (!ok || !next) break;
       }
       if (!ok && issued_any) {
         umma_commit(&bars->drain);
@@ -408,7 +419,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       lb_run = lb_run * alpha + rsb;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[t]);
+      mbar_arrive_warp(&bars->p_full[t]);
     }
     // ------------------------------------------------------------ epilogue
     if (ok && it >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done[t], (it - 1) & 1, w, kSiteO));
