@@ -209,7 +209,12 @@ class Step:
         api, w = self.api, self.w
         P_u, P_r, causal = w["P_u"], w["P_r"], w["causal"]
         st = self.stream
-        for n in ("q", "k", "v"):
+        if ev:
+            ev["perm"][0].record(st)
+        api.seq2head(self.rm["q"], P_u, P_r, out=self.hs["q"])
+        if ev:
+            ev["perm"][1].record(st)
+        for n in ("k", "v"):
             api.seq2head(self.rm[n], P_u, P_r, out=self.hs[n])
         if ev:
             ev["fwd"][0].record(st)
@@ -310,7 +315,7 @@ def bench_ours(args, w, world, rank, local):
     torch.cuda.synchronize()
     step.check_status()
     ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)] for k in ("fwd", "bwd", "dkdv")}
+              for _ in range(args.steps)] for k in ("fwd", "bwd", "dkdv", "perm")}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     with ClockSampler(local) as clk:
@@ -329,6 +334,7 @@ def bench_ours(args, w, world, rank, local):
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["fwd"])
     bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["bwd"])
     dkdv_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["dkdv"])
+    perm_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["perm"])
     # end to end: host buffers in, host buffers out, through the same C ABI calls
     h2d, d2h = step.host_io()
     for _ in range(2):
@@ -369,6 +375,12 @@ def bench_ours(args, w, world, rank, local):
                    "l2": "inputs larger than L2 (Q, K, V, dO 134 MB each)"},
         "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
         "fwd_tflops": round(f_fwd / (fwd_ms / 1e3) / 1e12, 2),
+        # the Ulysses seq->head permute of Q: read + write of every element once
+        "permute": {"kernel": "layout_gather_kernel (seq2head of Q)",
+                    "GB/s": round(2 * step.rm["q"].numel() * 2 / (perm_ms / 1e3) / 1e9, 1),
+                    "frac_of_hbm": round(2 * step.rm["q"].numel() * 2 / (perm_ms / 1e3) / 1e9 / peak_hbm, 4),
+                    "peak_source": f"{peak_src} hbm_gbs"},
+        "exp_count_fwd": int(flops_fwd(w) / (4 * w["D"])),  # B*Hq*S^2 (/2 causal); the backward recomputes them
         "bwd_tflops": round(bwd_tf, 2),
         "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel (key-major dK/dV; usp_attn_bwd_dkdv call)",
                      "achieved": round(dkdv_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",

@@ -19,8 +19,9 @@
 //                 dP^T = V dO^T    -> TMEM [128,256)   (overlaps the P^T phase below)
 //                 dV  += P^T dO    -> TMEM [256,256+D) (A = P^T read from TMEM)
 //                 dK  += dS^T Q    -> TMEM [384,384+D) (A = dS^T read from TMEM)
-//               S^T / dP^T of step k+1 are issued as soon as the UMMAs that read
-//               P^T / dS^T from those columns have completed.
+//               Order per step: dV(k), S^T(k+1) (as soon as dV has read P^T from
+//               its columns), dK(k), dP^T(k+1) (once dK has read dS^T), so that
+//               the P^T phase of step k+1 overlaps dK(k) and dP^T(k+1).
 //   warps 2..9  two warpgroups; warpgroup c owns query columns [64c, 64c+64).
 //               Thread = key row, in two phases per step: P^T as bf16 over the S^T
 //               columns as soon as S^T lands (dV starts on it while dP^T is still
@@ -293,6 +294,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       }
       for (; ok && have; ++k) {
         const int s = k % C::kStages;
+        const int s1 = (k + 1) % C::kStages;
         if (!mbar_wait(&bars->p_full, k & 1, w, kSiteBP)) { ok = false; break; }
         tc_fence_after();
         const uint32_t qb = aQ + s * C::kTileBytes, db = aDO + s * C::kTileBytes;
@@ -305,6 +307,16 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
                            kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->p_used);
+        if (!mbar_wait(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
+        have = bars->step[(k + 1) & 3][0] >= 0;
+        // S^T of the next step as soon as dV has read P^T from its columns, so that the
+        // P^T phase of the next step overlaps dK and dP^T
+        if (have) {
+          if (!mbar_wait(&bars->p_used, k & 1, w, kSiteBPUsed)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(s1);
+          umma_commit(&bars->s_full);
+        }
         if (!mbar_wait(&bars->ds_full, k & 1, w, kSiteBDs)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -315,15 +327,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         }
         umma_commit(&bars->ds_used);
         umma_commit(&bars->qd_empty[s]);  // this step's Q/dO stage is free once these UMMAs land
-        const int s1 = (k + 1) % C::kStages;
-        if (!mbar_wait(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
-        have = bars->step[(k + 1) & 3][0] >= 0;
         if (!have) break;
-        // the next S^T / dP^T overwrite the columns P^T / dS^T are read from
-        if (!mbar_wait(&bars->p_used, k & 1, w, kSiteBPUsed)) { ok = false; break; }
-        tc_fence_after();
-        issue_s(s1);
-        umma_commit(&bars->s_full);
+        // dP^T of the next step overwrites the dS^T that dK reads
         if (!mbar_wait(&bars->ds_used, k & 1, w, kSiteBDsUsed)) { ok = false; break; }
         tc_fence_after();
         issue_dp(s1);
