@@ -254,88 +254,81 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop; one elected lane issues each UMMA/commit.
+    {
       constexpr uint32_t kIdSS = idesc_bf16_f32(128, 128, 0, 0);  // both K-major
       constexpr uint32_t kIdKM = idesc_bf16_f32(128, D, 0, 1);    // A K-major, B MN-major
-      const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ), aDO = smem_addr(sDO);
-      auto issue_s = [&](int s) {  // S^T = K Q^T
-        const uint32_t qb = aQ + s * C::kTileBytes;
+      // tile-base descriptors; a byte offset inside shared memory adds (offset >> 4)
+      const uint64_t dK0 = sdesc_sw128(smem_addr(sK), 16, 1024), dV0 = sdesc_sw128(smem_addr(sV), 16, 1024);
+      const uint64_t dQ0 = sdesc_sw128(smem_addr(sQ), 16, 1024), dDO0 = sdesc_sw128(smem_addr(sDO), 16, 1024);
+      const uint64_t dQmn = sdesc_sw128(smem_addr(sQ), C::kPanelBytes, 1024);
+      const uint64_t dDOmn = sdesc_sw128(smem_addr(sDO), C::kPanelBytes, 1024);
+      auto issue_xt = [&](uint32_t col, uint64_t a0, uint64_t b0, int s) {  // X^T = A B_s^T (S^T or dP^T)
+        const uint64_t bd = b0 + ((s * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_bf16(tmem + kColS, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), kIdSS,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + col, a0 + off, bd + off, kIdSS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_dp = [&](int s) {  // dP^T = V dO^T
-        const uint32_t db = aDO + s * C::kTileBytes;
+      // acc += X^T Y_s with X^T packed in TMEM (warpgroup c's 64 queries at columns
+      // 64c .. 64c+31 of its block) and Y_s (Q or dO of stage s) read MN-major
+      auto issue_acc = [&](uint32_t acc, uint32_t xcol, uint64_t y0, int s, bool first) {
+        const uint64_t yd = y0 + ((s * C::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_bf16(tmem + kColDP, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(db + off, 16, 1024), kIdSS,
-                    kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kBM / 16; ++kk) {
+          const uint32_t pcol = (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
+          umma_bf16_tmem_a_w(tmem + acc, tmem + xcol + pcol, yd + ((kk * 16 * 128) >> 4), kIdKM,
+                             (!first || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(&bars->kv_full, 0, w, kSiteBKv);
+      bool ok = mbar_wait_w(&bars->kv_full, 0, w, kSiteBKv);
       bool issued_any = false;
       bool have = false;
       int k = 0;
-      if (ok) ok = mbar_wait(&bars->qd_full[0], 0, w, kSiteBQd);
+      if (ok) ok = mbar_wait_w(&bars->qd_full[0], 0, w, kSiteBQd);
       if (ok) {
         have = bars->step[0][0] >= 0;
         if (have) {
           tc_fence_after();
-          issue_s(0);
-          umma_commit(&bars->s_full);
-          issue_dp(0);
-          umma_commit(&bars->dp_full);
+          issue_xt(kColS, dK0, dQ0, 0);
+          umma_commit_w(&bars->s_full);
+          issue_xt(kColDP, dV0, dDO0, 0);
+          umma_commit_w(&bars->dp_full);
           issued_any = true;
         }
       }
       for (; ok && have; ++k) {
         const int s = k % C::kStages;
         const int s1 = (k + 1) % C::kStages;
-        if (!mbar_wait(&bars->p_full, k & 1, w, kSiteBP)) { ok = false; break; }
+        if (!mbar_wait_w(&bars->p_full, k & 1, w, kSiteBP)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t qb = aQ + s * C::kTileBytes, db = aDO + s * C::kTileBytes;
-        // P^T and dS^T live in TMEM: warpgroup c packed its 64 queries at columns 64c .. 64c+31
-        // of the S^T (P^T) and dP^T (dS^T) blocks.
-#pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk) {  // dV += P^T dO, K = 128 queries
-          const uint32_t pcol = (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
-          umma_bf16_tmem_a(tmem + kColDV, tmem + kColS + pcol, sdesc_sw128(db + kk * 16 * 128, C::kPanelBytes, 1024),
-                           kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars->p_used);
-        if (!mbar_wait(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
+        issue_acc(kColDV, kColS, dDOmn, s, k == 0);  // dV += P^T dO, K = 128 queries
+        umma_commit_w(&bars->p_used);
+        if (!mbar_wait_w(&bars->qd_full[s1], ((k + 1) / C::kStages) & 1, w, kSiteBQd)) { ok = false; break; }
         have = bars->step[(k + 1) & 3][0] >= 0;
         // S^T of the next step as soon as dV has read P^T from its columns, so that the
         // P^T phase of the next step overlaps dK and dP^T
         if (have) {
-          if (!mbar_wait(&bars->p_used, k & 1, w, kSiteBPUsed)) { ok = false; break; }
+          if (!mbar_wait_w(&bars->p_used, k & 1, w, kSiteBPUsed)) { ok = false; break; }
           tc_fence_after();
-          issue_s(s1);
-          umma_commit(&bars->s_full);
+          issue_xt(kColS, dK0, dQ0, s1);
+          umma_commit_w(&bars->s_full);
         }
-        if (!mbar_wait(&bars->ds_full, k & 1, w, kSiteBDs)) { ok = false; break; }
+        if (!mbar_wait_w(&bars->ds_full, k & 1, w, kSiteBDs)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk) {  // dK += dS^T Q, K = 128 queries
-          const uint32_t pcol = (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
-          umma_bf16_tmem_a(tmem + kColDK, tmem + kColDP + pcol, sdesc_sw128(qb + kk * 16 * 128, C::kPanelBytes, 1024),
-                           kIdKM, (k > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars->ds_used);
-        umma_commit(&bars->qd_empty[s]);  // this step's Q/dO stage is free once these UMMAs land
+        issue_acc(kColDK, kColDP, dQmn, s, k == 0);  // dK += dS^T Q, K = 128 queries
+        umma_commit_w(&bars->ds_used);
+        umma_commit_w(&bars->qd_empty[s]);  // this step's Q/dO stage is free once these UMMAs land
         if (!have) break;
         // dP^T of the next step overwrites the dS^T that dK reads
-        if (!mbar_wait(&bars->ds_used, k & 1, w, kSiteBDsUsed)) { ok = false; break; }
+        if (!mbar_wait_w(&bars->ds_used, k & 1, w, kSiteBDsUsed)) { ok = false; break; }
         tc_fence_after();
-        issue_dp(s1);
-        umma_commit(&bars->dp_full);
+        issue_xt(kColDP, dV0, dDO0, s1);
+        umma_commit_w(&bars->dp_full);
       }
       if (!ok && issued_any) {
-        umma_commit(&bars->drain);
+        umma_commit_w(&bars->drain);
         mbar_wait_drain(&bars->drain, 0, a.wait_ns);
       }
     }

@@ -212,34 +212,36 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop; one elected lane issues each UMMA/commit.
+    {
       constexpr uint32_t kIdSS = idesc_bf16_f32(128, 128, 0, 0);  // both K-major
       constexpr uint32_t kIdKM = idesc_bf16_f32(128, D, 0, 1);    // A (TMEM) K-major, B MN-major
-      const uint32_t aQ = smem_addr(sQ), aDO = smem_addr(sDO), aK = smem_addr(sK), aV = smem_addr(sV);
+      // tile-base descriptors; a byte offset inside shared memory adds (offset >> 4)
+      const uint64_t dQ0 = sdesc_sw128(smem_addr(sQ), 16, 1024), dDO0 = sdesc_sw128(smem_addr(sDO), 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(smem_addr(sK), 16, 1024), dV0 = sdesc_sw128(smem_addr(sV), 16, 1024);
+      const uint64_t dKmn = sdesc_sw128(smem_addr(sK), C::kPanelBytes, 1024);
       auto issue_s = [&](int it) {  // S_it = Q K_it^T into buffer it & 1
-        const uint32_t kb = aK + (it % C::kKStages) * C::kTileBytes;
+        const uint64_t kd = dK0 + (((it % C::kKStages) * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_bf16(tmem + col_sq(it & 1), sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdSS,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + col_sq(it & 1), dQ0 + off, kd + off, kIdSS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full[it & 1]);
+        umma_commit_w(&bars->s_full[it & 1]);
       };
       auto issue_dp = [&](int it) {  // dP_it = dO V_it^T
-        const uint32_t vb = aV + (it % C::kVStages) * C::kTileBytes;
+        const uint64_t vd = dV0 + (((it % C::kVStages) * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_bf16(tmem + kColDPq, sdesc_sw128(aDO + off, 16, 1024), sdesc_sw128(vb + off, 16, 1024), kIdSS,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + kColDPq, dDO0 + off, vd + off, kIdSS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->dp_full);
-        umma_commit(&bars->v_empty[it % C::kVStages]);
+        umma_commit_w(&bars->dp_full);
+        umma_commit_w(&bars->v_empty[it % C::kVStages]);
       };
       // tile `it` exists: wait for its K and read its descriptor
       auto has_tile = [&](int it, bool& ok_) -> bool {
-        if (!mbar_wait(&bars->k_full[it % C::kKStages], (it / C::kKStages) & 1, w, kSiteQK)) {
+        if (!mbar_wait_w(&bars->k_full[it % C::kKStages], (it / C::kKStages) & 1, w, kSiteQK)) {
           ok_ = false;
           return false;
         }
@@ -248,13 +250,13 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       bool ok = true;
       bool issued_any = false;
       bool have0 = has_tile(0, ok);
-      if (ok && have0) ok = mbar_wait(&bars->q_full, 0, w, kSiteQQ);
+      if (ok && have0) ok = mbar_wait_w(&bars->q_full, 0, w, kSiteQQ);
       bool have1 = false;
       if (ok && have0) {
         tc_fence_after();
         issue_s(0);
         issued_any = true;
-        if ((ok = mbar_wait(&bars->v_full[0], 0, w, kSiteQV))) {
+        if ((ok = mbar_wait_w(&bars->v_full[0], 0, w, kSiteQV))) {
           tc_fence_after();
           issue_dp(0);
           have1 = has_tile(1, ok);
@@ -265,39 +267,39 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
         // dP of the next tile as soon as this tile's dP has been read, ahead of dQ,
         // so that the warpgroups can start on the next tile while dQ accumulates
         if (have1) {
-          if (!mbar_wait(&bars->v_full[(it + 1) % C::kVStages], ((it + 1) / C::kVStages) & 1, w, kSiteQV)) {
+          if (!mbar_wait_w(&bars->v_full[(it + 1) % C::kVStages], ((it + 1) / C::kVStages) & 1, w, kSiteQV)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(&bars->dp_free, it & 1, w, kSiteQDpFree)) { ok = false; break; }
+          if (!mbar_wait_w(&bars->dp_free, it & 1, w, kSiteQDpFree)) { ok = false; break; }
           tc_fence_after();
           issue_dp(it + 1);
         }
-        if (!mbar_wait(&bars->ds_full, it & 1, w, kSiteQDs)) { ok = false; break; }
+        if (!mbar_wait_w(&bars->ds_full, it & 1, w, kSiteQDs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t kb = aK + (it % C::kKStages) * C::kTileBytes;
+        const uint64_t kd = dKmn + (((it % C::kKStages) * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {  // dQ += dS K, K = 128 keys
           // warpgroup c packed its 64 keys at columns 64c .. 64c+31 of the S buffer
           const uint32_t pcol = col_sq(it & 1) + (kk < 4 ? 0u : 64u) + (kk & 3) * 8;
-          umma_bf16_tmem_a(tmem + kColDQ, tmem + pcol, sdesc_sw128(kb + kk * 16 * 128, C::kPanelBytes, 1024), kIdKM,
-                           (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a_w(tmem + kColDQ, tmem + pcol, kd + ((kk * 16 * 128) >> 4), kIdKM,
+                             (it > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->dq_done[it & 1]);
-        umma_commit(&bars->k_empty[it % C::kKStages]);
+        umma_commit_w(&bars->dq_done[it & 1]);
+        umma_commit_w(&bars->k_empty[it % C::kKStages]);
         if (!have1) break;
         // S of tile it+2 into this tile's S buffer once dQ has read dS from it
         const bool have2 = has_tile(it + 2, ok);
         if (!ok) break;
         if (have2) {
-          if (!mbar_wait(&bars->dq_done[it & 1], (it >> 1) & 1, w, kSiteQDqDone)) { ok = false; break; }
+          if (!mbar_wait_w(&bars->dq_done[it & 1], (it >> 1) & 1, w, kSiteQDqDone)) { ok = false; break; }
           tc_fence_after();
           issue_s(it + 2);
         }
         have1 = have2;
       }
       if (!ok && issued_any) {
-        umma_commit(&bars->drain);
+        umma_commit_w(&bars->drain);
         mbar_wait_drain(&bars->drain, 0, a.wait_ns);
       }
     }

@@ -224,28 +224,32 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop; one elected lane issues each UMMA/commit.
+    {
       constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, 0, 1);
-      const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
-      auto issue_s = [&](int t, uint32_t kbase) {  // S_t = Q_t K^T
-        const uint32_t qbase = aQ + t * C::kTileBytes;
+      // descriptors of the tile bases; the start address is the low field, so a
+      // byte offset inside shared memory adds (offset >> 4)
+      const uint64_t dQ0 = sdesc_sw128(smem_addr(sQ), 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(smem_addr(sK), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_addr(sV), C::kPanelBytes, 1024);
+      auto issue_s = [&](int t, int ks) {  // S_t = Q_t K^T, K from stage ks
+        const uint64_t qd = dQ0 + ((t * C::kTileBytes) >> 4), kd = dK0 + ((ks * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_bf16(tmem + col_s(t), sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                    kIdescQK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + col_s(t), qd + off, kd + off, kIdescQK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full[t]);
+        umma_commit_w(&bars->s_full[t]);
       };
-      bool ok = mbar_wait(&bars->k_full[0], 0, w, kSiteK);
+      bool ok = mbar_wait_w(&bars->k_full[0], 0, w, kSiteK);
       const bool have = ok && bars->step[0][0] >= 0;
       bool issued_any = false;
-      if (have) ok = mbar_wait(&bars->q_full, 0, w, kSiteQ);
+      if (have) ok = mbar_wait_w(&bars->q_full, 0, w, kSiteQ);
       if (ok && have) {
         tc_fence_after();
-        issue_s(0, aK);
-        issue_s(1, aK);
+        issue_s(0, 0);
+        issue_s(1, 0);
         issued_any = true;
       }
       // Per key tile `it`, per query tile t in turn: O_t += P_t V, then S_t of
@@ -254,33 +258,32 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       for (int it = 0; ok && have; ++it) {
         const int s = it % C::kStages;
         const int s1 = (it + 1) % C::kStages;
-        if (!mbar_wait(&bars->v_full[s], (it / C::kStages) & 1, w, kSiteV)) { ok = false; break; }
-        const uint32_t vbase = aV + s * C::kTileBytes;
+        if (!mbar_wait_w(&bars->v_full[s], (it / C::kStages) & 1, w, kSiteV)) { ok = false; break; }
+        const uint64_t vd = dV0 + ((s * C::kTileBytes) >> 4);
         bool next = false;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!mbar_wait(&bars->p_full[t], it & 1, w, kSiteP)) { ok = false; break; }
+          if (!mbar_wait_w(&bars->p_full[t], it & 1, w, kSiteP)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_bf16_tmem_a(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                             sdesc_sw128(vbase + kk * 16 * 128, C::kPanelBytes, 1024), kIdescPV,
-                             (it > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars->pv_done[t]);
-          if (t == 1) umma_commit(&bars->kv_empty[s]);
+            umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_w(&bars->pv_done[t]);
+          if (t == 1) umma_commit_w(&bars->kv_empty[s]);
           if (t == 0) {
-            if (!mbar_wait(&bars->k_full[s1], ((it + 1) / C::kStages) & 1, w, kSiteK)) { ok = false; break; }
+            if (!mbar_wait_w(&bars->k_full[s1], ((it + 1) / C::kStages) & 1, w, kSiteK)) { ok = false; break; }
             next = bars->step[(it + 1) & 3][0] >= 0;
           }
           if (next) {
-            if (!mbar_wait(&bars->pv_done[t], it & 1, w, kSitePvDone)) { ok = false; break; }
+            if (!mbar_wait_w(&bars->pv_done[t], it & 1, w, kSitePvDone)) { ok = false; break; }
             tc_fence_after();
-            issue_s(t, aK + s1 * C::kTileBytes);
+            issue_s(t, s1);
           }
         }
         if (!ok || !next) break;
       }
       if (!ok && issued_any) {
-        umma_commit(&bars->drain);
+        umma_commit_w(&bars->drain);
         mbar_wait_drain(&bars->drain, 0, a.wait_ns);
       }
     }
