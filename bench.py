@@ -343,6 +343,30 @@ def cpu_baseline_sample(w, seconds=10.0, seed=0):
     return fl / el / 1e12, n, el, oracle.max_threads()
 
 
+def merge_bandwidth(w, dev):
+    """GB/s of usp_lse_merge over the stepwise partials of this workload: P_r
+    partials (O_t fp32 [rows, D], LSE_t fp32 [rows]) merged into O bf16 + LSE."""
+    from long_context_exact_tma_b200 import api
+    n, rows, D = w["P_r"], w["B"] * w["S"] * w["Hq"], w["D"]
+    rows = min(rows, (4 << 30) // (n * D * 4))  # at most 4 GiB of partials
+    g = torch.Generator(device=dev).manual_seed(7)
+    o = torch.randn((n, rows, D), generator=g, device=dev, dtype=torch.float32)
+    lse = torch.randn((n, rows), generator=g, device=dev, dtype=torch.float32)
+    api.lse_merge(o, lse)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    reps = 5
+    for _ in range(reps):
+        api.lse_merge(o, lse)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = n * rows * (4 * D + 4) + rows * (2 * D + 4)
+    del o, lse
+    return nbytes / (ms / 1e3) / 1e9
+
+
 def bench_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -393,6 +417,7 @@ def bench_ours(args, w, world, rank, local):
     e2e = world * args.steps * f_step / (e2e_ms / 1e3) / 1e12
     if rank != 0:
         return None
+    merge_gbs = merge_bandwidth(w, dev)
     bwd_tf = 2.5 * f_fwd / (bwd_ms / 1e3) / 1e12
     # dominant kernel: the key-major dK/dV kernel, whose algorithmic work is its four
     # GEMMs per (key tile, query tile) pair (S^T, dP^T, dV, dK) = 2 x the forward FLOPs
@@ -422,6 +447,9 @@ def bench_ours(args, w, world, rank, local):
                     "GB/s": round(2 * step.rm["q"].numel() * 2 / (perm_ms / 1e3) / 1e9, 1),
                     "frac_of_hbm": round(2 * step.rm["q"].numel() * 2 / (perm_ms / 1e3) / 1e9 / peak_hbm, 4),
                     "peak_source": f"{peak_src} hbm_gbs"},
+        # the log-sum-exp merge of the P_r stepwise partials (read every partial once, write O + LSE)
+        "merge": {"kernel": "lse_merge_kernel (P_r fp32 partials -> bf16 O + LSE)", "GB/s": round(merge_gbs, 1),
+                  "frac_of_hbm": round(merge_gbs / peak_hbm, 4), "peak_source": f"{peak_src} hbm_gbs"},
         "exp_count_fwd": int(flops_fwd(w) / (4 * w["D"])),  # B*Hq*S^2 (/2 causal); the backward recomputes them
         "bwd_tflops": round(bwd_tf, 2),
         "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel (key-major dK/dV; usp_attn_bwd_dkdv call)",

@@ -202,46 +202,55 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     // nothing issued, nothing to drain
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
+    // The whole warp walks the steps (the same values in every lane); one elected
+    // lane issues each copy and barrier operation.
+    {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+      }
+      __syncwarp();
       const int krb = jrank * g.B + b;
-      mbar_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+      mbar_expect_tx_w(&bars->kv_full, 2 * C::kTileBytes);
       for (int p = 0; p < C::kPanels; ++p) {
-        tma_load_4d(&tm_k, &bars->kv_full, sK + p * C::kPanelBytes, p * 64, gl, k0, krb);
-        tma_load_4d(&tm_v, &bars->kv_full, sV + p * C::kPanelBytes, p * 64, gl, k0, krb);
+        tma_load_4d_w(&tm_k, &bars->kv_full, sK + p * C::kPanelBytes, p * 64, gl, k0, krb);
+        tma_load_4d_w(&tm_v, &bars->kv_full, sV + p * C::kPanelBytes, p * 64, gl, k0, krb);
       }
       int issued = 0;
       QWalk qw = qwalk_begin(g, j, kmin, kmax);
       while (true) {
         const int s = issued % C::kStages;
         if (issued >= C::kStages &&
-            !mbar_wait(&bars->qd_empty[s], ((issued / C::kStages) - 1) & 1, w, kSiteBQdEmpty))
+            !mbar_wait_w(&bars->qd_empty[s], ((issued / C::kStages) - 1) & 1, w, kSiteBQdEmpty))
           break;
         int* slot = bars->step[issued & 3];
         if (!qw.valid) {  // publish the end of the walk on this stage's barrier
-          slot[0] = -1;
-          mbar_arrive(&bars->qd_full[s]);
+          if (lane == 0) slot[0] = -1;
+          __syncwarp();
+          mbar_arrive_w(&bars->qd_full[s]);
           break;
         }
-        slot[0] = qw.hh;
-        slot[1] = qw.i;
-        slot[2] = qw.m;
-        slot[3] = qw.kind;
+        if (lane == 0) {
+          slot[0] = qw.hh;
+          slot[1] = qw.i;
+          slot[2] = qw.m;
+          slot[3] = qw.kind;
+        }
+        __syncwarp();
         const int h = gl * g.G + qw.hh;
         const int qrb = (qw.i * g.P_u + u) * g.B + b;
         const int q0 = qw.m * kBM;
-        mbar_expect_tx(&bars->qd_full[s], 2 * C::kTileBytes + 1024);
+        mbar_expect_tx_w(&bars->qd_full[s], 2 * C::kTileBytes + 1024);
         for (int p = 0; p < C::kPanels; ++p) {
-          tma_load_4d(&tm_q, &bars->qd_full[s], sQ + s * C::kTileBytes + p * C::kPanelBytes, p * 64, h, q0, qrb);
-          tma_load_4d(&tm_do, &bars->qd_full[s], sDO + s * C::kTileBytes + p * C::kPanelBytes, p * 64, h, q0,
-                      qrb);
+          tma_load_4d_w(&tm_q, &bars->qd_full[s], sQ + s * C::kTileBytes + p * C::kPanelBytes, p * 64, h, q0, qrb);
+          tma_load_4d_w(&tm_do, &bars->qd_full[s], sDO + s * C::kTileBytes + p * C::kPanelBytes, p * 64, h, q0,
+                        qrb);
         }
         const size_t rowbase = (static_cast<size_t>(qrb) * g.Hq_l + h) * a.Lp + q0;
-        bulk_load_1d(sRow + s * 256, a.lse2 + rowbase, 512, &bars->qd_full[s]);
-        bulk_load_1d(sRow + s * 256 + 128, a.delta + rowbase, 512, &bars->qd_full[s]);
+        bulk_load_1d_w(sRow + s * 256, a.lse2 + rowbase, 512, &bars->qd_full[s]);
+        bulk_load_1d_w(sRow + s * 256 + 128, a.delta + rowbase, 512, &bars->qd_full[s]);
         ++issued;
         qwalk_next(g, j, kmin, kmax, qw);
       }

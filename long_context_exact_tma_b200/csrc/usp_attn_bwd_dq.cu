@@ -153,55 +153,64 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     // nothing issued, nothing to drain
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp walks the key tiles (the same values in every lane); one
+    // elected lane issues each copy and barrier operation.
+    {
       int qmin, qmax;
       pos_range(g, i, q0, q0 + kBM, qmin, qmax);
       KvWalk kw = kv_walk_begin(g, i, qmin, qmax, 0, g.P_r);
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+      }
+      __syncwarp();
       const int qrb = rank * g.B + b;
-      mbar_expect_tx(&bars->q_full, 2 * C::kTileBytes);
+      mbar_expect_tx_w(&bars->q_full, 2 * C::kTileBytes);
       for (int p = 0; p < C::kPanels; ++p) {
-        tma_load_4d(&tm_q, &bars->q_full, sQ + p * C::kPanelBytes, p * 64, h, q0, qrb);
-        tma_load_4d(&tm_do, &bars->q_full, sDO + p * C::kPanelBytes, p * 64, h, q0, qrb);
+        tma_load_4d_w(&tm_q, &bars->q_full, sQ + p * C::kPanelBytes, p * 64, h, q0, qrb);
+        tma_load_4d_w(&tm_do, &bars->q_full, sDO + p * C::kPanelBytes, p * 64, h, q0, qrb);
       }
       int k_issued = 0, v_issued = 0;
       while (true) {
         const int it = k_issued;
         const int sk = it % C::kKStages, sv = it % C::kVStages;
         if (it >= C::kKStages &&
-            !mbar_wait(&bars->k_empty[sk], ((it / C::kKStages) - 1) & 1, w, kSiteQKEmpty))
+            !mbar_wait_w(&bars->k_empty[sk], ((it / C::kKStages) - 1) & 1, w, kSiteQKEmpty))
           break;
         int* slot = bars->step[it & 3];
         if (!kw.valid) {  // publish the end of the walk on this stage's barrier
-          slot[0] = -1;
-          mbar_arrive(&bars->k_full[sk]);
+          if (lane == 0) slot[0] = -1;
+          __syncwarp();
+          mbar_arrive_w(&bars->k_full[sk]);
           break;
         }
-        slot[0] = 1;
-        slot[1] = kw.j;
-        slot[2] = kw.n;
-        slot[3] = kw.kind;
+        if (lane == 0) {
+          slot[0] = 1;
+          slot[1] = kw.j;
+          slot[2] = kw.n;
+          slot[3] = kw.kind;
+        }
+        __syncwarp();
         const int krb = (kw.j * g.P_u + u) * g.B + b;
-        mbar_expect_tx(&bars->k_full[sk], C::kTileBytes);
+        mbar_expect_tx_w(&bars->k_full[sk], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_4d(&tm_k, &bars->k_full[sk], sK + sk * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
-                      kw.n * kBN, krb);
+          tma_load_4d_w(&tm_k, &bars->k_full[sk], sK + sk * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
+                        kw.n * kBN, krb);
         ++k_issued;
         if (it >= C::kVStages &&
-            !mbar_wait(&bars->v_empty[sv], ((it / C::kVStages) - 1) & 1, w, kSiteQVEmpty))
+            !mbar_wait_w(&bars->v_empty[sv], ((it / C::kVStages) - 1) & 1, w, kSiteQVEmpty))
           break;
-        mbar_expect_tx(&bars->v_full[sv], C::kTileBytes);
+        mbar_expect_tx_w(&bars->v_full[sv], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_4d(&tm_v, &bars->v_full[sv], sV + sv * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
-                      kw.n * kBN, krb);
+          tma_load_4d_w(&tm_v, &bars->v_full[sv], sV + sv * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
+                        kw.n * kBN, krb);
         ++v_issued;
         kv_walk_next(g, i, qmin, qmax, g.P_r, kw);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
-        // Let every copy this thread started land before the CTA exits.
+        // Let every copy this warp started land before the CTA exits.
         mbar_wait_drain(&bars->q_full, 0, a.wait_ns);
         for (int it = k_issued - C::kKStages < 0 ? 0 : k_issued - C::kKStages; it < k_issued; ++it)
           mbar_wait_drain(&bars->k_full[it % C::kKStages], (it / C::kKStages) & 1, a.wait_ns);

@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     // nothing issued, nothing to drain
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp walks the tiles (the same values in every lane); one elected
+    // lane issues each copy and barrier operation.
+    {
       int qmin0, qmax0, qmin1, qmax1;
       pos_range(g, i, q0, q0 + kBM, qmin0, qmax0);
       pos_range(g, i, q0 + kBM, q0 + 2 * kBM, qmin1, qmax1);
@@ -176,44 +178,53 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       int issued = 0;
       const bool any = kw.valid;
       if (any) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        mbar_expect_tx(&bars->q_full, 2 * C::kTileBytes);
+        if (lane == 0) {
+          tma_prefetch_desc(&tm_q);
+          tma_prefetch_desc(&tm_k);
+          tma_prefetch_desc(&tm_v);
+        }
+        __syncwarp();
+        mbar_expect_tx_w(&bars->q_full, 2 * C::kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int p = 0; p < C::kPanels; ++p)
-            tma_load_4d(&tm_q, &bars->q_full, sQ + t * C::kTileBytes + p * C::kPanelBytes, p * 64, h,
-                        q0 + t * kBM, rank * g.B + b);
+            tma_load_4d_w(&tm_q, &bars->q_full, sQ + t * C::kTileBytes + p * C::kPanelBytes, p * 64, h,
+                          q0 + t * kBM, rank * g.B + b);
       }
       while (true) {
         const int s = issued % C::kStages;
         if (issued >= C::kStages &&
-            !mbar_wait(&bars->kv_empty[s], ((issued / C::kStages) - 1) & 1, w, kSiteKvEmpty))
+            !mbar_wait_w(&bars->kv_empty[s], ((issued / C::kStages) - 1) & 1, w, kSiteKvEmpty))
           break;
         int* slot = bars->step[issued & 3];
         if (!kw.valid) {  // publish the end of the walk on this stage's barrier
-          slot[0] = -1;
-          mbar_arrive(&bars->k_full[s]);
+          if (lane == 0) slot[0] = -1;
+          __syncwarp();
+          mbar_arrive_w(&bars->k_full[s]);
           break;
         }
-        slot[0] = 1;
-        slot[1] = kw.j;
-        slot[2] = kw.n;
-        slot[3] = classify_tile(g, qmin0, qmax0, kw.j, kw.n) | (classify_tile(g, qmin1, qmax1, kw.j, kw.n) << 4);
+        const int kinds =
+            classify_tile(g, qmin0, qmax0, kw.j, kw.n) | (classify_tile(g, qmin1, qmax1, kw.j, kw.n) << 4);
+        if (lane == 0) {
+          slot[0] = 1;
+          slot[1] = kw.j;
+          slot[2] = kw.n;
+          slot[3] = kinds;
+        }
+        __syncwarp();
         const int krb = (kw.j * g.P_u + u) * g.B + b;
-        mbar_expect_tx(&bars->k_full[s], C::kTileBytes);
+        mbar_expect_tx_w(&bars->k_full[s], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_4d(&tm_k, &bars->k_full[s], sK + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
-                      kw.n * kBN, krb);
-        mbar_expect_tx(&bars->v_full[s], C::kTileBytes);
+          tma_load_4d_w(&tm_k, &bars->k_full[s], sK + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
+                        kw.n * kBN, krb);
+        mbar_expect_tx_w(&bars->v_full[s], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_4d(&tm_v, &bars->v_full[s], sV + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
-                      kw.n * kBN, krb);
+          tma_load_4d_w(&tm_v, &bars->v_full[s], sV + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
+                        kw.n * kBN, krb);
         ++issued;
         kv_walk_next(g, i, qmin, qmax, t_end, kw);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
-        // Let every copy this thread started land before the CTA exits.
+        // Let every copy this warp started land before the CTA exits.
         if (any) mbar_wait_drain(&bars->q_full, 0, a.wait_ns);
         for (int it = issued - C::kStages < 0 ? 0 : issued - C::kStages; it < issued; ++it) {
           mbar_wait_drain(&bars->k_full[it % C::kStages], (it / C::kStages) & 1, a.wait_ns);
