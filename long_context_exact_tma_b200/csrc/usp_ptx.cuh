@@ -42,10 +42,6 @@ __device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -105,18 +101,10 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   return true;
 }
 
-// ---------------------------------------------------------------- TMA
-// 4-D tiled bulk tensor load into shared memory, completing on `bar`.
-__device__ __forceinline__ void tma_load_4d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1,
-                                            int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
-      : "memory");
-}
+// ---------------------------------------------------------------- TMA / bulk copies
 // Warp-wide forms of the producer's operations: the whole (converged) warp
 // executes them and one lane chosen by elect.sync performs them.
+// 4-D tiled bulk tensor load into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_4d_w(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1,
                                               int c2, int c3) {
   asm volatile(
@@ -137,7 +125,7 @@ __device__ __forceinline__ void mbar_arrive_w(uint64_t* bar) {
                "@e mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_addr(bar))
                : "memory");
 }
-
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16), completing on `bar`.
 __device__ __forceinline__ void bulk_load_1d_w(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -147,38 +135,10 @@ __device__ __forceinline__ void bulk_load_1d_w(void* dst, const void* src, uint3
       : "memory");
 }
 
-// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16), completing on `bar`.
-__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-// 4-D tiled bulk reduce-add shared -> global (fp32 add), tracked by the bulk group of this thread.
-__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
-                                                  int c3) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until every bulk operation of this thread's committed groups has finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Waits until every committed bulk operation of this thread has completed (global writes included).
-__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// ---------------------------------------------------------------- fences
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -194,26 +154,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-// UMMA D(tmem) (+)= A(smem desc) x B(smem desc), kind::f16 (bf16 in, fp32 acc).
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// UMMA with the A operand in TMEM (lane = row of A, K packed two bf16 per 32-bit column).
-__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 // Warp-wide forms: the whole (converged) warp executes them and one lane chosen
 // by elect.sync issues. Keeping the issuing warp converged lets the operand
 // descriptors stay warp-uniform; issuing from a one-lane branch measured slower.
@@ -246,13 +186,6 @@ __device__ __forceinline__ void umma_commit_w(uint64_t* bar) {
 // A bounded wait taken by a whole warp: true only if every lane saw the phase.
 __device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, const WaitCtl& w, int site) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, w, site));
-}
-
-// Arrive (once) on `bar` when every UMMA issued so far by this thread has completed.
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_addr(bar))
-               : "memory");
 }
 
 #define USP_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
@@ -376,17 +309,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // The two bf16 values packed in w, widened exactly to fp32.
 __device__ __forceinline__ float2 bf16x2_unpack(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-
-// Sum of the two bf16 values packed in w, in fp32 (exact widening).
-__device__ __forceinline__ float bf16x2_sum(uint32_t w) {
-  return __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
-}
-
-// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte
-// swizzled tile whose 8-row atoms are 1024-byte aligned.
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
-  return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
 }  // namespace usp
