@@ -43,8 +43,8 @@ UNIT = "TFLOP/s"
 # dK/dV kernel on causal_fwd_s16k_ring8, from the ncu capture summarised in
 # profiles/attn_bwd_kernel_causal_fwd_s16k_ring8.md. Reported only while the
 # kernel's sources hash to what was captured (else the figure is stale: null).
-DKDV_TRAFFIC = {"workload": "causal_fwd_s16k_ring8", "bytes": 1034001408,
-                "sources_sha256": "425d67e020b75dd774b0c80148df5c691974b155d0ddc2011d1f72cc4f203a7d"}
+DKDV_TRAFFIC = {"workload": "causal_fwd_s16k_ring8", "bytes": 1033810432,
+                "sources_sha256": "c4c2c0aef98c9bbc0fde6e4c595a16a60e7f467f380c9b78f24d6ed34cdf8d35"}
 DKDV_SOURCES = ("usp_attn_bwd.cu", "usp_attn_common.cuh", "usp_ptx.cuh", "usp_internal.h")
 
 

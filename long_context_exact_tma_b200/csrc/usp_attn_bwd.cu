@@ -41,6 +41,7 @@ constexpr int kThreadsBwd = 320;
 constexpr int kComputeThreads = 256;
 constexpr uint32_t kTmemColsBwd = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+constexpr int kPolyPer8 = 2;  // key pairs (of every 8) whose exp2 runs on the FMA pipe
 
 template <int D>
 struct BwdCfg {
@@ -414,7 +415,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         for (int c = 0; c < 32; c += 2) {
           const float2 nl = *reinterpret_cast<const float2*>(nlse2 + c0 + c);  // smem broadcast
           const float2 x = ffma2(make_float2(__uint_as_float(rs[c]), __uint_as_float(rs[c + 1])), sl2, nl);
-          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));  // -inf -> 0
+          // kPolyPer8 key pairs in every 8 take the polynomial exp2 on the FMA pipe,
+          // which has room in this kernel while the MUFU bounds the P phase. A -inf
+          // score gets ~2^-125 there instead of 0: a weight no dK/dV sum resolves.
+          const float2 pv = ((c >> 1) % 8 < kPolyPer8) ? exp2_poly2(x)
+                                                       : make_float2(ex2_approx(x.x), ex2_approx(x.y));
           pr[half * 16 + (c >> 1)] = pv;
           pk[c >> 1] = pack_bf16x2(pv.x, pv.y);
         }

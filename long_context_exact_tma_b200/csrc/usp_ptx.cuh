@@ -300,6 +300,39 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+// Packed add with explicit round-to-nearest (never contracted into an FMA).
+__device__ __forceinline__ float2 fadd2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for two values on the FMA and integer pipes instead of the MUFU: n =
+// round(x) by the 1.5*2^23 addition trick, f = x - n in [-1/2, 1/2] exactly, 2^f
+// by a degree-3 polynomial (Remez minimax in relative error, coefficients from
+// exp2_poly_coeffs.py: max relative error 7.5e-5, below a quarter of a bf16
+// half-ulp), and 2^n added into the exponent field. x is clamped to >= -125 so
+// that the exponent stays normal: inputs below give ~2^-125 instead of ~0, a
+// weight no softmax row can resolve next to its total weight of 1.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kC0 = 0.999928057f, kC1 = 0.693260968f, kC2 = 0.242611125f, kC3 = 0.0551716685f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2_rn(x, make_float2(kRound, kRound));      // low bits of t hold n
+  const float2 n = fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 p = ffma2(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  p = ffma2(p, f, make_float2(kC1, kC1));
+  p = ffma2(p, f, make_float2(kC0, kC0));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Three-input maximum.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
