@@ -203,12 +203,23 @@ class Step:
         self.dv_rm = torch.empty_like(self.dk_rm)
         self.ws_f = api.workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, w["causal"], P_u, P_r, 0, 0), dev)
         self.ws_b = api.workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, w["causal"], P_u, P_r, 0, 1), dev)
+        # the permutes of dO and O run on a second stream, overlapping the attention kernels
+        self.side = torch.cuda.Stream(device=dev)
+        self.e_start, self.e_do, self.e_fwd, self.e_o = (torch.cuda.Event() for _ in range(4))
 
     def run(self, ev=None):
         """One step; ev = (start, end) event pairs per timed call, or None."""
         api, w = self.api, self.w
         P_u, P_r, causal = w["P_u"], w["P_r"], w["causal"]
         st = torch.cuda.current_stream()
+        side = self.side
+        # Ulysses all-to-all of dO on the side stream while Q, K, V are permuted and
+        # the forward runs (it only waits for the previous step's use of hs["do"])
+        self.e_start.record(st)
+        side.wait_event(self.e_start)
+        with torch.cuda.stream(side):
+            api.seq2head(self.rm["do"], P_u, P_r, out=self.hs["do"])
+            self.e_do.record(side)
         if ev:
             ev["perm"][0].record(st)
         api.seq2head(self.rm["q"], P_u, P_r, out=self.hs["q"])
@@ -222,8 +233,13 @@ class Step:
                      lse=self.lse)
         if ev:
             ev["fwd"][1].record(st)
-        api.head2seq(self.out, P_u, P_r, out=self.o_rm)
-        api.seq2head(self.rm["do"], P_u, P_r, out=self.hs["do"])
+        # O back to the sequence layout on the side stream while the backward runs
+        self.e_fwd.record(st)
+        side.wait_event(self.e_fwd)
+        with torch.cuda.stream(side):
+            api.head2seq(self.out, P_u, P_r, out=self.o_rm)
+            self.e_o.record(side)
+        st.wait_event(self.e_do)
         # backward = prepare + key-major dK/dV kernel + query-major dQ kernel (what
         # usp_attn_bwd runs), called phase by phase so the dK/dV kernel is timed alone
         geo = (w["B"], w["S"], w["Hq"], w["Hkv"], w["D"], causal, P_u, P_r)
@@ -244,6 +260,7 @@ class Step:
         api.head2seq(self.dq, P_u, P_r, out=self.dq_rm)
         api.head2seq(self.dk, P_u, P_r, out=self.dk_rm)
         api.head2seq(self.dv, P_u, P_r, out=self.dv_rm)
+        st.wait_event(self.e_o)  # the step ends with O's permute done too
 
     def check_status(self):
         for ws in (self.ws_f, self.ws_b):
