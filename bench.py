@@ -427,22 +427,24 @@ def bench_ours(args, w, world, rank, local):
     dkdv_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["dkdv"])
     # end to end: host buffers in, host buffers out, through the same C ABI calls,
     # with the copies of neighbouring steps overlapping the kernels
-    h2d, d2h = step.host_io()
-    step2 = Step(w, dev, seed_offset=1000 * rank)
-    step2.host_io()
-    pipe = E2EPipeline([step, step2])
-    pipe.run(2)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    e0.record(pipe.s_in)
-    pipe.run(args.steps)
-    e1.record(pipe.s_out)
-    torch.cuda.synchronize()
-    for st_ in (step, step2):
-        st_.check_status()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e = world * args.steps * f_step / (e2e_ms / 1e3) / 1e12
+    e2e = h2d = d2h = None
+    if not args.no_e2e:
+        h2d, d2h = step.host_io()
+        step2 = Step(w, dev, seed_offset=1000 * rank)
+        step2.host_io()
+        pipe = E2EPipeline([step, step2])
+        pipe.run(2)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        e0.record(pipe.s_in)
+        pipe.run(args.steps)
+        e1.record(pipe.s_out)
+        torch.cuda.synchronize()
+        for st_ in (step, step2):
+            st_.check_status()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = world * args.steps * f_step / (e2e_ms / 1e3) / 1e12
     if rank != 0:
         return None
     merge_gbs = merge_bandwidth(w, dev)
@@ -483,8 +485,9 @@ def bench_ours(args, w, world, rank, local):
                      "achieved": round(dkdv_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(dkdv_tf / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "launch_ms": round(dkdv_ms, 4), "traffic": dkdv_traffic(w["name"])},
-        "e2e": {"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "overlap": "copies of neighbouring steps overlap the kernels (3 streams, 2 buffer sets)"},
+        "e2e": ({"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                 "overlap": "copies of neighbouring steps overlap the kernels (3 streams, 2 buffer sets)"}
+                if e2e is not None else None),
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
@@ -535,6 +538,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end host-buffer run (its pinned buffers are 2 x the step's IO)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warmup raised to the minimum of 3", file=sys.stderr)
