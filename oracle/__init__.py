@@ -13,6 +13,10 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   lse_merge -- pinned: chunked-and-merged == unchunked, empty partials.
   zigzag_* / seq2head / head2seq -- pinned: hand-written worked examples in
       tests/golden/, bijection and inverse checks.
+  dilated_fwd_rows (LongNet dilated attention) -- pinned: a hand-derived worked
+      example (tests/golden/dilated_tiny_closed_form.json), one pair (w = S,
+      r = 1) against torch's fp64 scaled_dot_product_attention, and torch's fp64
+      SDPA with the log of the key multiplicities as an additive mask.
 """
 from __future__ import annotations
 
@@ -42,13 +46,15 @@ def lib():
         L.oracle_attn_dq_rows.argtypes = [P, P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, P, P, P, i_]
         L.oracle_attn_dkdv_cols.argtypes = [P, P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, P, P, P, P, i_]
         L.oracle_lse_merge.argtypes = [l_, l_, l_, P, P, P, P, i_]
+        L.oracle_dilated_fwd_rows.argtypes = [P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, l_, P, P, P, i_]
         for name in ("oracle_zigzag_shard", "oracle_zigzag_unshard"):
             getattr(L, name).argtypes = [P, P, l_, l_, l_, l_, l_, l_]
         for name in ("oracle_seq2head", "oracle_head2seq"):
             getattr(L, name).argtypes = [P, P, l_, l_, l_, l_, l_, l_, l_]
         for name in ("oracle_attn_fwd_rows", "oracle_attn_full", "oracle_attn_dq_rows",
                      "oracle_attn_dkdv_cols", "oracle_lse_merge", "oracle_zigzag_shard",
-                     "oracle_zigzag_unshard", "oracle_seq2head", "oracle_head2seq"):
+                     "oracle_zigzag_unshard", "oracle_seq2head", "oracle_head2seq",
+                     "oracle_dilated_fwd_rows"):
             getattr(L, name).restype = ctypes.c_int
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
@@ -100,6 +106,24 @@ def attn_fwd_rows(q, k, v, causal, rows, ranges=None, scale=None, threads=0):
                                     scale, n, _ptr(rows), nr, rp, _ptr(o), _ptr(lse), threads)
     if rc != 0:
         raise ValueError(f"oracle_attn_fwd_rows failed ({rc})")
+    return o, lse
+
+
+def dilated_fwd_rows(q, k, v, causal, pairs, rows, scale=None, threads=0):
+    """LongNet dilated attention: O [n, D] and LSE [n] (float64) of query rows
+    (b, h, i) for the (w, r) pairs `pairs`, global-layout inputs."""
+    B, S, Hq, Hkv, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    (qa, ka, va), f64 = _inputs(q, k, v)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    n = rows.shape[0]
+    o = np.zeros((n, D), np.float64)
+    lse = np.zeros(n, np.float64)
+    rc = lib().oracle_dilated_fwd_rows(_ptr(qa), _ptr(ka), _ptr(va), f64, B, S, Hq, Hkv, D, int(causal), scale,
+                                       pr.shape[0], _ptr(pr), n, _ptr(rows), _ptr(o), _ptr(lse), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_dilated_fwd_rows failed ({rc})")
     return o, lse
 
 

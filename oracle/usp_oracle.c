@@ -426,3 +426,104 @@ int oracle_head2seq(const uint8_t *src, uint8_t *dst, long B, long S, long H, lo
                     }
     return 0;
 }
+
+/*
+ * LongNet dilated attention, forward, for a list of query rows.
+ *
+ * Source: the LongNet slides (page 4): "Abstract" (dilated attention is a
+ * drop-in replacement for standard attention; attention allocation falls
+ * exponentially with distance) and "Results" (segment lengths w = {2048, 4096,
+ * 8192, 16384, 32768} with dilation ratios r = {1, 2, 4, 6, 12}). The page's
+ * formula figures did not survive extraction; the steps below are the
+ * published method those slides summarise, in its order:
+ *   1. for each (w_k, r_k), split the sequence into segments of w_k tokens
+ *      (the last one shorter when w_k does not divide S);
+ *   2. in every segment keep every r_k-th row, starting at the offset
+ *      o = h mod r_k of the query head h: positions s*w + o + m*r, m >= 0,
+ *      inside the segment (key/value rows of kv head h / (Hq/Hkv) at the same
+ *      positions);
+ *   3. dense softmax attention among the kept rows of the segment (causal:
+ *      key position <= query position), giving the output O_k and the softmax
+ *      denominator Z_k = sum_j exp(s_ij) at every kept row; a row that is not
+ *      kept, or sees no key, has an empty result (Z_k = 0);
+ *   4. the k results are combined with weights proportional to their softmax
+ *      denominators: O = sum_k Z_k O_k / sum_k Z_k. The row's LSE is
+ *      log sum_k Z_k (-inf and O = 0 when every Z_k is 0).
+ * Denominators are carried as logarithms (LSE_k = log Z_k) so that they do not
+ * overflow; step 4 is then the log-sum-exp merge.
+ * pairs = [n_pairs][2] (w, r), w >= 1, 1 <= r. Layouts and rows as in
+ * oracle_attn_fwd_rows.
+ */
+int oracle_dilated_fwd_rows(const void *q, const void *k, const void *v, int f64, long B, long S,
+                            long Hq, long Hkv, long D, int causal, double scale, long n_pairs,
+                            const long *pairs, long n_rows, const long *rows, double *o,
+                            double *lse, int n_threads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || !rows_ok(n_rows, rows, B, Hq, S) || n_pairs <= 0) return -1;
+    for (long p = 0; p < n_pairs; p++)
+        if (pairs[2 * p] < 1 || pairs[2 * p + 1] < 1) return -1;
+    set_threads(n_threads);
+#pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)S);
+        double *o_k = (double *)malloc(sizeof(double) * (size_t)(n_pairs * D));
+        double *l_k = (double *)malloc(sizeof(double) * (size_t)n_pairs);
+#pragma omp for schedule(dynamic, 1)
+        for (long r_ = 0; r_ < n_rows; r_++) {
+            long b = rows[3 * r_], h = rows[3 * r_ + 1], i = rows[3 * r_ + 2];
+            long g = h / (Hq / Hkv);
+            long qi = idx4(b, i, h, 0, S, Hq, D);
+            /* steps 1-3 for every pair */
+            for (long p = 0; p < n_pairs; p++) {
+                long w = pairs[2 * p], r = pairs[2 * p + 1];
+                long off = h % r;
+                long seg0 = (i / w) * w;
+                long seg1 = seg0 + w < S ? seg0 + w : S;
+                double *op = o_k + p * D;
+                for (long d = 0; d < D; d++) op[d] = 0.0;
+                l_k[p] = -INFINITY;
+                if (i - seg0 < off || (i - seg0 - off) % r != 0) continue; /* row not kept */
+                long jend = causal ? i + 1 : seg1;
+                double m = -INFINITY;
+                for (long j = seg0 + off; j < jend; j += r) {
+                    long kj = idx4(b, j, g, 0, S, Hkv, D);
+                    double acc = 0.0;
+                    for (long d = 0; d < D; d++) acc += ld(q, qi + d, f64) * ld(k, kj + d, f64);
+                    s_buf[j] = scale * acc;
+                    if (s_buf[j] > m) m = s_buf[j];
+                }
+                if (m == -INFINITY) continue;
+                double z = 0.0;
+                for (long j = seg0 + off; j < jend; j += r) z += exp(s_buf[j] - m);
+                l_k[p] = m + log(z);
+                for (long j = seg0 + off; j < jend; j += r) {
+                    double wgt = exp(s_buf[j] - l_k[p]);
+                    long vj = idx4(b, j, g, 0, S, Hkv, D);
+                    for (long d = 0; d < D; d++) op[d] += wgt * ld(v, vj + d, f64);
+                }
+            }
+            /* step 4: weights proportional to the denominators exp(LSE_k) */
+            double *orow = o + r_ * D;
+            for (long d = 0; d < D; d++) orow[d] = 0.0;
+            double mx = -INFINITY;
+            for (long p = 0; p < n_pairs; p++)
+                if (l_k[p] > mx) mx = l_k[p];
+            if (mx == -INFINITY) {
+                lse[r_] = -INFINITY;
+                continue;
+            }
+            double zsum = 0.0;
+            for (long p = 0; p < n_pairs; p++) zsum += exp(l_k[p] - mx);
+            double L = mx + log(zsum);
+            lse[r_] = L;
+            for (long p = 0; p < n_pairs; p++) {
+                if (l_k[p] == -INFINITY) continue;
+                double alpha = exp(l_k[p] - L);
+                for (long d = 0; d < D; d++) orow[d] += alpha * o_k[p * D + d];
+            }
+        }
+        free(s_buf);
+        free(o_k);
+        free(l_k);
+    }
+    return 0;
+}
