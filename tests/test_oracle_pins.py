@@ -279,15 +279,127 @@ def test_layout_maps_are_bijections(P_u, P_r, H):
     assert torch.equal(oracle.from_head_sharded(oracle.to_head_sharded(xb, P_u, P_r), P_u, P_r), xb)
 
 
-def test_attention_result_is_split_invariant():
-    """The attention result, mapped back to token order, does not depend on (P_u, P_r)."""
-    B, S, H, D = 1, 48, 4, 8
+@pytest.mark.parametrize("P_u,P_r", [(1, 2), (2, 2), (4, 1), (2, 3), (1, 4)])
+def test_ring_steps_of_every_rank_merge_to_the_unsplit_result(P_u, P_r):
+    """The USP computation done rank by rank and ring step by ring step: ring rank
+    i's queries at step t attend the keys held by owner j = (i - t) mod P_r, the
+    P_r partials merge (oracle.lse_merge) to the unsplit attention of those rows.
+
+    The positions a rank holds are read off the oracle's own layout maps applied
+    to a tensor of token ids, and checked against the zigzag reading (rank r holds
+    chunks r and 2P-1-r), so a wrong chunk assignment, a ring schedule that misses
+    or repeats a key block, or a wrong merge all fail here."""
+    B, H, D = 1, 2 * P_u, 8
+    P = P_u * P_r
+    c = 3
+    S = 2 * P * c
     q, k, v = _rand(81, (B, S, H, D)), _rand(82, (B, S, H, D)), _rand(83, (B, S, H, D))
-    ref_o, ref_lse = oracle.attn_fwd_rows(q, k, v, True, _all_rows(B, S, H))
-    for P_u, P_r in ((1, 2), (2, 2), (4, 1), (2, 3)):
-        # permute to the head-sharded layout and back: the rows the oracle is asked
-        # about keep their global positions, so the answer must not move
-        qs = oracle.from_head_sharded(oracle.to_head_sharded(q, P_u, P_r), P_u, P_r)
-        o, lse = oracle.attn_fwd_rows(qs, k, v, True, _all_rows(B, S, H))
-        np.testing.assert_array_equal(o, ref_o)
-        np.testing.assert_array_equal(lse, ref_lse)
+    ids = torch.arange(S, dtype=torch.float32).view(1, S, 1, 1).expand(B, S, H, 1).contiguous()
+    hs = oracle.to_head_sharded(ids, P_u, P_r)  # [P_r, P_u, B, L, H/P_u, 1]
+    L, Hl = S // P_r, H // P_u
+
+    def chunks_of(r):
+        return [r, 2 * P - 1 - r]
+
+    def positions(i):  # original positions held by ring rank i (any u), in local order
+        return [ch * c + x for up in range(P_u) for ch in chunks_of(i * P_u + up) for x in range(c)]
+
+    for i in range(P_r):
+        for u in range(P_u):
+            assert hs[i, u, 0, :, 0, 0].long().tolist() == positions(i)
+    for i in range(P_r):
+        for u in range(P_u):
+            heads = range(u * Hl, (u + 1) * Hl)
+            rows = [(0, h, pos) for h in heads for pos in positions(i)]
+            ref_o, ref_lse = oracle.attn_fwd_rows(q, k, v, True, rows)
+            o_parts, l_parts, seen = [], [], []
+            for t in range(P_r):
+                j = (i - t) % P_r
+                ranges = [(ch * c, ch * c + c) for up in range(P_u) for ch in chunks_of(j * P_u + up)]
+                seen += [x for a, e in ranges for x in range(a, e)]
+                o_t, l_t = oracle.attn_fwd_rows(q, k, v, True, rows, ranges=ranges)
+                o_parts.append(o_t)
+                l_parts.append(l_t)
+            assert sorted(seen) == list(range(S))  # every key block exactly once per ring
+            o, lse = oracle.lse_merge(np.stack(o_parts), np.stack(l_parts))
+            np.testing.assert_allclose(o, ref_o, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- LongNet dilated attention
+def test_dilated_golden_tiny_closed_form():
+    g = json.load(open(os.path.join(GOLD, "dilated_tiny_closed_form.json")))
+    S = g["S"]
+    q = torch.zeros(1, S, 2, 2, dtype=torch.bfloat16)
+    v = torch.zeros(1, S, 2, 2, dtype=torch.float64)
+    for j in range(S):
+        v[0, j, 0] = torch.tensor([j, 1.0])
+        v[0, j, 1] = torch.tensor([10 - j, 2.0])
+    v = v.to(torch.bfloat16)  # small integers: exact in bf16
+    k = _rand(5, (1, S, 2, 2))  # irrelevant when Q = 0
+    for c in g["cases"]:
+        o, lse = oracle.dilated_fwd_rows(q, k, v, True, c["pairs"], [(0, c["head"], c["row"])])
+        np.testing.assert_allclose(o[0], c["o"], rtol=0, atol=1e-13)
+        want = -math.inf if c["lse"] == "-inf" else c["lse"]
+        if want == -math.inf:
+            assert lse[0] == -math.inf
+        else:
+            assert abs(lse[0] - want) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_dilated_one_pair_w_s_r1_is_full_attention(causal):
+    B, S, Hq, Hkv, D = 2, 48, 4, 2, 16
+    q, k, v = _rand(61, (B, S, Hq, D)), _rand(62, (B, S, Hkv, D)), _rand(63, (B, S, Hkv, D))
+    o, lse = oracle.dilated_fwd_rows(q, k, v, causal, [(S, 1)], _all_rows(B, S, Hq))
+    ref = _sdpa64(q, k, v, causal).numpy()
+    rows = _all_rows(B, S, Hq)
+    idx = np.array(rows)
+    np.testing.assert_allclose(o, ref[idx[:, 0], idx[:, 2], idx[:, 1]], rtol=0, atol=1e-12)
+
+
+def _multiplicity_mask(S, H, pairs, causal):
+    """[H, S, S] count of the pairs through which query i sees key j (from the
+    reading: segments of w, rows s*w + (h mod r) + m*r kept, causal within)."""
+    C = np.zeros((H, S, S))
+    for w, r in pairs:
+        for h in range(H):
+            off = h % r
+            for s0 in range(0, S, w):
+                kept = list(range(s0 + off, min(s0 + w, S), r))
+                for i in kept:
+                    for j in kept:
+                        if not causal or j <= i:
+                            C[h, i, j] += 1
+    return C
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("pairs", [[(8, 1), (16, 2), (32, 4)], [(12, 3), (24, 6)], [(10, 1), (40, 4), (40, 12)]])
+def test_dilated_matches_sdpa_with_multiplicity_mask(causal, pairs):
+    """Dilated attention is softmax attention in which key j counts C_ij times for
+    query i (C = the number of pairs that show it): torch fp64 SDPA with the
+    additive mask log C (-inf where C = 0) gives the same O."""
+    B, S, Hq, Hkv, D = 1, 40, 4, 2, 8
+    q, k, v = _rand(71, (B, S, Hq, D)), _rand(72, (B, S, Hkv, D)), _rand(73, (B, S, Hkv, D))
+    rows = _all_rows(B, S, Hq)
+    o, lse = oracle.dilated_fwd_rows(q, k, v, causal, pairs, rows)
+    C = _multiplicity_mask(S, Hq, pairs, causal)
+    with np.errstate(divide="ignore"):
+        mask = torch.tensor(np.log(C))
+    G = Hq // Hkv
+    qt = q.double().transpose(1, 2)
+    kt = k.double().repeat_interleave(G, dim=2).transpose(1, 2)
+    vt = v.double().repeat_interleave(G, dim=2).transpose(1, 2)
+    idx = np.array(rows)
+    seen = C.sum(-1)[idx[:, 1], idx[:, 2]] > 0
+    ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask.unsqueeze(0)).transpose(1, 2).numpy()
+    ref = ref[idx[:, 0], idx[:, 2], idx[:, 1]]
+    np.testing.assert_allclose(o[seen], ref[seen], rtol=0, atol=1e-12)
+    # rows no pair keeps: empty result
+    assert np.all(o[~seen] == 0) and np.all(np.isneginf(lse[~seen]))
+    # LSE = log sum_j C_ij exp(s_ij)
+    s = torch.einsum("bhid,bhjd->bhij", qt, kt).numpy()[0] / math.sqrt(D)
+    with np.errstate(divide="ignore"):
+        lref = np.log((C * np.exp(s)).sum(-1))[idx[:, 1], idx[:, 2]]
+    np.testing.assert_allclose(lse[seen], lref[seen], rtol=0, atol=1e-12)
