@@ -40,9 +40,9 @@ from usp_inputs import WORKLOADS, workload  # noqa: E402
 METRIC = "attention TFLOP/s fwd+bwd at S=16K-256K; % of bf16 dense tensor peak"
 UNIT = "TFLOP/s"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# dK/dV kernel on causal_fwd_s16k_ring8, from the ncu capture summarised in
-# profiles/attn_bwd_kernel_causal_fwd_s16k_ring8.md. Reported only while the
-# kernel's sources hash to what was captured (else the figure is stale: null).
+# dK/dV kernel on causal_fwd_s16k_ring8, from an ncu capture of that kernel.
+# Reported only while the kernel's sources hash to what was captured (else the
+# figure is stale: null).
 DKDV_TRAFFIC = {"workload": "causal_fwd_s16k_ring8", "bytes": 1033810432,
                 "sources_sha256": "c4c2c0aef98c9bbc0fde6e4c595a16a60e7f467f380c9b78f24d6ed34cdf8d35"}
 DKDV_SOURCES = ("usp_attn_bwd.cu", "usp_attn_common.cuh", "usp_ptx.cuh", "usp_internal.h")
@@ -63,8 +63,6 @@ def dkdv_traffic(workload_name: str):
         return None
     return rec["bytes"] if dkdv_sources_sha256() == rec["sources_sha256"] else None
 
-
-LAUNCHES_PER_STEP = 12  # 3 seq2head + fwd + head2seq(O) + seq2head(dO) + prep + dK/dV + dQ + 3 head2seq
 
 
 def flops_fwd(w) -> float:
@@ -220,8 +218,9 @@ class Step:
         with torch.cuda.stream(side):
             api.seq2head(self.rm["do"], P_u, P_r, out=self.hs["do"])
             self.e_do.record(side)
-        for n in ("q", "k", "v"):
-            api.seq2head(self.rm[n], P_u, P_r, out=self.hs[n])
+        # the Ulysses all-to-all of Q, K and V in one launch
+        api.seq2head_many([self.rm[n] for n in ("q", "k", "v")], P_u, P_r,
+                          outs=[self.hs[n] for n in ("q", "k", "v")])
         if ev:
             ev["fwd"][0].record(st)
         api.attn_fwd(self.hs["q"], self.hs["k"], self.hs["v"], causal, P_u, P_r, ws=self.ws_f, out=self.out,
@@ -252,9 +251,8 @@ class Step:
                            ws_b, ws_b.numel(), st)
         if ev:
             ev["bwd"][1].record(st)
-        api.head2seq(self.dq, P_u, P_r, out=self.dq_rm)
-        api.head2seq(self.dk, P_u, P_r, out=self.dk_rm)
-        api.head2seq(self.dv, P_u, P_r, out=self.dv_rm)
+        # the regather of dQ, dK and dV in one launch
+        api.head2seq_many([self.dq, self.dk, self.dv], P_u, P_r, outs=[self.dq_rm, self.dk_rm, self.dv_rm])
         st.wait_event(self.e_o)  # the step ends with O's permute done too
 
     def check_status(self):
@@ -355,45 +353,121 @@ def cpu_baseline_sample(w, seconds=10.0, seed=0):
     return fl / el / 1e12, n, el, oracle.max_threads()
 
 
+def _time_ms(fn, reps=5):
+    """Mean device time of fn() over `reps` back-to-back calls (CUDA events on the
+    current stream, one untimed call first)."""
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
 def permute_bandwidth(step):
-    """GB/s of the seq->head permute of Q timed alone (inside the step it shares
-    HBM with the side stream's permutes): read + write of every element once."""
+    """GB/s of the step's seq->head all-to-all of Q, K and V (one launch), timed
+    alone (inside the step it shares HBM with the side stream's permutes): read +
+    write of every element once."""
     api, w = step.api, step.w
-    reps = 5
-    api.seq2head(step.rm["q"], w["P_u"], w["P_r"], out=step.hs["q"])
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        api.seq2head(step.rm["q"], w["P_u"], w["P_r"], out=step.hs["q"])
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
-    return 2 * step.rm["q"].numel() * step.rm["q"].element_size() / (ms / 1e3) / 1e9
+    names = ("q", "k", "v")
+    ms = _time_ms(lambda: api.seq2head_many([step.rm[n] for n in names], w["P_u"], w["P_r"],
+                                            outs=[step.hs[n] for n in names]))
+    nbytes = 2 * sum(step.rm[n].numel() * step.rm[n].element_size() for n in names)
+    return nbytes / (ms / 1e3) / 1e9, nbytes
 
 
-def merge_bandwidth(w, dev):
-    """GB/s of usp_lse_merge over the stepwise partials of this workload: P_r
-    partials (O_t fp32 [rows, D], LSE_t fp32 [rows]) merged into O bf16 + LSE."""
-    from long_context_exact_tma_b200 import api
-    n, rows, D = w["P_r"], w["B"] * w["S"] * w["Hq"], w["D"]
-    rows = min(rows, (4 << 30) // (n * D * 4))  # at most 4 GiB of partials
-    g = torch.Generator(device=dev).manual_seed(7)
-    o = torch.randn((n, rows, D), generator=g, device=dev, dtype=torch.float32)
-    lse = torch.randn((n, rows), generator=g, device=dev, dtype=torch.float32)
-    api.lse_merge(o, lse)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    reps = 5
-    for _ in range(reps):
-        api.lse_merge(o, lse)
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
-    nbytes = n * rows * (4 * D + 4) + rows * (2 * D + 4)
-    del o, lse
+def merge_bandwidth(step):
+    """GB/s of usp_lse_merge on the partials the stepwise forward really leaves in
+    its workspace: the running merge of ring steps 0..P_r-2 and step P_r-1's
+    partial (fp32 O [rows, D] + LSE [rows] each), merged into O bf16 + LSE, the
+    last step of the streamed ring merge. Read 2*(4D+4), write 2D+4 bytes a row."""
+    api, B_, w = step.api, step.B_, step.w
+    B, S, Hq, Hkv, D, P_u, P_r = (w[k] for k in ("B", "S", "Hq", "Hkv", "D", "P_u", "P_r"))
+    need = B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, w["causal"], P_u, P_r, B_.USP_MODE_STEPWISE, 0)
+    ws = api.workspace(need, step.out.device)
+    api.attn_fwd(step.hs["q"], step.hs["k"], step.hs["v"], w["causal"], P_u, P_r, mode=B_.USP_MODE_STEPWISE, ws=ws,
+                 check_status=True)
+    rows = B * S * Hq
+    body = ws[256:]
+    o_parts = body[: 2 * rows * D * 4].view(torch.float32).view(2, rows, D)
+    l_parts = body[2 * rows * D * 4:].view(torch.float32).view(2, rows)
+    out = torch.empty((rows, D), dtype=torch.bfloat16, device=ws.device)
+    lse = torch.empty(rows, dtype=torch.float32, device=ws.device)
+    ms = _time_ms(lambda: B_.usp_lse_merge(o_parts, l_parts, 2, rows, D, out, B_.USP_BF16, lse))
+    nbytes = 2 * rows * (4 * D + 4) + rows * (2 * D + 4)
+    del ws
     return nbytes / (ms / 1e3) / 1e9
+
+
+def per_workload(dev, peak_tf, peak_hbm):
+    """Event-timed figures on the workloads the targets are stated for: the causal
+    GQA S=128K USP 4x2 forward and its permutes (seq->head of Q, K, V in one launch;
+    head->seq of O), and the causal B=2 S=32K ring-4 backward. Inputs are seeded
+    N(0,1) of each shape, already resident; 3 timed calls after one untimed."""
+    from long_context_exact_tma_b200 import api
+    from long_context_exact_tma_b200 import binding as B_
+    res = {}
+    for cfg, kind in ((3, "fwd"), (4, "bwd")):
+        w = dict(WORKLOADS[cfg])
+        P_u, P_r, causal = w["P_u"], w["P_r"], w["causal"]
+        t = workload(w, device=dev, which=("q", "k", "v", "do") if kind == "bwd" else ("q", "k", "v"))
+        rm = {n: api.zigzag_shard(t[n], P_u, P_r) for n in t if n != "spec"}
+        del t
+        names = ("q", "k", "v")
+        hs = api.seq2head_many([rm[n] for n in names], P_u, P_r)
+        hs = dict(zip(names, hs))
+        f_fwd = flops_fwd(w)
+        rec = {"workload": w["name"]}
+        if kind == "fwd":
+            ms = _time_ms(lambda: api.seq2head_many([rm[n] for n in names], P_u, P_r,
+                                                    outs=[hs[n] for n in names]), reps=3)
+            nb = 2 * sum(rm[n].numel() * rm[n].element_size() for n in names)
+            rec["seq2head_qkv"] = {"GB/s": round(nb / (ms / 1e3) / 1e9, 1),
+                                   "frac_of_hbm": round(nb / (ms / 1e3) / 1e9 / peak_hbm, 4), "bytes": nb}
+            ws = api.workspace(256, dev)
+            out, lse = api.attn_fwd(hs["q"], hs["k"], hs["v"], causal, P_u, P_r, ws=ws)
+            ms = _time_ms(lambda: api.attn_fwd(hs["q"], hs["k"], hs["v"], causal, P_u, P_r, ws=ws, out=out, lse=lse),
+                          reps=3)
+            api.check_workspace(ws)
+            tf = f_fwd / (ms / 1e3) / 1e12
+            rec["fwd"] = {"TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / peak_tf, 4), "ms": round(ms, 3)}
+            o_rm = torch.empty((P_u * P_r,) + tuple(rm["q"].shape[1:]), dtype=torch.bfloat16, device=dev)
+            ms = _time_ms(lambda: api.head2seq(out, P_u, P_r, out=o_rm), reps=3)
+            nb = 2 * out.numel() * out.element_size()
+            rec["head2seq_o"] = {"GB/s": round(nb / (ms / 1e3) / 1e9, 1),
+                                 "frac_of_hbm": round(nb / (ms / 1e3) / 1e9 / peak_hbm, 4), "bytes": nb}
+            del out, lse, o_rm
+        else:
+            do = api.seq2head(rm["do"], P_u, P_r)
+            out, lse = api.attn_fwd(hs["q"], hs["k"], hs["v"], causal, P_u, P_r)
+            geo = (w["B"], w["S"], w["Hq"], w["Hkv"], w["D"], causal, P_u, P_r)
+            ws = api.workspace(B_.usp_attn_workspace_size(*geo, 0, 1), dev)
+            dq, dk, dv = api.attn_bwd(hs["q"], hs["k"], hs["v"], out, lse, do, causal, P_u, P_r, ws=ws)
+            ms = _time_ms(lambda: api.attn_bwd(hs["q"], hs["k"], hs["v"], out, lse, do, causal, P_u, P_r, ws=ws,
+                                               dq=dq, dk=dk, dv=dv), reps=3)
+            api.check_workspace(ws)
+            tf = 2.5 * f_fwd / (ms / 1e3) / 1e12
+            rec["bwd"] = {"TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / peak_tf, 4), "ms": round(ms, 3),
+                          "convention": "2.5 x forward FLOPs (5 GEMMs per visible 128x128 pair)"}
+            del do, out, lse, dq, dk, dv
+        res[f"cfg{cfg}"] = rec
+        del rm, hs
+        torch.cuda.empty_cache()
+    return res
+
+
+def l2_note(step, dev):
+    """Whether every input of the step is larger than L2 (then no flush is needed
+    between timed iterations)."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    sizes = {n: t.numel() * t.element_size() for n, t in step.rm.items()}
+    big = all(v > l2 for v in sizes.values())
+    txt = ", ".join(f"{n} {v / 1e6:.0f} MB" for n, v in sizes.items())
+    return (f"inputs larger than L2 ({txt}; L2 {l2 / 1e6:.0f} MB)" if big else
+            f"NOT all inputs larger than L2 ({txt}; L2 {l2 / 1e6:.0f} MB)")
 
 
 def bench_ours(args, w, world, rank, local):
@@ -409,12 +483,14 @@ def bench_ours(args, w, world, rank, local):
               for _ in range(args.steps)] for k in ("fwd", "bwd", "dkdv")}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
+    n_launch0 = step.B_.usp_launch_count()
     with ClockSampler(local) as clk:
         start.record()
         for s in range(args.steps):
             step.run({k: ev[k][s] for k in ev})
         end.record()
         torch.cuda.synchronize()
+    gpu_launches = step.B_.usp_launch_count() - n_launch0
     barrier(world)
     step.check_status()
     ms_local = start.elapsed_time(end)
@@ -447,8 +523,9 @@ def bench_ours(args, w, world, rank, local):
         e2e = world * args.steps * f_step / (e2e_ms / 1e3) / 1e12
     if rank != 0:
         return None
-    merge_gbs = merge_bandwidth(w, dev)
-    perm_gbs = permute_bandwidth(step)
+    merge_gbs = merge_bandwidth(step)
+    perm_gbs, perm_bytes = permute_bandwidth(step)
+    per_wl = None if args.no_per_workload else per_workload(dev, peak_tf, peak_hbm)
     bwd_tf = 2.5 * f_fwd / (bwd_ms / 1e3) / 1e12
     # dominant kernel: the key-major dK/dV kernel, whose algorithmic work is its four
     # GEMMs per (key tile, query tile) pair (S^T, dP^T, dV, dK) = 2 x the forward FLOPs
@@ -470,15 +547,17 @@ def bench_ours(args, w, world, rank, local):
                    "D": w["D"], "causal": bool(w["causal"]), "P_ulysses": w["P_u"], "P_ring": w["P_r"],
                    "global_batch": w["B"] * world, "seq_len": w["S"],
                    "parallelism": f"{world} independent replicas x (USP {w['P_u']}x{w['P_r']} virtual ranks)",
-                   "l2": "inputs larger than L2 (Q, K, V, dO 134 MB each)"},
+                   "l2": l2_note(step, dev)},
         "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
         "fwd_tflops": round(f_fwd / (fwd_ms / 1e3) / 1e12, 2),
-        # the Ulysses seq->head permute of Q: read + write of every element once
-        "permute": {"kernel": "layout_gather_kernel (seq2head of Q, timed alone)", "GB/s": round(perm_gbs, 1),
+        # the Ulysses seq->head all-to-all of Q, K, V (one launch): read + write of every element once
+        "permute": {"kernel": "layout_gather_kernel (seq2head of Q, K, V in one launch, timed alone)",
+                    "GB/s": round(perm_gbs, 1), "bytes": perm_bytes,
                     "frac_of_hbm": round(perm_gbs / peak_hbm, 4), "peak_source": f"{peak_src} hbm_gbs"},
-        # the log-sum-exp merge of the P_r stepwise partials (read every partial once, write O + LSE)
-        "merge": {"kernel": "lse_merge_kernel (P_r fp32 partials -> bf16 O + LSE)", "GB/s": round(merge_gbs, 1),
-                  "frac_of_hbm": round(merge_gbs / peak_hbm, 4), "peak_source": f"{peak_src} hbm_gbs"},
+        # the last step of the streamed ring merge, on the stepwise forward's own partials
+        "merge": {"kernel": "lse_merge_kernel (running fp32 merge + last ring step's partial -> bf16 O + LSE)",
+                  "GB/s": round(merge_gbs, 1), "frac_of_hbm": round(merge_gbs / peak_hbm, 4),
+                  "peak_source": f"{peak_src} hbm_gbs"},
         "exp_count_fwd": int(flops_fwd(w) / (4 * w["D"])),  # B*Hq*S^2 (/2 causal); the backward recomputes them
         "bwd_tflops": round(bwd_tf, 2),
         "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel (key-major dK/dV; usp_attn_bwd_dkdv call)",
@@ -488,7 +567,8 @@ def bench_ours(args, w, world, rank, local):
         "e2e": ({"value": round(e2e, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                  "overlap": "copies of neighbouring steps overlap the kernels (3 streams, 2 buffer sets)"}
                 if e2e is not None else None),
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": gpu_launches,
+        "per_workload": per_wl,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -538,6 +618,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the event-timed S=128K forward/permute and S=32K backward figures")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end host-buffer run (its pinned buffers are 2 x the step's IO)")
     args = ap.parse_args()

@@ -71,6 +71,10 @@ int usp_version(void);
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char* usp_last_error(void);
 
+/* Number of kernels this library has launched in this process (all threads,
+ * all devices): a counter for measurement, incremented at every launch. */
+unsigned long long usp_launch_count(void);
+
 /*
  * Zigzag shard: global [B][S][H][D] -> rank-major [P][B][2c][H][D]; rank r
  * receives chunks r and 2P-1-r (load balancing of the causal ring, "Boosting
@@ -97,10 +101,37 @@ int usp_head2seq_permute(const void* src, void* dst, int B, int S, int H, int D,
                          void* stream);
 
 /*
+ * Several layout gathers of one map and mesh in ONE launch, e.g. the seq->head
+ * all-to-all of Q, K and V before the attention, or the head->seq regather of
+ * dQ, dK and dV after it (DeepSpeed-Ulysses summary, "Wie DeepSpeed-Ulysses
+ * funktioniert"). Each job is a tensor with its own head count, head-row
+ * length and element type, moved exactly as the single call of that map would
+ * move it (bit-exact); the launch and its tail are paid once for all of them.
+ *   map     USP_MAP_ZIGZAG_SHARD, USP_MAP_ZIGZAG_UNSHARD, USP_MAP_SEQ2HEAD or
+ *           USP_MAP_HEAD2SEQ (the layouts of usp_zigzag_shard, usp_zigzag_unshard,
+ *           usp_seq2head_permute, usp_head2seq_permute)
+ *   jobs    HOST array of n_jobs (1 .. USP_MAX_PERMUTE_JOBS) descriptors; each
+ *           job is checked as the single call would check it. Destinations must
+ *           not overlap any source or each other.
+ */
+enum { USP_MAP_ZIGZAG_SHARD = 0, USP_MAP_ZIGZAG_UNSHARD = 1, USP_MAP_SEQ2HEAD = 2, USP_MAP_HEAD2SEQ = 3 };
+#define USP_MAX_PERMUTE_JOBS 4
+typedef struct {
+  const void* src; /* device pointer, 16-byte aligned */
+  void* dst;       /* device pointer, 16-byte aligned */
+  int H;           /* heads of this tensor */
+  int D;           /* elements per head row (1 for an LSE tensor) */
+  int dtype;       /* USP_BF16 or USP_F32 */
+} usp_permute_job;
+int usp_permute_batch(int map, const usp_permute_job* jobs, int n_jobs, int B, int S, int P_u, int P_r,
+                      void* stream);
+
+/*
  * Bytes of workspace needed by usp_attn_fwd (bwd = 0, by mode) or
  * usp_attn_bwd (bwd = 1). Returns 0 for an unsupported shape.
  *   fused fwd   : 256 (status word)
- *   stepwise fwd: 256 + P_r * B*S*Hq * (4*D + 4)  (fp32 partials of every ring step)
+ *   stepwise fwd: 256 + 2 * B*S*Hq * (4*D + 4)  (two fp32 partials: the running
+ *                 merge of the ring steps done so far and the current step's)
  *   bwd         : 256 + 2 * 4 * B*P_u*P_r*(Hq/P_u)*Lp, Lp = S/P_r rounded up to a
  *                 multiple of 128 (-LSE*log2(e) and -Delta per head and row)
  */
@@ -121,8 +152,15 @@ size_t usp_attn_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal,
  * causal: key visible iff its original token position <= the query's.
  * scale = 1/sqrt(D).
  * mode USP_MODE_FUSED: one launch, ring steps merged online in the kernel.
- * mode USP_MODE_STEPWISE: one launch per ring step writing fp32 partials into
- * the workspace, then usp_lse_merge -- the ring algorithm step for step.
+ * mode USP_MODE_STEPWISE: the ring algorithm step for step. Each ring step is
+ * one launch that writes its fp32 partial (O_t, LSE_t) into the workspace, and
+ * the log-sum-exp merge (the kernel of usp_lse_merge) folds it into a running
+ * fp32 (O, LSE): two partials in, one out per step, so the workspace holds two
+ * partials whatever P_r is. The last step's merge writes out and lse. On return
+ * the workspace holds, after the 256-byte status header, o_parts [2][rows][D]
+ * and lse_parts [2][rows] (rows = B*S*Hq in the head-sharded row order): slot 0
+ * the merge of steps 0..P_r-2, slot 1 the partial of step P_r-1 (for P_r = 1,
+ * slot 0 is step 0's partial and slot 1 is unused).
  */
 int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
                  int Hkv, int D, int causal, int P_u, int P_r, int mode, void* workspace, size_t ws_bytes,
@@ -178,24 +216,69 @@ int usp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
  * that must not allocate after initialisation (cudaMalloc can synchronise the
  * device).
  *
- * Arguments and results are those of usp_attn_bwd. The scratch (status word,
- * fp32 dQ accumulator, per-head LSE and Delta tables) is a file-scope static
- * __device__ array of USP_NOALLOC_SCRATCH_BYTES bytes, which every GPU that
- * loads this part of the library holds until the process exits. A problem
+ * Arguments and results are those of usp_attn_bwd. The scratch is a
+ * file-scope static __device__ array of USP_NOALLOC_SCRATCH_BYTES bytes, which
+ * every GPU that loads this part of the library holds until the process exits.
+ * It has the layout of the usp_attn_bwd workspace: the 256-byte status header,
+ * then the per-head -LSE*log2(e) and -Delta tables. Each call clears the status
+ * word; the two tables are rewritten in full (padding rows included) by the
+ * prepare step of every call, so nothing else has to start at zero. A problem
  * whose usp_attn_workspace_size(..., bwd=1) exceeds that size is rejected with
  * USP_ERR_WORKSPACE before anything is launched. The call allocates nothing:
  * no cudaMalloc, no cudaFree, no allocating library routine.
  *
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, which may load the library's device code); make that
- * first call before any stream capture. Every call shares the one array and
- * clears the parts that must start at zero; calls whose work overlaps on the
- * GPU (other streams, other threads) race on it and must be serialised by the
- * caller.
+ * (cudaGetSymbolAddress, which may load the library's device code) and keeps
+ * it for the life of the process; make that first call before any stream
+ * capture, and do not use this entry point across a cudaDeviceReset (the
+ * device code, and with it the array, may then load at another address).
+ * Every call shares the one array; calls whose work overlaps on the GPU (other
+ * streams, other threads) race on it and must be serialised by the caller. A
+ * bounded device wait that gives up during a call records its site in the
+ * array's status word; usp_attn_bwd_noalloc_status reads it.
  */
 int usp_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out, const float* lse,
                          const void* dO, void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D,
                          int causal, int P_u, int P_r, void* stream);
+
+/*
+ * LongNet dilated attention, forward (LongNet slides, "Abstract": dilated
+ * attention is a drop-in replacement for standard attention; "Results":
+ * segment lengths w = {2048, ..., 32768} with dilation ratios r = {1, 2, 4, 6,
+ * 12}). For each of the n_pairs pairs (w[p], r[p]):
+ *   - the sequence is cut into segments of w[p] tokens;
+ *   - in every segment, every r[p]-th row is kept, starting at the offset
+ *     h mod r[p] of query head h (the kv head h / (Hq/Hkv) uses the same rows);
+ *   - exact softmax attention runs among the kept rows of each segment
+ *     (causal: key position <= query position);
+ * and the pairs' results are combined with weights proportional to their
+ * softmax denominators: O = sum_p Z_p O_p / sum_p Z_p, LSE = log sum_p Z_p,
+ * i.e. the log-sum-exp merge. A row that no pair keeps gets O = 0, LSE = -inf.
+ *   q            [B][S][Hq][D]  bf16 (global layout; one device's sequence)
+ *   k, v         [B][S][Hkv][D] bf16
+ *   out          [B][S][Hq][D]  bf16;  lse [B][S][Hq] fp32, natural log
+ *   w, r         HOST arrays of n_pairs (1 .. USP_DILATED_MAX_PAIRS) ints;
+ *                S % w[p] == 0 and 1 <= r[p] <= w[p]
+ *   workspace    usp_dilated_workspace_size(B, S, Hq, D) bytes: the status
+ *                header, then the running fp32 O [B*S*Hq][D] and LSE [B*S*Hq]
+ * D in {64, 128}. One kernel launch per (pair, head offset), each reading the
+ * kept rows straight from q, k, v through strided TMA tensor maps, plus an
+ * initialisation and a final merge launch. Scale 1/sqrt(D).
+ */
+#define USP_DILATED_MAX_PAIRS 16
+size_t usp_dilated_workspace_size(int B, int S, int Hq, int D);
+int usp_dilated_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
+                         int Hkv, int D, int causal, int n_pairs, const int* w, const int* r, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/*
+ * usp_workspace_status for the static scratch of usp_attn_bwd_noalloc (which a
+ * caller cannot name): synchronises `stream`, returns USP_ERR_TIMEOUT if a
+ * kernel of an earlier usp_attn_bwd_noalloc call on the current device recorded
+ * a timed-out wait (and clears the word), USP_OK otherwise; `site` (may be
+ * NULL) receives the recorded site code. Allocates nothing.
+ */
+int usp_attn_bwd_noalloc_status(int* site, void* stream);
 
 /*
  * Log-sum-exp merge of n_parts ring-step partials (the partial results each
@@ -206,7 +289,10 @@ int usp_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
  * every LSE_t = -inf yields O = 0, LSE = -inf.
  *   o_parts    [n_parts][rows][D] fp32;  lse_parts [n_parts][rows] fp32
  *   out        [rows][D], bf16 or fp32 (out_dtype);  lse_out [rows] fp32
- * D must be a multiple of 4 (<= 256).
+ * D must be a multiple of 4 (<= 256). With out_dtype USP_F32 the merge may run
+ * in place: out == o_parts and lse_out == lse_parts (partial 0 is overwritten
+ * by the result), which is how the stepwise forward streams its ring merge.
+ * Any other overlap of the outputs with the inputs is undefined.
  */
 int usp_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,
                   int out_dtype, float* lse_out, void* stream);

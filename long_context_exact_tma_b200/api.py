@@ -65,6 +65,41 @@ def head2seq(x: torch.Tensor, P_u: int, P_r: int, out=None, stream=None) -> torc
     return out
 
 
+def seq2head_many(xs, P_u: int, P_r: int, outs=None, stream=None):
+    """The seq->head all-to-all of several rank-major tensors [P, B, S/P, H_x, D_x]
+    (e.g. Q, K, V) in one launch; returns the head-sharded tensors."""
+    _require_cuda(*xs)
+    outs = list(outs) if outs is not None else [None] * len(xs)
+    jobs = []
+    for x_, (x, o) in enumerate(zip(xs, outs)):
+        P, B, c2, H, D = x.shape
+        if o is None:
+            o = torch.empty((P_r, P_u, B, P * c2 // P_r, H // P_u, D), dtype=x.dtype, device=x.device)
+            outs[x_] = o
+        jobs.append((x, o, H, D, _dt(x)))
+    P, B, c2 = xs[0].shape[:3]
+    B_.usp_permute_batch(B_.USP_MAP_SEQ2HEAD, jobs, B, P * c2, P_u, P_r, stream)
+    return outs
+
+
+def head2seq_many(xs, P_u: int, P_r: int, outs=None, stream=None):
+    """The head->seq regather of several head-sharded tensors (e.g. dQ, dK, dV)
+    in one launch; returns the rank-major tensors [P, B, S/P, H_x, D_x]."""
+    _require_cuda(*xs)
+    outs = list(outs) if outs is not None else [None] * len(xs)
+    jobs = []
+    P = P_u * P_r
+    for x_, (x, o) in enumerate(zip(xs, outs)):
+        Pr, Pu, B, L, Hl, D = x.shape
+        if o is None:
+            o = torch.empty((P, B, L * P_r // P, Hl * P_u, D), dtype=x.dtype, device=x.device)
+            outs[x_] = o
+        jobs.append((x, o, Hl * P_u, D, _dt(x)))
+    Pr, Pu, B, L = xs[0].shape[:4]
+    B_.usp_permute_batch(B_.USP_MAP_HEAD2SEQ, jobs, B, L * P_r, P_u, P_r, stream)
+    return outs
+
+
 def to_head_sharded(x, P_u, P_r, stream=None):
     return seq2head(zigzag_shard(x, P_u, P_r, stream=stream), P_u, P_r, stream=stream)
 
@@ -78,10 +113,19 @@ def workspace(nbytes: int, device) -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def check_workspace(ws: torch.Tensor, stream=None) -> None:
+    """Synchronise the stream and raise UspError(USP_ERR_TIMEOUT) if a kernel that
+    used `ws` recorded a timed-out device wait (the word is cleared by the read)."""
+    rc, site = B_.usp_workspace_status(ws, stream)
+    if rc != B_.USP_OK:
+        raise B_.UspError(rc, f"device wait timed out (site {site:#x}): {B_.usp_last_error()}")
+
+
 def attn_fwd(q, k, v, causal: bool, P_u: int, P_r: int, mode: int = B_.USP_MODE_FUSED,
-             ws: torch.Tensor | None = None, out=None, lse=None, stream=None):
+             ws: torch.Tensor | None = None, out=None, lse=None, stream=None, check_status: bool = False):
     """Forward over head-sharded q [P_r, P_u, B, L, Hq/P_u, D], k/v [..., Hkv/P_u, D].
-    Returns (out bf16 like q, lse fp32 [P_r, P_u, B, L, Hq/P_u])."""
+    Returns (out bf16 like q, lse fp32 [P_r, P_u, B, L, Hq/P_u]). With
+    check_status=True the call synchronises and raises on a timed-out device wait."""
     _require_cuda(q, k, v)
     Pr, Pu, B, L, Hql, D = q.shape
     Hkv = k.shape[4] * P_u
@@ -93,12 +137,15 @@ def attn_fwd(q, k, v, causal: bool, P_u: int, P_r: int, mode: int = B_.USP_MODE_
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device) if lse is None else lse
     B_.usp_attn_fwd(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, P_u, P_r, mode, ws, ws.numel(), stream)
+    if check_status:
+        check_workspace(ws, stream)
     return out, lse
 
 
 def attn_bwd(q, k, v, out, lse, dO, causal: bool, P_u: int, P_r: int, ws=None, dq=None, dk=None, dv=None,
-             stream=None):
-    """Backward; returns (dQ bf16 like q, dK fp32 like k, dV fp32 like v)."""
+             stream=None, check_status: bool = False):
+    """Backward; returns (dQ bf16 like q, dK fp32 like k, dV fp32 like v). With
+    check_status=True the call synchronises and raises on a timed-out device wait."""
     _require_cuda(q, k, v, out, lse, dO)
     Pr, Pu, B, L, Hql, D = q.shape
     Hkv = k.shape[4] * P_u
@@ -112,7 +159,26 @@ def attn_bwd(q, k, v, out, lse, dO, causal: bool, P_u: int, P_r: int, ws=None, d
     dv = torch.empty(v.shape, dtype=torch.float32, device=v.device) if dv is None else dv
     B_.usp_attn_bwd(q, k, v, out, lse, dO, dq, dk, dv, B, S, Hq, Hkv, D, causal, P_u, P_r, ws, ws.numel(),
                     stream)
+    if check_status:
+        check_workspace(ws, stream)
     return dq, dk, dv
+
+
+def dilated_attn_fwd(q, k, v, causal: bool, pairs, ws=None, out=None, lse=None, stream=None,
+                     check_status: bool = False):
+    """LongNet dilated attention over global-layout q [B, S, Hq, D], k/v [B, S, Hkv, D]
+    for the (w, r) pairs `pairs`. Returns (out bf16 like q, lse fp32 [B, S, Hq])."""
+    _require_cuda(q, k, v)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if ws is None:
+        ws = workspace(B_.usp_dilated_workspace_size(B, S, Hq, D), q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device) if lse is None else lse
+    B_.usp_dilated_attn_fwd(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, pairs, ws, ws.numel(), stream)
+    if check_status:
+        check_workspace(ws, stream)
+    return out, lse
 
 
 def lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype=torch.bfloat16, stream=None):

@@ -24,6 +24,19 @@ USP_BF16 = 0
 USP_F32 = 1
 USP_MODE_FUSED = 0
 USP_MODE_STEPWISE = 1
+USP_MAP_ZIGZAG_SHARD = 0
+USP_MAP_ZIGZAG_UNSHARD = 1
+USP_MAP_SEQ2HEAD = 2
+USP_MAP_HEAD2SEQ = 3
+USP_MAX_PERMUTE_JOBS = 4
+USP_DILATED_MAX_PAIRS = 16
+
+
+class PermuteJob(ctypes.Structure):
+    """usp_permute_job of include/usp.h."""
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("H", ctypes.c_int), ("D", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
 
 # name -> (restype, argtypes); mirrors include/usp.h
 _P = ctypes.c_void_p
@@ -34,17 +47,22 @@ _LAYOUT = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
 SIGNATURES = {
     "usp_version": (_I, []),
     "usp_last_error": (ctypes.c_char_p, []),
+    "usp_launch_count": (ctypes.c_ulonglong, []),
     "usp_zigzag_shard": (_I, _LAYOUT),
     "usp_zigzag_unshard": (_I, _LAYOUT),
     "usp_seq2head_permute": (_I, _LAYOUT),
     "usp_head2seq_permute": (_I, _LAYOUT),
+    "usp_permute_batch": (_I, [_I, ctypes.POINTER(PermuteJob), _I, _I, _I, _I, _I, _P]),
     "usp_attn_workspace_size": (_SZ, [_I] * 10),
+    "usp_dilated_workspace_size": (_SZ, [_I] * 4),
+    "usp_dilated_attn_fwd": (_I, [_P] * 5 + [_I] * 7 + [_P, _P, _P, _SZ, _P]),
     "usp_attn_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_P, _SZ, _P]),
     "usp_attn_bwd": (_I, [_P] * 9 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_prepare": (_I, [_P, _P, _P] + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_dkdv": (_I, [_P] * 6 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_dq": (_I, [_P] * 5 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 8 + [_P]),
+    "usp_attn_bwd_noalloc_status": (_I, [_P, _P]),
     "usp_lse_merge": (_I, [_P, _P, _I, _LL, _I, _P, _I, _P, _P]),
     "usp_bwd_preprocess": (_I, [_P, _P, _P, _LL, _I, _P]),
     "usp_workspace_status": (_I, [_P, _P, _P]),
@@ -102,6 +120,10 @@ def usp_version() -> int:
     return lib().usp_version()
 
 
+def usp_launch_count() -> int:
+    return int(lib().usp_launch_count())
+
+
 def usp_last_error() -> str:
     return lib().usp_last_error().decode()
 
@@ -127,8 +149,32 @@ def usp_head2seq_permute(src, dst, B, S, H, D, dtype, P_u, P_r, stream=None, che
     return _layout("usp_head2seq_permute", src, dst, B, S, H, D, dtype, P_u, P_r, stream, check)
 
 
+def usp_permute_batch(map_, jobs, B, S, P_u, P_r, stream=None, check=True):
+    """jobs: sequence of (src, dst, H, D, dtype)."""
+    arr = (PermuteJob * max(len(jobs), 1))()
+    for x, (src, dst, H, D, dtype) in enumerate(jobs):
+        arr[x] = PermuteJob(_ptr(src), _ptr(dst), H, D, dtype)
+    rc = lib().usp_permute_batch(map_, arr, len(jobs), B, S, P_u, P_r, _stream(stream))
+    return _check(rc) if check else rc
+
+
 def usp_attn_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, mode, bwd) -> int:
     return int(lib().usp_attn_workspace_size(B, S, Hq, Hkv, D, int(causal), P_u, P_r, mode, int(bwd)))
+
+
+def usp_dilated_workspace_size(B, S, Hq, D) -> int:
+    return int(lib().usp_dilated_workspace_size(B, S, Hq, D))
+
+
+def usp_dilated_attn_fwd(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, pairs, workspace, ws_bytes, stream=None,
+                         check=True):
+    """pairs: sequence of (w, r)."""
+    n = len(pairs)
+    w = (ctypes.c_int * max(n, 1))(*[int(p[0]) for p in pairs])
+    r = (ctypes.c_int * max(n, 1))(*[int(p[1]) for p in pairs])
+    rc = lib().usp_dilated_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D, int(causal),
+                                    n, w, r, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
 
 
 def usp_attn_fwd(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, P_u, P_r, mode, workspace, ws_bytes,
@@ -172,6 +218,13 @@ def usp_attn_bwd_noalloc(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, ca
     rc = lib().usp_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO), _ptr(dQ),
                                     _ptr(dK), _ptr(dV), B, S, Hq, Hkv, D, int(causal), P_u, P_r, _stream(stream))
     return _check(rc) if check else rc
+
+
+def usp_attn_bwd_noalloc_status(stream=None):
+    """(status, site) of the static scratch's status word; clears it."""
+    site = ctypes.c_int(0)
+    rc = lib().usp_attn_bwd_noalloc_status(ctypes.byref(site), _stream(stream))
+    return rc, site.value
 
 
 def usp_lse_merge(o_parts, lse_parts, n_parts, rows, D, out, out_dtype, lse_out, stream=None, check=True):

@@ -6,6 +6,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/usp.h"
@@ -65,6 +66,30 @@ int run_layout(int map, const void* src, void* dst, int B, int S, int H, int D, 
   return e == cudaSuccess ? USP_OK : cuda_fail(e, "layout kernel launch");
 }
 
+int run_layout_batch(int map, const usp_permute_job* jobs, int n, int B, int S, int P_u, int P_r, void* stream) {
+  if (map < kZigzagShard || map > kHead2Seq) return fail(USP_ERR_INVALID_ARG, "bad map %d", map);
+  if (!jobs || n <= 0 || n > kMaxLayoutJobs)
+    return fail(USP_ERR_INVALID_ARG, "n_jobs must be 1..%d with a job array", kMaxLayoutJobs);
+  LayoutArgs a[kMaxLayoutJobs];
+  for (int x = 0; x < n; ++x) {
+    const usp_permute_job& j = jobs[x];
+    const int rc = check_layout(j.src, j.dst, B, S, j.H, j.D, j.dtype, P_u, P_r);
+    if (rc != USP_OK) {
+      char why[sizeof g_err];
+      snprintf(why, sizeof why, "%s", g_err);
+      return fail(rc, "job %d: %s", x, why);
+    }
+    a[x] = LayoutArgs{};
+    a[x].src = static_cast<const uint8_t*>(j.src);
+    a[x].dst = static_cast<uint8_t*>(j.dst);
+    a[x].map = map;
+    a[x].B = B; a[x].S = S; a[x].H = j.H; a[x].P_u = P_u; a[x].P_r = P_r;
+    a[x].row_bytes = static_cast<uint32_t>(j.D * elem_size(j.dtype));
+  }
+  cudaError_t e = launch_layout_batch(a, n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? USP_OK : cuda_fail(e, "layout kernel launch");
+}
+
 int check_geom(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, AttnGeom* g) {
   if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || P_u <= 0 || P_r <= 0)
     return fail(USP_ERR_INVALID_ARG, "sizes must be positive");
@@ -117,11 +142,39 @@ int make_tmap(CUtensorMap* m, const void* base, int D, int H_l, int L, int n_rb)
   return USP_OK;
 }
 
+}  // namespace
+
+namespace usp {
+// Tensor map of a bf16 tensor viewed as 4-D {D, H, rows, n4}: head rows of D
+// elements 2*D bytes apart, `rows` rows row_stride bytes apart and n4 blocks
+// stride4 bytes apart; box 64 x 1 x 128 x 1, 128-byte swizzle.
+int make_tmap_strided(CUtensorMap* m, const void* base, int D, int H, long long rows, long long n4,
+                      unsigned long long row_stride, unsigned long long stride4) {
+  auto fn = encode_fn();
+  if (!fn) return record_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(n4)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, row_stride, stride4};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return record_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return USP_OK;
+}
+unsigned long long current_wait_ns() { return g_wait_ns; }
+}  // namespace usp
+
+namespace {
+
 size_t rows_of(const AttnGeom& g) { return static_cast<size_t>(g.B) * g.S * g.Hq; }
 
+// Stepwise mode streams the merge: two fp32 partials, the running merge of the
+// steps done so far (slot 0) and the current step's partial (slot 1).
 size_t fwd_ws(const AttnGeom& g, int mode) {
   if (mode == USP_MODE_FUSED) return kStatusBytes;
-  return kStatusBytes + static_cast<size_t>(g.P_r) * rows_of(g) * (4 * static_cast<size_t>(g.D) + 4);
+  return kStatusBytes + 2 * rows_of(g) * (4 * static_cast<size_t>(g.D) + 4);
 }
 int padded_L(const AttnGeom& g) { return (g.L + 127) / 128 * 128; }
 // [status][-LSE*log2e per head: n_rb*Hq_l*Lp][-Delta per head: same]
@@ -133,6 +186,11 @@ size_t bwd_ws(const AttnGeom& g) {
 }  // namespace
 
 namespace usp {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 // Records `msg` as this thread's last error and returns `code` (for entry points in other files).
 int record_error(int code, const char* fmt, ...) {
   va_list ap;
@@ -148,6 +206,8 @@ extern "C" {
 int usp_version(void) { return 100; }
 
 const char* usp_last_error(void) { return g_err; }
+
+unsigned long long usp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 void usp_set_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns; }
 
@@ -166,6 +226,15 @@ int usp_seq2head_permute(const void* src, void* dst, int B, int S, int H, int D,
 int usp_head2seq_permute(const void* src, void* dst, int B, int S, int H, int D, int dtype, int P_u, int P_r,
                          void* stream) {
   return run_layout(kHead2Seq, src, dst, B, S, H, D, dtype, P_u, P_r, stream);
+}
+
+int usp_permute_batch(int map, const usp_permute_job* jobs, int n_jobs, int B, int S, int P_u, int P_r,
+                      void* stream) {
+  static_assert(USP_MAX_PERMUTE_JOBS == kMaxLayoutJobs, "job limit");
+  static_assert(USP_MAP_SEQ2HEAD == kSeq2Head && USP_MAP_HEAD2SEQ == kHead2Seq && USP_MAP_ZIGZAG_SHARD == kZigzagShard &&
+                    USP_MAP_ZIGZAG_UNSHARD == kZigzagUnshard,
+                "map codes");
+  return run_layout_batch(map, jobs, n_jobs, B, S, P_u, P_r, stream);
 }
 
 size_t usp_attn_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, int mode,
@@ -207,18 +276,27 @@ int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
     e = launch_attn_fwd(L, st);
     return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention forward launch");
   }
+  // The ring step for step: step t's partial goes to slot 1 (step 0's to slot 0)
+  // and is folded into the running result in slot 0 by the log-sum-exp merge,
+  // 2 partials in and 1 out; the last step's merge writes O (bf16) and LSE.
   const size_t rows = rows_of(g);
   float* o_parts = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
-  float* lse_parts = o_parts + static_cast<size_t>(P_r) * rows * D;
+  float* lse_parts = o_parts + 2 * rows * D;
   for (int t = 0; t < P_r; ++t) {
+    const int slot = t == 0 ? 0 : 1;
     L.step = t;
-    L.o_part = o_parts + static_cast<size_t>(t) * rows * D;
-    L.lse_part = lse_parts + static_cast<size_t>(t) * rows;
+    L.o_part = o_parts + static_cast<size_t>(slot) * rows * D;
+    L.lse_part = lse_parts + static_cast<size_t>(slot) * rows;
     e = launch_attn_fwd(L, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention forward (step) launch");
+    const bool last = t == P_r - 1;
+    if (t == 0 && !last) continue;
+    e = last ? launch_lse_merge(o_parts, lse_parts, t == 0 ? 1 : 2, static_cast<long long>(rows), D, out, 0, lse,
+                                st)
+             : launch_lse_merge(o_parts, lse_parts, 2, static_cast<long long>(rows), D, o_parts, 1, lse_parts, st);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
-  e = launch_lse_merge(o_parts, lse_parts, P_r, static_cast<long long>(rows), D, out, 0, lse, st);
-  return e == cudaSuccess ? USP_OK : cuda_fail(e, "merge launch");
+  return USP_OK;
 }
 
 int usp_attn_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,

@@ -464,6 +464,7 @@ cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   attn_bwd_dq_kernel<D><<<static_cast<unsigned>(blocks), kThreadsDq, C::kSmemBytes, stream>>>(
       L.tm_q, L.tm_k, L.tm_v, L.tm_do, a);
+  note_launch();
   return cudaGetLastError();
 }
 

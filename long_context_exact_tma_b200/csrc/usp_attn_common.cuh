@@ -36,8 +36,11 @@ inline Geo make_geo(const AttnGeom& a) {
   return g;
 }
 
-// Original token position of local token tau of ring rank i (tau < L).
+// Original token position of local token tau of ring rank i (tau < L). With
+// kPlain (the one-rank geometry of the sub-problem mode) tau is the position.
+template <bool kPlain = false>
 __device__ __forceinline__ int token_pos(const Geo& g, int i, int tau) {
+  if (kPlain) return tau;
   const int kappa = tau / g.c;
   const int rp = i * g.P_u + (kappa >> 1);
   const int chunk = (kappa & 1) ? (2 * g.P - 1 - rp) : rp;
@@ -45,11 +48,17 @@ __device__ __forceinline__ int token_pos(const Geo& g, int i, int tau) {
 }
 
 // Smallest and largest original position among local tokens [t0, t1) of ring rank i.
+template <bool kPlain = false>
 __device__ __forceinline__ void pos_range(const Geo& g, int i, int t0, int t1, int& pmin, int& pmax) {
   if (t1 > g.L) t1 = g.L;
   pmin = INT_MAX;
   pmax = -1;
   if (t0 >= t1) return;  // the range lies wholly in the padding past L
+  if (kPlain) {
+    pmin = t0;
+    pmax = t1 - 1;
+    return;
+  }
   for (int kap = t0 / g.c; kap * g.c < t1; ++kap) {
     const int a = max(t0, kap * g.c);
     const int e = min(t1, (kap + 1) * g.c) - 1;
@@ -78,12 +87,13 @@ __device__ __forceinline__ void tile_in_position_order(const Geo& g, int o, int&
 enum TileKind { kSkip = 0, kFull = 1, kMasked = 2 };
 
 // Kind of the pair (query tile with positions [qmin, qmax], key tile n of ring rank j).
+template <bool kPlain = false>
 __device__ __forceinline__ int classify_tile(const Geo& g, int qmin, int qmax, int j, int n) {
   const int k0 = n * kBN;
   const bool ragged = k0 + kBN > g.L;
   if (!g.causal) return ragged ? kMasked : kFull;
   int kmin, kmax;
-  pos_range(g, j, k0, k0 + kBN, kmin, kmax);
+  pos_range<kPlain>(g, j, k0, k0 + kBN, kmin, kmax);
   if (qmax < kmin) return kSkip;
   if (qmin >= kmax && !ragged) return kFull;
   return kMasked;
@@ -98,11 +108,12 @@ struct KvWalk {
   bool valid;
 };
 
+template <bool kPlain = false>
 __device__ __forceinline__ void kv_walk_settle(const Geo& g, int i, int qmin, int qmax, int t_end, KvWalk& w) {
   while (w.t < t_end) {
     w.j = (i - w.t + g.P_r) % g.P_r;
     while (w.n < g.n_ktiles) {
-      w.kind = classify_tile(g, qmin, qmax, w.j, w.n);
+      w.kind = classify_tile<kPlain>(g, qmin, qmax, w.j, w.n);
       if (w.kind != kSkip) {
         w.valid = true;
         return;
@@ -115,15 +126,17 @@ __device__ __forceinline__ void kv_walk_settle(const Geo& g, int i, int qmin, in
   w.valid = false;
 }
 
+template <bool kPlain = false>
 __device__ __forceinline__ KvWalk kv_walk_begin(const Geo& g, int i, int qmin, int qmax, int t_begin, int t_end) {
   KvWalk w{t_begin, 0, 0, 0, false};
-  kv_walk_settle(g, i, qmin, qmax, t_end, w);
+  kv_walk_settle<kPlain>(g, i, qmin, qmax, t_end, w);
   return w;
 }
 
+template <bool kPlain = false>
 __device__ __forceinline__ void kv_walk_next(const Geo& g, int i, int qmin, int qmax, int t_end, KvWalk& w) {
   ++w.n;
-  kv_walk_settle(g, i, qmin, qmax, t_end, w);
+  kv_walk_settle<kPlain>(g, i, qmin, qmax, t_end, w);
 }
 
 }  // namespace usp

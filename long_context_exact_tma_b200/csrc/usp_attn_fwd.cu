@@ -68,6 +68,7 @@ struct FwdArgs {
   int step;  // -1 fused, else the ring step
   int* status;
   unsigned long long wait_ns;
+  FwdSub sub;  // sub-problem mode (kSub): see usp_internal.h
 };
 
 struct FwdBars {
@@ -102,7 +103,7 @@ __device__ __forceinline__ void pair_in_position_order(const Geo& g, int o, int&
   }
 }
 
-template <int D>
+template <int D, bool kSub>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -115,24 +116,37 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
 
-  const Geo& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // Work item: CTAs of one (b, Ulysses rank, head) run together so that its K/V
-  // stay in L2; inside it, query-tile pairs in decreasing original position
-  // (the causally heaviest first).
-  const int np = (g.n_qtiles + 1) / 2;
-  const int n_pairs = g.P_r * np;
-  int wi = blockIdx.x;
-  const int order = n_pairs - 1 - wi % n_pairs;
-  wi /= n_pairs;
-  const int h = wi % g.Hq_l;
-  wi /= g.Hq_l;
-  const int u = wi % g.P_u;
-  const int b = wi / g.P_u;
-  int i, m;
-  pair_in_position_order(g, order, i, m);
-  const int rank = i * g.P_u + u;
+  const Geo& g = a.g;  // in the sub-problem mode: the one-rank geometry of every problem
+  int h, u, b, i, m, qc4;
+  if constexpr (kSub) {
+    // work item: (problem, head, pair of query tiles), the pairs of a (problem,
+    // head) heaviest first
+    const int np = (g.n_qtiles + 1) / 2;
+    int wi = blockIdx.x;
+    const int order = np - 1 - wi % np;
+    wi /= np;
+    h = a.sub.h0 + (wi % a.sub.n_heads) * a.sub.h_step;
+    qc4 = wi / a.sub.n_heads;  // the problem
+    u = b = i = 0;
+    m = 2 * order;
+  } else {
+    // Work item: CTAs of one (b, Ulysses rank, head) run together so that its K/V
+    // stay in L2; inside it, query-tile pairs in decreasing original position
+    // (the causally heaviest first).
+    const int np = (g.n_qtiles + 1) / 2;
+    const int n_pairs = g.P_r * np;
+    int wi = blockIdx.x;
+    const int order = n_pairs - 1 - wi % n_pairs;
+    wi /= n_pairs;
+    h = wi % g.Hq_l;
+    wi /= g.Hq_l;
+    u = wi % g.P_u;
+    b = wi / g.P_u;
+    pair_in_position_order(g, order, i, m);
+    qc4 = 0;
+  }
+  const int rank = kSub ? 0 : i * g.P_u + u;
   const int kvh = h / g.G;
   const int q0 = m * kBM;
   const int t_begin = a.step < 0 ? 0 : a.step;
@@ -171,10 +185,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     // lane issues each copy and barrier operation.
     {
       int qmin0, qmax0, qmin1, qmax1;
-      pos_range(g, i, q0, q0 + kBM, qmin0, qmax0);
-      pos_range(g, i, q0 + kBM, q0 + 2 * kBM, qmin1, qmax1);
+      pos_range<kSub>(g, i, q0, q0 + kBM, qmin0, qmax0);
+      pos_range<kSub>(g, i, q0 + kBM, q0 + 2 * kBM, qmin1, qmax1);
       const int qmin = min(qmin0, qmin1), qmax = max(qmax0, qmax1);
-      KvWalk kw = kv_walk_begin(g, i, qmin, qmax, t_begin, t_end);
+      KvWalk kw = kv_walk_begin<kSub>(g, i, qmin, qmax, t_begin, t_end);
       int issued = 0;
       const bool any = kw.valid;
       if (any) {
@@ -188,7 +202,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         for (int t = 0; t < 2; ++t)
           for (int p = 0; p < C::kPanels; ++p)
             tma_load_4d_w(&tm_q, &bars->q_full, sQ + t * C::kTileBytes + p * C::kPanelBytes, p * 64, h,
-                          q0 + t * kBM, rank * g.B + b);
+                          q0 + t * kBM, kSub ? qc4 : rank * g.B + b);
       }
       while (true) {
         const int s = issued % C::kStages;
@@ -203,7 +217,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           break;
         }
         const int kinds =
-            classify_tile(g, qmin0, qmax0, kw.j, kw.n) | (classify_tile(g, qmin1, qmax1, kw.j, kw.n) << 4);
+            classify_tile<kSub>(g, qmin0, qmax0, kw.j, kw.n) | (classify_tile<kSub>(g, qmin1, qmax1, kw.j, kw.n) << 4);
         if (lane == 0) {
           slot[0] = 1;
           slot[1] = kw.j;
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           slot[3] = kinds;
         }
         __syncwarp();
-        const int krb = (kw.j * g.P_u + u) * g.B + b;
+        const int krb = kSub ? qc4 : (kw.j * g.P_u + u) * g.B + b;
         mbar_expect_tx_w(&bars->k_full[s], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_4d_w(&tm_k, &bars->k_full[s], sK + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           tma_load_4d_w(&tm_v, &bars->v_full[s], sV + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
                         kw.n * kBN, krb);
         ++issued;
-        kv_walk_next(g, i, qmin, qmax, t_end, kw);
+        kv_walk_next<kSub>(g, i, qmin, qmax, t_end, kw);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         // Let every copy this warp started land before the CTA exits.
@@ -307,7 +321,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t cS = col_s(t), cO = col_o(t);
     const int tau_q = q0 + t * kBM + row;
-    const int pos_q = tau_q < g.L ? token_pos(g, i, tau_q) : INT_MAX;
+    const int pos_q = tau_q < g.L ? token_pos<kSub>(g, i, tau_q) : INT_MAX;
     const bool aligned = (g.c % kBN) == 0;
     // l_run: sum of the fp32 weights (for LSE); lb_run: sum of the bf16-rounded
     // weights the PV UMMA consumes (normalises O, so O stays a convex combination
@@ -329,7 +343,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       if (kkind != kFull) {
         const int k0 = kn * kBN;
         int lim = kkind == kSkip ? -1 : min(127, g.L - k0 - 1);  // keys at or past L are padding
-        if (kkind == kMasked && aligned && g.causal) lim = min(lim, pos_q - token_pos(g, kj, k0));
+        if (kkind == kMasked && aligned && g.causal) lim = min(lim, pos_q - token_pos<kSub>(g, kj, k0));
         const bool per_key = kkind == kMasked && !aligned;  // chunks shorter than a tile
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -341,7 +355,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
             vis = 0u;
             for (int c = 0; c < 32; ++c) {
               const int tau = k0 + c0 + c;
-              if (tau < g.L && (!g.causal || token_pos(g, kj, tau) <= pos_q)) vis |= 1u << c;
+              if (tau < g.L && (!g.causal || token_pos<kSub>(g, kj, tau) <= pos_q)) vis |= 1u << c;
             }
           }
           uint32_t r[32];
@@ -440,9 +454,53 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     if (ok) {
       tc_fence_after();
       const bool store = tau_q < g.L;
-      const size_t row_idx = (static_cast<size_t>(rank * g.B + b) * g.L + (store ? tau_q : 0)) * g.Hq_l + h;
       const float inv_l = lb_run > 0.f ? 1.f / lb_run : 0.f;
       const float lse_val = l_run > 0.f ? (m_use + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+      if constexpr (kSub) {
+        // fold this pair's (O_k, LSE_k) into the running fp32 (O, LSE) of the row:
+        // weights exp(LSE_k - LSE) and exp(LSE_old - LSE), LSE = logaddexp of both
+        const int pb = qc4 / a.sub.n_seg, ps = qc4 % a.sub.n_seg;
+        const size_t orow = static_cast<size_t>(pb) * a.sub.S + static_cast<size_t>(ps) * a.sub.w + a.sub.off +
+                            static_cast<size_t>(store ? tau_q : 0) * a.sub.r;
+        const size_t ridx = orow * a.sub.Hq + h;
+        float lse_old = -INFINITY;
+        if (store) lse_old = a.sub.lse_run[ridx];
+        const float mx = fmaxf(lse_old, lse_val);
+        float w_old = 0.f, w_new = 0.f, lse_new = -INFINITY;
+        if (mx != -INFINITY) {
+          const float e_old = ex2_approx((lse_old - mx) * 1.4426950408889634f);
+          const float e_new = ex2_approx((lse_val - mx) * 1.4426950408889634f);
+          const float inv = 1.f / (e_old + e_new);
+          w_old = e_old * inv;
+          w_new = e_new * inv * inv_l;
+          lse_new = mx + __logf(e_old + e_new);
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          if (it >= 1) {
+            tmem_ld32(trow + cO + c0, o);
+            tmem_ld_wait();
+            reg_fence32(o);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = 0u;
+          }
+          if (store) {
+            float4* dst = reinterpret_cast<float4*>(a.sub.o_run + ridx * D + c0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 ov = dst[q];
+              dst[q] = make_float4(ov.x * w_old + __uint_as_float(o[q * 4 + 0]) * w_new,
+                                   ov.y * w_old + __uint_as_float(o[q * 4 + 1]) * w_new,
+                                   ov.z * w_old + __uint_as_float(o[q * 4 + 2]) * w_new,
+                                   ov.w * w_old + __uint_as_float(o[q * 4 + 3]) * w_new);
+            }
+          }
+        }
+        if (store) a.sub.lse_run[ridx] = lse_new;
+      } else {
+      const size_t row_idx = (static_cast<size_t>(rank * g.B + b) * g.L + (store ? tau_q : 0)) * g.Hq_l + h;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -481,6 +539,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         else
           a.lse_part[row_idx] = lse_val;
       }
+      }  // USP epilogue
     }
   }
 
@@ -492,11 +551,11 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   }
 }
 
-template <int D>
+template <int D, bool kSub>
 cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
   using C = FwdCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, kSub>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a{};
@@ -508,20 +567,37 @@ cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
   a.step = L.step;
   a.status = L.status;
   a.wait_ns = L.wait_ns;
-  const long long blocks =
-      static_cast<long long>((a.g.n_qtiles + 1) / 2) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;
+  a.sub = L.sub;
+  long long blocks;
+  if (kSub) {
+    // every problem: one rank, L = sub.L rows whose local index is the position
+    // (contiguous, so the aligned masking path applies)
+    a.g.P_u = a.g.P_r = a.g.P = a.g.n_ranks = 1;
+    a.g.L = L.sub.L;
+    a.g.c = kBN;
+    a.g.n_qtiles = a.g.n_ktiles = (L.sub.L + kBM - 1) / kBM;
+    blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * L.sub.n_heads * L.sub.n_prob;
+  } else {
+    blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;
+  }
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  attn_fwd_kernel<D><<<static_cast<unsigned>(blocks), kThreadsFwd, C::kSmemBytes, stream>>>(L.tm_q, L.tm_k,
-                                                                                           L.tm_v, a);
+  attn_fwd_kernel<D, kSub><<<static_cast<unsigned>(blocks), kThreadsFwd, C::kSmemBytes, stream>>>(L.tm_q, L.tm_k,
+                                                                                                 L.tm_v, a);
+  note_launch();
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_fwd(const FwdLaunch& L, cudaStream_t stream) {
-  if (L.g.D == 128) return launch_fwd_d<128>(L, stream);
-  if (L.g.D == 64) return launch_fwd_d<64>(L, stream);
+  if (L.sub.active) {
+    if (L.g.D == 128) return launch_fwd_d<128, true>(L, stream);
+    if (L.g.D == 64) return launch_fwd_d<64, true>(L, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (L.g.D == 128) return launch_fwd_d<128, false>(L, stream);
+  if (L.g.D == 64) return launch_fwd_d<64, false>(L, stream);
   return cudaErrorInvalidValue;
 }
 

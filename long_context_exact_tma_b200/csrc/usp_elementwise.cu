@@ -13,28 +13,31 @@ namespace usp {
 namespace {
 
 // One warp per row; lane l handles elements 4l, 4l+1, 4l+2, 4l+3 (+128 per pass).
+// The output may alias partial 0 (out == o_parts, lse_out == lse_parts): the
+// streamed ring merge folds each step into the running result in place. Every
+// element is read and then written by the same lane, and the row's LSE is
+// written only after the whole warp has read the partial LSEs (plain coherent
+// loads, no restrict: the buffers may overlap).
 template <bool kOutF32>
-__global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ o_parts,
-                                                        const float* __restrict__ lse_parts, int n_parts,
-                                                        long long rows, int D, void* __restrict__ out,
-                                                        float* __restrict__ lse_out) {
+__global__ void __launch_bounds__(256) lse_merge_kernel(const float* o_parts, const float* lse_parts, int n_parts,
+                                                        long long rows, int D, void* out, float* lse_out) {
   const int lane = threadIdx.x & 31;
   const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
        r += n_warps) {
     float m = -INFINITY;
-    for (int t = 0; t < n_parts; ++t) m = fmaxf(m, __ldg(lse_parts + static_cast<long long>(t) * rows + r));
+    for (int t = 0; t < n_parts; ++t) m = fmaxf(m, lse_parts[static_cast<long long>(t) * rows + r]);
     float lse = -INFINITY;
     if (m != -INFINITY) {
       float acc = 0.f;
-      for (int t = 0; t < n_parts; ++t) acc += expf(__ldg(lse_parts + static_cast<long long>(t) * rows + r) - m);
+      for (int t = 0; t < n_parts; ++t) acc += expf(lse_parts[static_cast<long long>(t) * rows + r] - m);
       lse = m + logf(acc);
     }
     for (int d4 = lane; d4 * 4 < D; d4 += 32) {
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
       if (lse != -INFINITY) {
         for (int t = 0; t < n_parts; ++t) {
-          const float lt = __ldg(lse_parts + static_cast<long long>(t) * rows + r);
+          const float lt = lse_parts[static_cast<long long>(t) * rows + r];
           if (lt == -INFINITY) continue;
           const float w = expf(lt - lse);
           const float4 p = __ldcs(reinterpret_cast<const float4*>(o_parts + (static_cast<long long>(t) * rows + r) * D) + d4);
@@ -53,6 +56,64 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
         reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + r * D)[d4] = packed;
       }
     }
+    __syncwarp();
+    if (lane == 0) lse_out[r] = lse;
+  }
+}
+
+// The merge of one or two partials with D <= 128 (the streamed ring merge: the
+// running result and one step's partial): every load of a row -- its partial
+// LSEs and its lane's float4 of each partial O -- is issued before any of them
+// is used, so a row costs one memory round trip. Alias-safe like the general
+// kernel above (out may be partial 0).
+template <bool kOutF32, int kN>
+__global__ void __launch_bounds__(256) lse_merge_small_kernel(const float* o_parts, const float* lse_parts,
+                                                              long long rows, int D, void* out, float* lse_out) {
+  const int lane = threadIdx.x & 31;
+  const bool active = lane * 4 < D;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += n_warps) {
+    float lt[kN];
+    float4 p[kN];
+#pragma unroll
+    for (int t = 0; t < kN; ++t) {
+      lt[t] = lse_parts[static_cast<long long>(t) * rows + r];
+      p[t] = active ? __ldcs(reinterpret_cast<const float4*>(o_parts + (static_cast<long long>(t) * rows + r) * D) +
+                             lane)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float m = lt[0];
+#pragma unroll
+    for (int t = 1; t < kN; ++t) m = fmaxf(m, lt[t]);
+    float lse = -INFINITY;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (m != -INFINITY) {
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < kN; ++t) acc += expf(lt[t] - m);
+      lse = m + logf(acc);
+#pragma unroll
+      for (int t = 0; t < kN; ++t) {
+        if (lt[t] == -INFINITY) continue;
+        const float w = expf(lt[t] - lse);
+        o.x += w * p[t].x;
+        o.y += w * p[t].y;
+        o.z += w * p[t].z;
+        o.w += w * p[t].w;
+      }
+    }
+    if (active) {
+      if (kOutF32) {
+        reinterpret_cast<float4*>(static_cast<float*>(out) + r * D)[lane] = o;
+      } else {
+        uint2 packed;
+        packed.x = pack_bf16x2(o.x, o.y);
+        packed.y = pack_bf16x2(o.z, o.w);
+        reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + r * D)[lane] = packed;
+      }
+    }
+    __syncwarp();
     if (lane == 0) lse_out[r] = lse;
   }
 }
@@ -134,6 +195,16 @@ __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16*
   }
 }
 
+// The empty running result of a merge: O = 0 (rows x D) and LSE = -inf (rows).
+__global__ void __launch_bounds__(256) fill_running_kernel(float4* __restrict__ o, float* __restrict__ lse,
+                                                           long long n4, long long rows) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < n4; x += stride)
+    o[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < rows; x += stride)
+    lse[x] = -INFINITY;
+}
+
 // Waits on an mbarrier that nothing completes; the bounded wait must give up.
 __global__ void wait_selftest_kernel(int* status, unsigned long long limit_ns) {
   __shared__ uint64_t bar;
@@ -170,10 +241,22 @@ cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n
                              void* out, int out_f32, float* lse_out, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = grid_for(8, rows);
-  if (out_f32)
+  if (D <= 128 && n_parts == 2) {
+    if (out_f32)
+      lse_merge_small_kernel<true, 2><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, rows, D, out, lse_out);
+    else
+      lse_merge_small_kernel<false, 2><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, rows, D, out, lse_out);
+  } else if (D <= 128 && n_parts == 1) {
+    if (out_f32)
+      lse_merge_small_kernel<true, 1><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, rows, D, out, lse_out);
+    else
+      lse_merge_small_kernel<false, 1><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, rows, D, out, lse_out);
+  } else if (out_f32) {
     lse_merge_kernel<true><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, n_parts, rows, D, out, lse_out);
-  else
+  } else {
     lse_merge_kernel<false><<<blocks, 256, 0, stream>>>(o_parts, lse_parts, n_parts, rows, D, out, lse_out);
+  }
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -183,6 +266,7 @@ cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta,
   bwd_preprocess_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
                                                                static_cast<const __nv_bfloat16*>(dO), delta,
                                                                rows, D);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -193,11 +277,21 @@ cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* l
   bwd_prep_rows_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
                                                               static_cast<const __nv_bfloat16*>(dO), lse, delta_t,
                                                               lse2_t, rows, L, Hl, D, Lp);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_running(float* o, float* lse, long long rows, int D, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const long long n4 = rows * D / 4;
+  fill_running_kernel<<<grid_for(256 * 4, n4), 256, 0, stream>>>(reinterpret_cast<float4*>(o), lse, n4, rows);
+  note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  note_launch();
   return cudaGetLastError();
 }
 

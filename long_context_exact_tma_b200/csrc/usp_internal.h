@@ -12,6 +12,20 @@ constexpr int kStatusBytes = 256;  // workspace header: device status word + pad
 // Sets the calling thread's usp_last_error() message; returns `code`.
 int record_error(int code, const char* fmt, ...);
 
+// Counts one kernel launch of this library (read by usp_launch_count).
+void note_launch();
+
+// The calling thread's bounded-wait limit (usp_set_wait_limit_ns).
+unsigned long long current_wait_ns();
+
+// Tensor map of a bf16 tensor viewed as {D, H, rows, n4} with the given row and
+// block strides in bytes (box 64 x 1 x 128 x 1, 128-byte swizzle); usp_status.
+int make_tmap_strided(CUtensorMap* m, const void* base, int D, int H, long long rows, long long n4,
+                      unsigned long long row_stride, unsigned long long stride4);
+
+// Fills a running fp32 (O, LSE) with the empty result: O = 0, LSE = -inf.
+cudaError_t launch_fill_running(float* o, float* lse, long long rows, int D, cudaStream_t stream);
+
 // Layout maps of the gather kernel (see usp_layout.cu).
 enum LayoutMap { kZigzagShard = 0, kZigzagUnshard = 1, kSeq2Head = 2, kHead2Seq = 3 };
 
@@ -23,6 +37,10 @@ struct LayoutArgs {
   uint32_t row_bytes;          // bytes of one head row (D * element size)
 };
 cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t stream);
+// Up to kMaxLayoutJobs gathers in one launch (each with its own map, shape and
+// element size).
+constexpr int kMaxLayoutJobs = 4;
+cudaError_t launch_layout_batch(const LayoutArgs* a, int n, cudaStream_t stream);
 
 cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D,
                              void* out, int out_f32, float* lse_out, cudaStream_t stream);
@@ -37,6 +55,21 @@ struct AttnGeom {
   int n_ranks;                  // P_r * P_u head-sharded ranks
 };
 
+// The forward's sub-problem mode: one launch over n_prob independent one-rank
+// problems of L rows each (plain order; the 4th TMA coordinate selects the
+// problem), query heads h0 + j*h_step (j < n_heads). The result of row tau of
+// problem p is folded into a running fp32 (O, LSE) at output row
+// (p / n_seg) * S + (p % n_seg) * w + off + tau * r by the log-sum-exp merge.
+// LongNet's dilated attention runs one such launch per (w, r) pair and head
+// offset off, with tensor maps that step r rows from the offset.
+struct FwdSub {
+  int active;
+  int n_prob, L, h0, h_step, n_heads;
+  int n_seg, w, off, r, S, Hq;
+  float* o_run;    // fp32 [B*S][Hq][D]
+  float* lse_run;  // fp32 [B*S][Hq]
+};
+
 struct FwdLaunch {
   AttnGeom g;
   CUtensorMap tm_q, tm_k, tm_v;
@@ -47,6 +80,7 @@ struct FwdLaunch {
   int step;           // ring step (stepwise) or -1 (fused)
   int* status;
   unsigned long long wait_ns;
+  FwdSub sub;         // sub-problem mode when sub.active
 };
 cudaError_t launch_attn_fwd(const FwdLaunch& a, cudaStream_t stream);
 

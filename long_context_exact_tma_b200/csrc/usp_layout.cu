@@ -6,12 +6,19 @@
 // 2P-1-r. Ulysses all-to-all (DeepSpeed-Ulysses summary, "Wie DeepSpeed-Ulysses
 // funktioniert"): rank (i,u) receives head group u of every rank (i,u').
 //
-// Each kernel thread group walks DESTINATION runs ("pull"): a run is a
-// contiguous row that is also contiguous in the source (a whole token of H
-// heads for the zigzag maps, the H/P_u heads of one group for the all-to-all).
-// Index math is done once per run, then the run is copied with 16-byte vectors
-// (4-byte words when the run is not a multiple of 16 bytes, e.g. LSE rows).
-// HBM-bound: 2 * tensor bytes of traffic per call.
+// The kernel walks DESTINATION runs ("pull"): a run is a contiguous row that is
+// also contiguous in the source (a whole token of H heads for the zigzag maps,
+// the H/P_u heads of one group for the all-to-all). One launch may move up to
+// kMaxLayoutJobs tensors with the same map and mesh (Q, K, V of a step; or dQ, dK,
+// dV), so launch and tail are paid once.
+//
+// Work is split into warp tasks of (nearly) equal size, four vectors per lane:
+// a long run is cut into pieces of 128 vectors (each group of 32 lanes reading
+// 512 contiguous bytes), shorter runs are packed several to a task. Warp w
+// takes tasks w, w + W, ... (W warps in the grid) two at a time, with all their
+// loads in flight before the stores, so that no warp has more than one task
+// more than another whatever the run length. The index math of a task is done
+// once, for its first run. HBM-bound: 2 x tensor bytes per job.
 #include "usp_internal.h"
 
 namespace usp {
@@ -24,6 +31,26 @@ struct RunMap {
   uint32_t run_bytes;  // bytes per run
   uint32_t n_runs;
   uint64_t row_bytes;  // bytes per head row
+};
+
+struct Job {
+  const uint8_t* src;
+  uint8_t* dst;
+  RunMap m;
+  uint32_t nvec;        // vectors per run
+  uint32_t lanes;       // lanes per run (32 for long and medium runs)
+  uint32_t pieces;      // tasks per run (long runs); 0 otherwise
+  uint32_t xslots;      // slots per run (medium runs)
+  uint32_t runs_per_task;
+  uint32_t seg;         // runs per contiguous source segment
+  uint64_t src_step;    // source bytes between consecutive runs of a segment
+  uint32_t task_begin;  // first flat task index of this job
+};
+
+struct Batch {
+  Job job[kMaxLayoutJobs];
+  int n_jobs;
+  uint32_t n_tasks;
 };
 
 // Byte offsets (src, dst) of destination run q.
@@ -63,34 +90,106 @@ __device__ __forceinline__ void run_offsets(const RunMap& m, uint32_t q, uint64_
   }
 }
 
-template <typename V, int kUnroll>
-__global__ void __launch_bounds__(256) layout_gather_kernel(const uint8_t* __restrict__ src,
-                                                            uint8_t* __restrict__ dst, RunMap m,
-                                                            uint32_t lanes_per_run) {
+constexpr int kSlots = 4;  // vectors a lane moves per task (one per slot)
+
+// Where this lane's vectors of flat task `task` are. A task is kSlots slots of
+// one 16-byte (or 4-byte) vector per lane:
+//   long runs (>= 128 vectors): slot x is vector piece*128 + 32x + lane of one run;
+//   medium runs (32..127 vectors): X = ceil(nvec/32) slots per run, 4/X runs;
+//   short runs (< 32 vectors): `lanes` lanes per run, 32/lanes runs per slot.
+// The offsets of a task's first run are computed once; the next runs of the
+// task lie `src_step` / run_bytes further on while they stay in the same
+// contiguous source segment of `seg` runs, else they are computed afresh.
+template <typename V>
+__device__ __forceinline__ void task_lane(const Batch& bt, uint32_t task, uint32_t lane, const V* (&s)[kSlots],
+                                          V* (&d)[kSlots]) {
+  int k = 0;
+#pragma unroll
+  for (int x = 1; x < kMaxLayoutJobs; ++x)
+    if (x < bt.n_jobs && task >= bt.job[x].task_begin) k = x;
+  const Job& jb = bt.job[k];
+  const uint32_t local = task - jb.task_begin;
+  if (jb.pieces > 0) {
+    const uint32_t run = local / jb.pieces;
+    const uint32_t v0 = (local % jb.pieces) * (32 * kSlots) + lane;
+    uint64_t so, dof;
+    run_offsets(jb.m, run, so, dof);
+    const V* sp = reinterpret_cast<const V*>(jb.src + so);
+    V* dp = reinterpret_cast<V*>(jb.dst + dof);
+#pragma unroll
+    for (int x = 0; x < kSlots; ++x) {
+      const uint32_t vec = v0 + 32 * x;
+      s[x] = vec < jb.nvec ? sp + vec : nullptr;
+      d[x] = dp + vec;
+    }
+    return;
+  }
+  const uint32_t q0 = local * jb.runs_per_task;
+  uint64_t so0, dof0;
+  run_offsets(jb.m, q0, so0, dof0);
+  const uint32_t in_seg = q0 % jb.seg;
+  const bool medium = jb.lanes == 32;
+#pragma unroll
+  for (int x = 0; x < kSlots; ++x) {
+    uint32_t dq, vec;
+    bool ok;
+    if (medium) {
+      dq = x / jb.xslots;
+      vec = (x % jb.xslots) * 32 + lane;
+      ok = dq < jb.runs_per_task;
+    } else {
+      dq = x * (32 / jb.lanes) + lane / jb.lanes;
+      vec = lane % jb.lanes;
+      ok = true;
+    }
+    const uint32_t q = q0 + dq;
+    ok = ok && q < jb.m.n_runs && vec < jb.nvec;
+    s[x] = nullptr;
+    d[x] = nullptr;
+    if (ok) {
+      uint64_t so, dof;
+      if (in_seg + dq < jb.seg) {
+        so = so0 + static_cast<uint64_t>(dq) * jb.src_step;
+        dof = dof0 + static_cast<uint64_t>(dq) * jb.m.run_bytes;
+      } else {
+        run_offsets(jb.m, q, so, dof);
+      }
+      s[x] = reinterpret_cast<const V*>(jb.src + so) + vec;
+      d[x] = reinterpret_cast<V*>(jb.dst + dof) + vec;
+    }
+  }
+}
+
+template <typename V>
+__global__ void __launch_bounds__(256) layout_gather_kernel(const __grid_constant__ Batch bt) {
+  constexpr int kTasks = 2;  // tasks per warp in flight
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
-  const uint32_t runs_per_warp = 32u / lanes_per_run;
-  const uint32_t sub = lane / lanes_per_run, sl = lane % lanes_per_run;
-  const uint32_t nvec = m.run_bytes / sizeof(V);
-  for (uint32_t q = warp * runs_per_warp + sub; q < m.n_runs; q += n_warps * runs_per_warp) {
-    uint64_t so, dof;
-    run_offsets(m, q, so, dof);
-    const V* s = reinterpret_cast<const V*>(src + so);
-    V* d = reinterpret_cast<V*>(dst + dof);
-    for (uint32_t v0 = sl; v0 < nvec; v0 += kUnroll * lanes_per_run) {
-      V buf[kUnroll];
+  for (uint32_t t0 = warp; t0 < bt.n_tasks; t0 += kTasks * n_warps) {
+    V buf[kTasks][kSlots];
+    V* dst[kTasks][kSlots];
 #pragma unroll
-      for (int k = 0; k < kUnroll; ++k) {
-        const uint32_t v = v0 + k * lanes_per_run;
-        if (v < nvec) buf[k] = __ldcs(s + v);
+    for (int y = 0; y < kTasks; ++y) {
+      const uint32_t task = t0 + y * n_warps;
+      const V* src[kSlots];
+      if (task < bt.n_tasks) {
+        task_lane<V>(bt, task, lane, src, dst[y]);
+      } else {
+#pragma unroll
+        for (int x = 0; x < kSlots; ++x) src[x] = nullptr;
       }
 #pragma unroll
-      for (int k = 0; k < kUnroll; ++k) {
-        const uint32_t v = v0 + k * lanes_per_run;
-        if (v < nvec) __stcs(d + v, buf[k]);
+      for (int x = 0; x < kSlots; ++x) {
+        if (src[x] != nullptr) buf[y][x] = __ldcs(src[x]);
+        if (src[x] == nullptr) dst[y][x] = nullptr;
       }
     }
+#pragma unroll
+    for (int y = 0; y < kTasks; ++y)
+#pragma unroll
+      for (int x = 0; x < kSlots; ++x)
+        if (dst[y][x] != nullptr) __stcs(dst[y][x], buf[y][x]);
   }
 }
 
@@ -100,45 +199,96 @@ uint32_t pow2_at_least(uint32_t x) {
   return p;
 }
 
+RunMap make_map(int map, uint32_t B, uint32_t S, uint32_t H, uint32_t P_u, uint32_t P_r, uint32_t row_bytes) {
+  RunMap m{};
+  m.map = map;
+  m.B = B; m.S = S; m.H = H; m.P_u = P_u; m.P_r = P_r;
+  m.P = P_u * P_r;
+  m.c = S / (2 * m.P);
+  m.c2 = 2 * m.c;
+  m.L = m.c2 * P_u;
+  m.Hl = H / P_u;
+  m.row_bytes = row_bytes;
+  if (map == kZigzagShard || map == kZigzagUnshard) {
+    m.run_bytes = H * row_bytes;
+    m.n_runs = B * S;
+  } else {
+    m.run_bytes = m.Hl * row_bytes;
+    m.n_runs = B * S * P_u;
+  }
+  return m;
+}
+
 }  // namespace
 
-cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t stream) {
-  RunMap m{};
-  m.map = a.map;
-  m.B = a.B; m.S = a.S; m.H = a.H; m.P_u = a.P_u; m.P_r = a.P_r;
-  m.P = a.P_u * a.P_r;
-  m.c = a.S / (2 * m.P);
-  m.c2 = 2 * m.c;
-  m.L = m.c2 * a.P_u;
-  m.Hl = a.H / a.P_u;
-  m.row_bytes = a.row_bytes;
-  if (a.map == kZigzagShard || a.map == kZigzagUnshard) {
-    m.run_bytes = a.H * a.row_bytes;
-    m.n_runs = a.B * a.S;
-  } else {
-    m.run_bytes = m.Hl * a.row_bytes;
-    m.n_runs = a.B * a.S * a.P_u;
+cudaError_t launch_layout_batch(const LayoutArgs* a, int n, cudaStream_t stream) {
+  if (n <= 0 || n > kMaxLayoutJobs) return cudaErrorInvalidValue;
+  Batch bt{};
+  bt.n_jobs = n;
+  // 16-byte vectors when every run of every job starts on a 16-byte boundary:
+  // every source and destination offset is a multiple of run_bytes (or of
+  // H*row_bytes = P_u*run_bytes), so 16-byte runs on 16-byte bases qualify.
+  bool vec16 = true;
+  for (int x = 0; x < n; ++x) {
+    bt.job[x].m = make_map(a[x].map, a[x].B, a[x].S, a[x].H, a[x].P_u, a[x].P_r, a[x].row_bytes);
+    vec16 = vec16 && bt.job[x].m.run_bytes % 16 == 0 && reinterpret_cast<uintptr_t>(a[x].src) % 16 == 0 &&
+            reinterpret_cast<uintptr_t>(a[x].dst) % 16 == 0;
   }
-  if (m.n_runs == 0) return cudaSuccess;
+  const uint32_t vsz = vec16 ? 16 : 4;
+  uint64_t tasks = 0;
+  for (int x = 0; x < n; ++x) {
+    Job& jb = bt.job[x];
+    jb.src = a[x].src;
+    jb.dst = a[x].dst;
+    jb.nvec = jb.m.run_bytes / vsz;
+    jb.task_begin = static_cast<uint32_t>(tasks);
+    const RunMap& m = jb.m;
+    // contiguous source segments of consecutive destination runs
+    switch (m.map) {
+      case kZigzagShard:
+      case kZigzagUnshard: jb.seg = m.c; jb.src_step = m.run_bytes; break;
+      case kSeq2Head: jb.seg = m.c2; jb.src_step = static_cast<uint64_t>(m.H) * m.row_bytes; break;
+      default: jb.seg = m.P_u; jb.src_step = static_cast<uint64_t>(m.B) * m.L * m.run_bytes; break;
+    }
+    if (jb.nvec >= 32 * kSlots) {
+      jb.lanes = 32;
+      jb.pieces = (jb.nvec + 32 * kSlots - 1) / (32 * kSlots);
+      jb.xslots = 0;
+      jb.runs_per_task = 1;
+      tasks += static_cast<uint64_t>(m.n_runs) * jb.pieces;
+    } else {
+      jb.pieces = 0;
+      if (jb.nvec >= 32) {
+        jb.lanes = 32;
+        jb.xslots = (jb.nvec + 31) / 32;
+        jb.runs_per_task = kSlots / jb.xslots;
+      } else {
+        jb.lanes = pow2_at_least(jb.nvec);
+        jb.xslots = 1;
+        jb.runs_per_task = kSlots * (32 / jb.lanes);
+      }
+      tasks += (static_cast<uint64_t>(m.n_runs) + jb.runs_per_task - 1) / jb.runs_per_task;
+    }
+  }
+  if (tasks == 0) return cudaSuccess;
+  if (tasks >= (1ull << 32) - (1ull << 28)) return cudaErrorInvalidValue;
+  bt.n_tasks = static_cast<uint32_t>(tasks);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // Every source and destination offset is a multiple of run_bytes (or of
-  // H*row_bytes = P_u*run_bytes), so 16-byte runs keep 16-byte alignment.
-  const bool vec16 = (m.run_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(a.src) % 16 == 0) &&
-                     (reinterpret_cast<uintptr_t>(a.dst) % 16 == 0);
-  const uint32_t nvec = m.run_bytes / (vec16 ? 16 : 4);
-  const uint32_t lpr = nvec >= 32 ? 32 : pow2_at_least(nvec);
-  const uint64_t threads_needed = static_cast<uint64_t>(m.n_runs) * lpr;
-  uint64_t blocks = (threads_needed + 255) / 256;
+  // 8 CTAs of 8 warps per SM (the SM's full 2048 threads), fewer when there are
+  // fewer tasks: each warp then takes an equal share of the tasks.
+  uint64_t blocks = (tasks + 7) / 8;
   const uint64_t cap = static_cast<uint64_t>(sms) * 8;
   if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
   if (vec16)
-    layout_gather_kernel<uint4, 4><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(a.src, a.dst, m, lpr);
+    layout_gather_kernel<uint4><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(bt);
   else
-    layout_gather_kernel<uint32_t, 4><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(a.src, a.dst, m, lpr);
+    layout_gather_kernel<uint32_t><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(bt);
+  note_launch();
   return cudaGetLastError();
 }
+
+cudaError_t launch_layout(const LayoutArgs& a, cudaStream_t stream) { return launch_layout_batch(&a, 1, stream); }
 
 }  // namespace usp

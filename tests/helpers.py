@@ -54,7 +54,7 @@ def gpu_fwd(spec, tensors, mode=B_.USP_MODE_FUSED):
     q = head_shard_cpu(tensors["q"], spec).to(dev)
     k = head_shard_cpu(tensors["k"], spec).to(dev)
     v = head_shard_cpu(tensors["v"], spec).to(dev)
-    out, lse = api.attn_fwd(q, k, v, spec["causal"], spec["P_u"], spec["P_r"], mode=mode)
+    out, lse = api.attn_fwd(q, k, v, spec["causal"], spec["P_u"], spec["P_r"], mode=mode, check_status=True)
     torch.cuda.synchronize()
     return unshard_cpu(out, spec), lse_to_global(lse, spec)
 
@@ -68,8 +68,16 @@ def sample_rows(spec, n, seed):
     return rows
 
 
-def compare_fwd(o_gpu, lse_gpu, tensors, spec, rows=None):
-    """Compare global-layout GPU O/LSE with the oracle at `rows` (all rows if None)."""
+def compare_fwd(o_gpu, lse_gpu, tensors, spec, rows=None, name=None):
+    """Compare global-layout GPU O/LSE with the oracle at `rows` (all rows if None).
+
+    The max-abs bound on O is applied raw to every element whose reference value
+    has |O_ref| < 4. O is delivered in bf16, and for |O_ref| >= 4 the spacing of
+    bf16 is 2^-5, so rounding the exact value alone may move it by half of that,
+    2^-6 = 0.0156 > 1e-2: only there is the error beyond that half-ulp held to the
+    bound. (For |O_ref| in [2, 4) the half-ulp is 2^-7 = 0.0078, which still fits
+    inside 1e-2, so those elements get no allowance.)
+    """
     B, S, H = spec["B"], spec["S"], spec["Hq"]
     if rows is None:
         rows = [(b, h, i) for b in range(B) for h in range(H) for i in range(S)]
@@ -77,14 +85,30 @@ def compare_fwd(o_gpu, lse_gpu, tensors, spec, rows=None):
     idx = np.array(rows)
     o_g = o_gpu.float().numpy()[idx[:, 0], idx[:, 2], idx[:, 1]].astype(np.float64)
     l_g = lse_gpu.float().numpy()[idx[:, 0], idx[:, 2], idx[:, 1]].astype(np.float64)
-    err = np.abs(o_g - o_ref)
-    lerr = np.abs(l_g - lse_ref)
-    # O is delivered in bf16: its final rounding alone may move a value by half a
-    # bf16 ulp of the reference (2^-9 relative), which exceeds 1e-2 once |O| > 2.6.
-    # The max-abs bound applies to the error beyond that rounding.
-    excess = np.maximum(err - half_ulp_bf16(o_ref), 0.0)
-    return dict(o_max=float(err.max()), o_max_excess=float(excess.max()), o_mean=float(err.mean()),
-                lse_max=float(lerr.max()))
+    return fwd_stats(o_g, l_g, o_ref, lse_ref, name=name)
+
+
+def fwd_stats(o_g, l_g, o_ref, lse_ref, name=None, bf16_out=True):
+    """Error statistics of a forward result against the oracle (see compare_fwd).
+    With bf16_out=False (an fp32 O) no rounding allowance applies anywhere."""
+    err = np.abs(np.asarray(o_g, np.float64) - o_ref)
+    lerr = np.abs(np.asarray(l_g, np.float64) - lse_ref)
+    big = np.abs(o_ref) >= 4.0
+    allow = np.where(big, half_ulp_bf16(o_ref), 0.0) if bf16_out else np.zeros_like(o_ref)
+    excess = np.maximum(err - allow, 0.0)
+    st = dict(o_max=float(err.max()), o_max_below4=float(err[~big].max()) if (~big).any() else 0.0,
+              o_max_excess=float(excess.max()), n_big=int(big.sum()), o_mean=float(err.mean()),
+              lse_max=float(lerr.max()))
+    if name is not None:
+        FWD_STATS.append((name, st))
+    return st
+
+
+# (case name, stats) of every forward comparison made in this process; printed by
+# the terminal summary hook in conftest.py.
+FWD_STATS: list = []
+# (case name, {gradient: relative L2 error}) of every backward comparison.
+GRAD_STATS: list = []
 
 
 def half_ulp_bf16(x):
@@ -94,6 +118,7 @@ def half_ulp_bf16(x):
 
 
 def assert_fwd_ok(stats):
+    assert stats["o_max_below4"] <= O_MAX_ABS, stats
     assert stats["o_max_excess"] <= O_MAX_ABS, stats
     assert stats["o_mean"] <= O_MEAN_ABS, stats
     assert stats["lse_max"] <= LSE_MAX_ABS, stats

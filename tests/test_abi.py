@@ -128,3 +128,41 @@ def test_product_package_does_not_import_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "usp_oracle" not in text and "liboracle" not in text, f
+
+
+def test_permute_batch_rejects_bad_arguments():
+    L = B_.lib()
+    arr = (B_.PermuteJob * 2)(B_.PermuteJob(FAKE, FAKE + 4096, 4, 64, 0), B_.PermuteJob(FAKE, FAKE, 3, 64, 0))
+    assert L.usp_permute_batch(2, arr, 2, 1, 256, 2, 2, None) == B_.USP_ERR_UNSUPPORTED  # job 1: H % P_u
+    assert "job 1" in B_.usp_last_error()
+    assert L.usp_permute_batch(2, arr, 0, 1, 256, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_permute_batch(2, arr, 5, 1, 256, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_permute_batch(9, arr, 1, 1, 256, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_permute_batch(2, None, 1, 1, 256, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+    arr[0].dtype = 7
+    assert L.usp_permute_batch(2, arr, 1, 1, 256, 2, 2, None) == B_.USP_ERR_INVALID_ARG
+
+
+def test_dilated_rejects_bad_arguments():
+    L = B_.lib()
+    import ctypes
+    w = (ctypes.c_int * 2)(256, 512)
+    r = (ctypes.c_int * 2)(1, 2)
+
+    def call(S=1024, D=128, n=2, ws_bytes=1 << 30, causal=1, Hq=4, Hkv=2, ww=w, rr=r, ws=FAKE):
+        return L.usp_dilated_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, S, Hq, Hkv, D, causal, n, ww, rr, ws,
+                                      ws_bytes, None)
+    assert call(S=1000) == B_.USP_ERR_UNSUPPORTED            # S % w != 0
+    assert call(D=96) == B_.USP_ERR_UNSUPPORTED
+    assert call(Hq=3) == B_.USP_ERR_UNSUPPORTED
+    assert call(n=0) == B_.USP_ERR_INVALID_ARG
+    assert call(n=17) == B_.USP_ERR_INVALID_ARG
+    assert call(causal=3) == B_.USP_ERR_INVALID_ARG
+    assert call(ws_bytes=100) == B_.USP_ERR_WORKSPACE
+    assert call(ws=None) == B_.USP_ERR_WORKSPACE
+    bad_r = (ctypes.c_int * 2)(1, 600)
+    assert call(rr=bad_r) == B_.USP_ERR_UNSUPPORTED          # r > w
+    zero_w = (ctypes.c_int * 2)(0, 512)
+    assert call(ww=zero_w) == B_.USP_ERR_INVALID_ARG
+    assert B_.usp_dilated_workspace_size(1, 1024, 4, 128) == 256 + 1024 * 4 * (4 * 128 + 4)
+    assert B_.usp_dilated_workspace_size(1, 1024, 4, 96) == 0

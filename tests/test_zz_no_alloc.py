@@ -37,6 +37,8 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls(cuda):
         dv = torch.full(v.shape, float("nan"), dtype=torch.float32, device=cuda)
         B_.usp_attn_bwd_noalloc(q, k, v, out, lse, do, dq, dk, dv, B, S, Hq, Hkv, D, 1, P_u, P_r)
         torch.cuda.synchronize()
+        # no bounded device wait gave up during the call (the reader clears the word)
+        assert B_.usp_attn_bwd_noalloc_status() == (B_.USP_OK, 0)
         for got, want, name in ((dq, ref[0], "dq"), (dk, ref[1], "dk"), (dv, ref[2], "dv")):
             g = got.double().cpu().numpy()
             w = want.double().cpu().numpy()
