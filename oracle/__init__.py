@@ -17,6 +17,10 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
       example (tests/golden/dilated_tiny_closed_form.json), one pair (w = S,
       r = 1) against torch's fp64 scaled_dot_product_attention, and torch's fp64
       SDPA with the log of the key multiplicities as an additive mask.
+  masked_fwd_rows / masked_attn_full (block-sparse and document masks) --
+      pinned: a hand-derived worked example (tests/golden/masked_tiny_closed_form.json),
+      the all-ones mask against the unmasked pinned oracle, torch fp64 SDPA with
+      the boolean mask (forward) and its autograd (backward).
 """
 from __future__ import annotations
 
@@ -47,6 +51,10 @@ def lib():
         L.oracle_attn_dkdv_cols.argtypes = [P, P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, P, P, P, P, i_]
         L.oracle_lse_merge.argtypes = [l_, l_, l_, P, P, P, P, i_]
         L.oracle_dilated_fwd_rows.argtypes = [P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, l_, P, P, P, i_]
+        L.oracle_masked_fwd_rows.argtypes = [P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, P, l_, P, l_, l_, P, P, P,
+                                             i_]
+        L.oracle_masked_attn_full.argtypes = [P, P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, P, l_, P, l_, P, P, P,
+                                              P, P, i_]
         for name in ("oracle_zigzag_shard", "oracle_zigzag_unshard"):
             getattr(L, name).argtypes = [P, P, l_, l_, l_, l_, l_, l_]
         for name in ("oracle_seq2head", "oracle_head2seq"):
@@ -54,7 +62,7 @@ def lib():
         for name in ("oracle_attn_fwd_rows", "oracle_attn_full", "oracle_attn_dq_rows",
                      "oracle_attn_dkdv_cols", "oracle_lse_merge", "oracle_zigzag_shard",
                      "oracle_zigzag_unshard", "oracle_seq2head", "oracle_head2seq",
-                     "oracle_dilated_fwd_rows"):
+                     "oracle_dilated_fwd_rows", "oracle_masked_fwd_rows", "oracle_masked_attn_full"):
             getattr(L, name).restype = ctypes.c_int
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
@@ -125,6 +133,48 @@ def dilated_fwd_rows(q, k, v, causal, pairs, rows, scale=None, threads=0):
     if rc != 0:
         raise ValueError(f"oracle_dilated_fwd_rows failed ({rc})")
     return o, lse
+
+
+def _mask_args(block_mask, block, cu_seqlens):
+    bm = None if block_mask is None else np.ascontiguousarray(np.asarray(block_mask, dtype=np.uint8))
+    cu = None if cu_seqlens is None else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    return (bm, None if bm is None else _ptr(bm), int(block), cu, None if cu is None else _ptr(cu),
+            0 if cu is None else cu.shape[0] - 1)
+
+
+def masked_fwd_rows(q, k, v, causal, rows, block_mask=None, block=128, cu_seqlens=None, scale=None, threads=0):
+    """Masked attention O [n, D], LSE [n] of query rows (b, h, i): block_mask
+    [B, Hq, nb, nb] (0/1 per block of `block` positions) and/or document
+    boundaries cu_seqlens [n_docs + 1] (shared by the batch)."""
+    B, S, Hq, Hkv, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    (qa, ka, va), f64 = _inputs(q, k, v)
+    bm, bmp, bs, cu, cup, nd = _mask_args(block_mask, block, cu_seqlens)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    o = np.zeros((n, D), np.float64)
+    lse = np.zeros(n, np.float64)
+    rc = lib().oracle_masked_fwd_rows(_ptr(qa), _ptr(ka), _ptr(va), f64, B, S, Hq, Hkv, D, int(causal), scale,
+                                      bmp, bs, cup, nd, n, _ptr(rows), _ptr(o), _ptr(lse), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_masked_fwd_rows failed ({rc})")
+    return o, lse
+
+
+def masked_attn_full(q, k, v, do, causal, block_mask=None, block=128, cu_seqlens=None, scale=None, threads=0):
+    """Whole-tensor masked forward and backward: dict of float64 o, lse, dq, dk, dv."""
+    B, S, Hq, Hkv, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    (qa, ka, va, da), f64 = _inputs(q, k, v, do)
+    bm, bmp, bs, cu, cup, nd = _mask_args(block_mask, block, cu_seqlens)
+    o = np.zeros((B, S, Hq, D)); lse = np.zeros((B, S, Hq)); dq = np.zeros((B, S, Hq, D))
+    dk = np.zeros((B, S, Hkv, D)); dv = np.zeros((B, S, Hkv, D))
+    rc = lib().oracle_masked_attn_full(_ptr(qa), _ptr(ka), _ptr(va), _ptr(da), f64, B, S, Hq, Hkv, D,
+                                       int(causal), scale, bmp, bs, cup, nd, _ptr(o), _ptr(lse), _ptr(dq),
+                                       _ptr(dk), _ptr(dv), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_masked_attn_full failed ({rc})")
+    return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv)
 
 
 def attn_full(q, k, v, do, causal, scale=None, threads=0):

@@ -527,3 +527,165 @@ int oracle_dilated_fwd_rows(const void *q, const void *k, const void *v, int f64
     }
     return 0;
 }
+
+/*
+ * Attention with a visibility mask: block-sparse and packed variable-length
+ * (document) attention.
+ *
+ * Source: DeepSpeed-Ulysses summary (page 3), "Hauptmerkmale von
+ * DeepSpeed-Ulysses", item 3: the Ulysses layout serves dense and sparse
+ * attention alike (after the all-to-all every rank holds whole sequences for
+ * its heads, so any attention pattern applies unchanged). The pages give no
+ * pattern; the readings are the plain ones:
+ *   - block-sparse: a 0/1 mask over (query block, key block) of bs x bs
+ *     positions, per batch and query head: bm[b][h][i / bs][j / bs];
+ *   - packed variable-length sequences: documents [cu[d], cu[d+1]) of the
+ *     sequence (cu[0] = 0, cu[n_docs] = S, shared by the batch); a query sees
+ *     only keys of its own document.
+ * Key j is visible to query i iff (not causal or j <= i) and the block bit is
+ * set (when bm != NULL) and doc(i) == doc(j) (when cu != NULL). Otherwise the
+ * definition is that of oracle_attn_fwd_rows / oracle_attn_full over the
+ * visible set V(i); a row with an empty V(i) has O = 0, LSE = -inf and
+ * contributes no gradient.
+ */
+static long doc_of(const long *cu, long n_docs, long x) {
+    long d = 0;
+    while (d + 1 < n_docs && cu[d + 1] <= x) d++;
+    return d;
+}
+
+static int masked_visible(long b, long h, long i, long j, long Hq, int causal, const uint8_t *bm,
+                          long bs, long nb, const long *cu, long n_docs) {
+    if (causal && j > i) return 0;
+    if (bm && !bm[((b * Hq + h) * nb + i / bs) * nb + j / bs]) return 0;
+    if (cu && doc_of(cu, n_docs, i) != doc_of(cu, n_docs, j)) return 0;
+    return 1;
+}
+
+/* Forward of one query row over its visible set; s_buf holds S doubles and
+ * vis S flags. Returns LSE (-inf for an empty visible set). */
+static double masked_fwd_row(const void *q, const void *k, const void *v, int f64, long S, long Hq,
+                             long Hkv, long D, double scale, long b, long h, long i,
+                             const char *vis, double *s_buf, double *o) {
+    long g = h / (Hq / Hkv);
+    long qi = idx4(b, i, h, 0, S, Hq, D);
+    double m = -INFINITY;
+    for (long j = 0; j < S; j++) {
+        if (!vis[j]) continue;
+        long kj = idx4(b, j, g, 0, S, Hkv, D);
+        double acc = 0.0;
+        for (long d = 0; d < D; d++) acc += ld(q, qi + d, f64) * ld(k, kj + d, f64);
+        s_buf[j] = scale * acc;
+        if (s_buf[j] > m) m = s_buf[j];
+    }
+    for (long d = 0; d < D; d++) o[d] = 0.0;
+    if (m == -INFINITY) return -INFINITY;
+    double l = 0.0;
+    for (long j = 0; j < S; j++)
+        if (vis[j]) l += exp(s_buf[j] - m);
+    double L = m + log(l);
+    for (long j = 0; j < S; j++) {
+        if (!vis[j]) continue;
+        double w = exp(s_buf[j] - L);
+        long vj = idx4(b, j, g, 0, S, Hkv, D);
+        for (long d = 0; d < D; d++) o[d] += w * ld(v, vj + d, f64);
+    }
+    return L;
+}
+
+static int masked_args_ok(long S, const uint8_t *bm, long bs, const long *cu, long n_docs) {
+    if (bm && bs <= 0) return 0;
+    if (cu) {
+        if (n_docs < 1 || cu[0] != 0 || cu[n_docs] != S) return 0;
+        for (long d = 0; d < n_docs; d++)
+            if (cu[d + 1] < cu[d]) return 0;
+    }
+    return 1;
+}
+
+/* Forward rows (b, h, i) of the masked attention: o [n_rows][D], lse [n_rows].
+ * bm = [B][Hq][nb][nb] bytes with nb = ceil(S / bs), or NULL; cu = [n_docs + 1]
+ * or NULL. */
+int oracle_masked_fwd_rows(const void *q, const void *k, const void *v, int f64, long B, long S,
+                           long Hq, long Hkv, long D, int causal, double scale, const uint8_t *bm,
+                           long bs, const long *cu, long n_docs, long n_rows, const long *rows,
+                           double *o, double *lse, int n_threads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || !rows_ok(n_rows, rows, B, Hq, S) ||
+        !masked_args_ok(S, bm, bs, cu, n_docs))
+        return -1;
+    long nb = bm ? (S + bs - 1) / bs : 0;
+    set_threads(n_threads);
+#pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)S);
+        char *vis = (char *)malloc((size_t)S);
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < n_rows; r++) {
+            long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+            for (long j = 0; j < S; j++)
+                vis[j] = (char)masked_visible(b, h, i, j, Hq, causal, bm, bs, nb, cu, n_docs);
+            lse[r] = masked_fwd_row(q, k, v, f64, S, Hq, Hkv, D, scale, b, h, i, vis, s_buf, o + r * D);
+        }
+        free(s_buf);
+        free(vis);
+    }
+    return 0;
+}
+
+/* Whole-tensor forward and backward of the masked attention (layouts as in
+ * oracle_attn_full). Backward over the visible set: Delta_i = dO_i . O_i,
+ * P_ij = exp(s_ij - LSE_i), dS_ij = P_ij (dO_i . V_j - Delta_i),
+ * dQ_i = scale sum_j dS_ij K_j, dK_j = scale sum dS_ij Q_i, dV_j = sum P_ij dO_i.
+ * Work is split over (b, kv-head) so each task owns its dK/dV rows. */
+int oracle_masked_attn_full(const void *q, const void *k, const void *v, const void *dO, int f64,
+                            long B, long S, long Hq, long Hkv, long D, int causal, double scale,
+                            const uint8_t *bm, long bs, const long *cu, long n_docs, double *o,
+                            double *lse, double *dq, double *dk, double *dv, int n_threads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || !masked_args_ok(S, bm, bs, cu, n_docs)) return -1;
+    long G = Hq / Hkv;
+    long nb = bm ? (S + bs - 1) / bs : 0;
+    set_threads(n_threads);
+    memset(dk, 0, sizeof(double) * (size_t)(B * S * Hkv * D));
+    memset(dv, 0, sizeof(double) * (size_t)(B * S * Hkv * D));
+#pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)S);
+        char *vis = (char *)malloc((size_t)S);
+#pragma omp for schedule(dynamic, 1)
+        for (long bg = 0; bg < B * Hkv; bg++) {
+            long b = bg / Hkv, g = bg % Hkv;
+            for (long hh = 0; hh < G; hh++) {
+                long h = g * G + hh;
+                for (long i = 0; i < S; i++) {
+                    for (long j = 0; j < S; j++)
+                        vis[j] = (char)masked_visible(b, h, i, j, Hq, causal, bm, bs, nb, cu, n_docs);
+                    long qi = idx4(b, i, h, 0, S, Hq, D);
+                    double *oi = o + qi;
+                    double L = masked_fwd_row(q, k, v, f64, S, Hq, Hkv, D, scale, b, h, i, vis, s_buf, oi);
+                    lse[(b * S + i) * Hq + h] = L;
+                    double *dqi = dq + qi;
+                    for (long d = 0; d < D; d++) dqi[d] = 0.0;
+                    if (L == -INFINITY) continue;
+                    double delta = 0.0;
+                    for (long d = 0; d < D; d++) delta += ld(dO, qi + d, f64) * oi[d];
+                    for (long j = 0; j < S; j++) {
+                        if (!vis[j]) continue;
+                        double p = exp(s_buf[j] - L);
+                        long kj = idx4(b, j, g, 0, S, Hkv, D);
+                        double dp = 0.0;
+                        for (long d = 0; d < D; d++) dp += ld(dO, qi + d, f64) * ld(v, kj + d, f64);
+                        double ds = p * (dp - delta);
+                        for (long d = 0; d < D; d++) {
+                            dqi[d] += scale * ds * ld(k, kj + d, f64);
+                            dk[kj + d] += scale * ds * ld(q, qi + d, f64);
+                            dv[kj + d] += p * ld(dO, qi + d, f64);
+                        }
+                    }
+                }
+            }
+        }
+        free(s_buf);
+        free(vis);
+    }
+    return 0;
+}

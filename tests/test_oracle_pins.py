@@ -403,3 +403,80 @@ def test_dilated_matches_sdpa_with_multiplicity_mask(causal, pairs):
     with np.errstate(divide="ignore"):
         lref = np.log((C * np.exp(s)).sum(-1))[idx[:, 1], idx[:, 2]]
     np.testing.assert_allclose(lse[seen], lref[seen], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- block-sparse / document masks
+def test_masked_golden_tiny_closed_form():
+    g = json.load(open(os.path.join(GOLD, "masked_tiny_closed_form.json")))
+    S = g["S"]
+    q = torch.zeros(1, S, 1, 2, dtype=torch.bfloat16)
+    v = torch.tensor([[j, 1.0] for j in range(S)], dtype=torch.float64).view(1, S, 1, 2).to(torch.bfloat16)
+    k = _rand(6, (1, S, 1, 2))
+    for c in g["cases"]:
+        bm = None if c["mask"] is None else np.array(g["masks"][c["mask"]], np.uint8).reshape(1, 1, 3, 3)
+        o, lse = oracle.masked_fwd_rows(q, k, v, c["causal"], [(0, 0, c["row"])], block_mask=bm, block=g["block"],
+                                        cu_seqlens=g["cu_seqlens"])
+        np.testing.assert_allclose(o[0], c["o"], rtol=0, atol=1e-13)
+        if c["lse"] == "-inf":
+            assert lse[0] == -math.inf
+        else:
+            assert abs(lse[0] - c["lse"]) < 1e-13
+
+
+def _bool_mask(B, S, H, causal, bm, bs, cu):
+    """[B, H, S, S] visibility from the reading: causal, block bit, same document."""
+    vis = np.ones((B, H, S, S), bool)
+    if causal:
+        vis &= np.tril(np.ones((S, S), bool))
+    if bm is not None:
+        vis &= np.repeat(np.repeat(bm.astype(bool), bs, axis=2), bs, axis=3)[:, :, :S, :S]
+    if cu is not None:
+        doc = np.searchsorted(np.asarray(cu), np.arange(S), side="right") - 1
+        vis &= doc[:, None] == doc[None, :]
+    return vis
+
+
+def _sdpa_masked(q, k, v, vis):
+    G = q.shape[2] // k.shape[2]
+    qt = q.double().transpose(1, 2)
+    kt = k.double().repeat_interleave(G, dim=2).transpose(1, 2)
+    vt = v.double().repeat_interleave(G, dim=2).transpose(1, 2)
+    return F.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.tensor(vis)).transpose(1, 2)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_masked_all_ones_is_unmasked(causal):
+    B, S, Hq, Hkv, D, bs = 1, 40, 4, 2, 8, 8
+    q, k, v, do = (_rand(90 + n, (B, S, h, D)) for n, h in enumerate((Hq, Hkv, Hkv, Hq)))
+    bm = np.ones((B, Hq, 5, 5), np.uint8)
+    m = oracle.masked_attn_full(q, k, v, do, causal, block_mask=bm, block=bs, cu_seqlens=[0, S])
+    u = oracle.attn_full(q, k, v, do, causal)
+    for n in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_allclose(m[n], u[n], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("kind", ["block", "docs", "both"])
+def test_masked_matches_sdpa_forward_and_autograd(causal, kind):
+    """Forward against torch fp64 SDPA with the boolean mask, gradients against
+    its autograd; rows whose visible set is empty are checked to be O = 0,
+    LSE = -inf and are left out of the SDPA comparison (SDPA gives NaN there)."""
+    B, S, Hq, Hkv, D, bs = 2, 36, 4, 2, 8, 6
+    q, k, v, do = (_rand(95 + n, (B, S, h, D)).double() for n, h in enumerate((Hq, Hkv, Hkv, Hq)))
+    rng = np.random.default_rng(3)
+    bm = (rng.random((B, Hq, 6, 6)) < 0.6).astype(np.uint8) if kind in ("block", "both") else None
+    cu = [0, 5, 13, 14, 30, 36] if kind in ("docs", "both") else None
+    vis = _bool_mask(B, S, Hq, causal, bm, bs, cu)
+    m = oracle.masked_attn_full(q, k, v, do, causal, block_mask=bm, block=bs, cu_seqlens=cu)
+    empty = ~vis.any(-1)  # [B, H, S]
+    e_bsh = empty.transpose(0, 2, 1)
+    assert np.all(np.isneginf(m["lse"][e_bsh])) and np.all(m["o"][e_bsh] == 0)
+    qr, kr, vr = (t.clone().requires_grad_(True) for t in (q, k, v))
+    vis_safe = vis | empty[..., None]  # SDPA needs one visible key per row; those rows are dropped below
+    o = _sdpa_masked(qr, kr, vr, vis_safe)
+    keep = torch.tensor(~e_bsh)[..., None].double()
+    (o * do * keep).sum().backward()
+    on = o.detach().numpy()
+    np.testing.assert_allclose(m["o"][~e_bsh], on[~e_bsh], rtol=0, atol=1e-12)
+    for n, t in (("dq", qr), ("dk", kr), ("dv", vr)):
+        np.testing.assert_allclose(m[n], t.grad.numpy(), rtol=0, atol=1e-11)
