@@ -203,6 +203,93 @@ int usp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
                     int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Sparse and variable-length attention under the Ulysses layout
+ * (DeepSpeed-Ulysses summary, "Hauptmerkmale von DeepSpeed-Ulysses", item 3:
+ * dense and sparse attention alike -- after the all-to-all each rank holds
+ * whole sequences for its heads, so an attention pattern applies unchanged).
+ * usp_attn_fwd_masked / usp_attn_bwd_masked are usp_attn_fwd (fused mode) and
+ * usp_attn_bwd with a visibility mask on top of causality, both in ORIGINAL
+ * token positions (the zigzag and the all-to-all are undone by the kernels):
+ *   block_mask  DEVICE bytes [B][Hq][S/128][S/128] (global query head index):
+ *               key block kb is visible to query block qb iff
+ *               block_mask[b][h][qb][kb] != 0; blocks are 128 positions, the
+ *               kernels' tile, so masked-off blocks are skipped whole; or NULL.
+ *   cu_seqlens  DEVICE int32 [n_docs + 1]: packed variable-length sequences
+ *               (documents [cu[d], cu[d+1]), non-decreasing, cu[0] = 0,
+ *               cu[n_docs] = S, shared by the batch); a query sees only keys of
+ *               its own document; or NULL. Other values give undefined results
+ *               but never an access outside cu[0 .. n_docs].
+ * A query row with no visible key gets O = 0 and LSE = -inf and contributes no
+ * gradient. Masks need zigzag chunks that are whole tiles: S / (2 P_u P_r) a
+ * multiple of 128 (else USP_ERR_UNSUPPORTED). Workspaces are those of
+ * usp_attn_fwd (fused) and usp_attn_bwd. A NULL mask, or one with both
+ * pointers NULL, is the unmasked call.
+ */
+typedef struct {
+  const unsigned char* block_mask;
+  const int* cu_seqlens;
+  int n_docs;
+} usp_attn_mask;
+int usp_attn_fwd_masked(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
+                        int Hkv, int D, int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace,
+                        size_t ws_bytes, void* stream);
+int usp_attn_bwd_masked(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                        const void* dO, void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D,
+                        int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * The per-rank compute of a REAL multi-GPU USP mesh: one process per GPU holds
+ * one rank r = i * P_u + u and calls these between its own NCCL collectives
+ * ("Boosting Spec Eagle", "The Solution": ring devices hold slices of the
+ * sequence and pass key/value blocks to their neighbours; DeepSpeed-Ulysses
+ * summary, "Wie DeepSpeed-Ulysses funktioniert": all-to-all before and after
+ * attention). Shapes (B, S, Hq, Hkv, D, causal, P_u, P_r) are the GLOBAL ones
+ * of the mesh, as for usp_attn_fwd; the buffers are the rank's own:
+ *   rank-local tokens  [B][T][H][D], T = S / (P_u P_r) (zigzag chunks r, 2P-1-r)
+ *   head-sharded       [B][L][H/P_u][D], L = S / P_r (the slice [i][u] of the
+ *                      one-GPU head-sharded layout)
+ *
+ * usp_ulysses_pack: the local halves of the Ulysses all-to-all among the G =
+ * P_u ranks of a group (jobs as for usp_permute_batch, H = the tensor's total
+ * heads, a multiple of G; T tokens per rank):
+ *   USP_MAP_PACK_HEADS    [B][T][H][D] -> [G][B][T][H/G][D]  send buffer, seq->head
+ *   USP_MAP_UNPACK_TOKENS [G][B][T][H/G][D] -> [B][G*T][H/G][D] received, seq->head
+ *   USP_MAP_PACK_TOKENS   [B][G*T][H/G][D] -> [G][B][T][H/G][D] send buffer, head->seq
+ *   USP_MAP_UNPACK_HEADS  [G][B][T][H/G][D] -> [B][T][H][D]  received, head->seq
+ * with an equal-split all-to-all over the group between pack and unpack.
+ *
+ * usp_ring_fwd_step: ring step t of rank (i, u): its head-sharded q against the
+ * KV block of ring rank j = (i - t) mod P_r (same u) that it holds now; writes
+ * the step's fp32 partial o_part [B][L][Hq/P_u][D] and lse_part [B][L][Hq/P_u]
+ * (rows that see no key of the block: LSE = -inf, O = 0). Fold the partials
+ * with usp_lse_merge (in place into a running fp32 result). Workspace 256 B.
+ *
+ * usp_ring_bwd_prepare: the per-head -LSE*log2(e) and -Delta tables of the
+ * rank's rows from its final out, lse and dO (workspace of
+ * usp_ring_workspace_size(..., bwd = 1)).
+ * usp_ring_bwd_step: ring step t: ADDS this rank's contribution to the
+ * gradients of the block it holds, dk_acc / dv_acc (fp32, the gradients
+ * travelling with the block), and to its own dq_acc (fp32); when dq_out (bf16,
+ * may be NULL) is given, the final dQ = dq_acc + this step is written there
+ * instead of into dq_acc (call it so on the last step).
+ */
+#define USP_MAP_PACK_HEADS 4
+#define USP_MAP_UNPACK_TOKENS 5
+#define USP_MAP_PACK_TOKENS 6
+#define USP_MAP_UNPACK_HEADS 7
+int usp_ulysses_pack(int map, const usp_permute_job* jobs, int n_jobs, int B, int T, int G, void* stream);
+size_t usp_ring_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, int bwd);
+int usp_ring_fwd_step(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int S,
+                      int Hq, int Hkv, int D, int causal, int P_u, int P_r, int i, int u, int t, void* workspace,
+                      size_t ws_bytes, void* stream);
+int usp_ring_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,
+                         int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream);
+int usp_ring_bwd_step(const void* q, const void* k, const void* v, const void* dO, float* dq_acc, void* dq_out,
+                      float* dk_acc, float* dv_acc, int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r,
+                      int i, int u, int t, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Bytes of the static device scratch behind usp_attn_bwd_noalloc (32 MiB).
  */
 #define USP_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

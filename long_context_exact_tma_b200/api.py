@@ -164,6 +164,49 @@ def attn_bwd(q, k, v, out, lse, dO, causal: bool, P_u: int, P_r: int, ws=None, d
     return dq, dk, dv
 
 
+def attn_fwd_masked(q, k, v, causal: bool, P_u: int, P_r: int, block_mask=None, cu_seqlens=None, ws=None, out=None,
+                    lse=None, stream=None, check_status: bool = False):
+    """usp_attn_fwd (fused) with a block mask [B, Hq, S/128, S/128] (uint8, CUDA)
+    and/or document boundaries cu_seqlens [n_docs + 1] (int32, CUDA), both in
+    original positions."""
+    _require_cuda(q, k, v)
+    Pr, Pu, B, L, Hql, D = q.shape
+    Hkv = k.shape[4] * P_u
+    Hq = Hql * P_u
+    S = L * P_r
+    n_docs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if ws is None:
+        ws = workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 0, 0), q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device) if lse is None else lse
+    B_.usp_attn_fwd_masked(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, P_u, P_r, block_mask, cu_seqlens, n_docs, ws,
+                           ws.numel(), stream)
+    if check_status:
+        check_workspace(ws, stream)
+    return out, lse
+
+
+def attn_bwd_masked(q, k, v, out, lse, dO, causal: bool, P_u: int, P_r: int, block_mask=None, cu_seqlens=None,
+                    ws=None, stream=None, check_status: bool = False):
+    """usp_attn_bwd with the masks of attn_fwd_masked; returns (dQ, dK, dV)."""
+    _require_cuda(q, k, v, out, lse, dO)
+    Pr, Pu, B, L, Hql, D = q.shape
+    Hkv = k.shape[4] * P_u
+    Hq = Hql * P_u
+    S = L * P_r
+    n_docs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if ws is None:
+        ws = workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 0, 1), q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=k.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=v.device)
+    B_.usp_attn_bwd_masked(q, k, v, out, lse, dO, dq, dk, dv, B, S, Hq, Hkv, D, causal, P_u, P_r, block_mask,
+                           cu_seqlens, n_docs, ws, ws.numel(), stream)
+    if check_status:
+        check_workspace(ws, stream)
+    return dq, dk, dv
+
+
 def dilated_attn_fwd(q, k, v, causal: bool, pairs, ws=None, out=None, lse=None, stream=None,
                      check_status: bool = False):
     """LongNet dilated attention over global-layout q [B, S, Hq, D], k/v [B, S, Hkv, D]

@@ -29,7 +29,16 @@ USP_MAP_ZIGZAG_UNSHARD = 1
 USP_MAP_SEQ2HEAD = 2
 USP_MAP_HEAD2SEQ = 3
 USP_MAX_PERMUTE_JOBS = 4
+USP_MAP_PACK_HEADS = 4
+USP_MAP_UNPACK_TOKENS = 5
+USP_MAP_PACK_TOKENS = 6
+USP_MAP_UNPACK_HEADS = 7
 USP_DILATED_MAX_PAIRS = 16
+
+
+class AttnMask(ctypes.Structure):
+    """usp_attn_mask of include/usp.h."""
+    _fields_ = [("block_mask", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p), ("n_docs", ctypes.c_int)]
 
 
 class PermuteJob(ctypes.Structure):
@@ -54,10 +63,17 @@ SIGNATURES = {
     "usp_head2seq_permute": (_I, _LAYOUT),
     "usp_permute_batch": (_I, [_I, ctypes.POINTER(PermuteJob), _I, _I, _I, _I, _I, _P]),
     "usp_attn_workspace_size": (_SZ, [_I] * 10),
+    "usp_ulysses_pack": (_I, [_I, ctypes.POINTER(PermuteJob), _I, _I, _I, _I, _P]),
+    "usp_ring_workspace_size": (_SZ, [_I] * 9),
+    "usp_ring_fwd_step": (_I, [_P] * 5 + [_I] * 11 + [_P, _SZ, _P]),
+    "usp_ring_bwd_prepare": (_I, [_P] * 3 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_ring_bwd_step": (_I, [_P] * 8 + [_I] * 11 + [_P, _SZ, _P]),
     "usp_dilated_workspace_size": (_SZ, [_I] * 4),
     "usp_dilated_attn_fwd": (_I, [_P] * 5 + [_I] * 7 + [_P, _P, _P, _SZ, _P]),
     "usp_attn_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_P, _SZ, _P]),
     "usp_attn_bwd": (_I, [_P] * 9 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_attn_fwd_masked": (_I, [_P] * 5 + [_I] * 8 + [ctypes.POINTER(AttnMask), _P, _SZ, _P]),
+    "usp_attn_bwd_masked": (_I, [_P] * 9 + [_I] * 8 + [ctypes.POINTER(AttnMask), _P, _SZ, _P]),
     "usp_attn_bwd_prepare": (_I, [_P, _P, _P] + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_dkdv": (_I, [_P] * 6 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_dq": (_I, [_P] * 5 + [_I] * 8 + [_P, _SZ, _P]),
@@ -158,6 +174,41 @@ def usp_permute_batch(map_, jobs, B, S, P_u, P_r, stream=None, check=True):
     return _check(rc) if check else rc
 
 
+def usp_ulysses_pack(map_, jobs, B, T, G, stream=None, check=True):
+    """jobs: sequence of (src, dst, H, D, dtype)."""
+    arr = (PermuteJob * max(len(jobs), 1))()
+    for x, (src, dst, H, D, dtype) in enumerate(jobs):
+        arr[x] = PermuteJob(_ptr(src), _ptr(dst), H, D, dtype)
+    rc = lib().usp_ulysses_pack(map_, arr, len(jobs), B, T, G, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, bwd) -> int:
+    return int(lib().usp_ring_workspace_size(B, S, Hq, Hkv, D, int(causal), P_u, P_r, int(bwd)))
+
+
+def usp_ring_fwd_step(q, k, v, o_part, lse_part, B, S, Hq, Hkv, D, causal, P_u, P_r, i, u, t, workspace, ws_bytes,
+                      stream=None, check=True):
+    rc = lib().usp_ring_fwd_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, S, Hq, Hkv, D,
+                                 int(causal), P_u, P_r, i, u, t, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_ring_bwd_prepare(out, lse, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream=None,
+                         check=True):
+    rc = lib().usp_ring_bwd_prepare(_ptr(out), _ptr(lse), _ptr(dO), B, S, Hq, Hkv, D, int(causal), P_u, P_r,
+                                    _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_ring_bwd_step(q, k, v, dO, dq_acc, dq_out, dk_acc, dv_acc, B, S, Hq, Hkv, D, causal, P_u, P_r, i, u, t,
+                      workspace, ws_bytes, stream=None, check=True):
+    rc = lib().usp_ring_bwd_step(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq_acc), _ptr(dq_out), _ptr(dk_acc),
+                                 _ptr(dv_acc), B, S, Hq, Hkv, D, int(causal), P_u, P_r, i, u, t, _ptr(workspace),
+                                 ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
 def usp_attn_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, mode, bwd) -> int:
     return int(lib().usp_attn_workspace_size(B, S, Hq, Hkv, D, int(causal), P_u, P_r, mode, int(bwd)))
 
@@ -189,6 +240,27 @@ def usp_attn_bwd(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_
     rc = lib().usp_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
                             _ptr(dV), B, S, Hq, Hkv, D, int(causal), P_u, P_r, _ptr(workspace), ws_bytes,
                             _stream(stream))
+    return _check(rc) if check else rc
+
+
+def _mask(block_mask, cu_seqlens, n_docs):
+    return AttnMask(_ptr(block_mask), _ptr(cu_seqlens), int(n_docs))
+
+
+def usp_attn_fwd_masked(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, P_u, P_r, block_mask, cu_seqlens, n_docs,
+                        workspace, ws_bytes, stream=None, check=True):
+    m = _mask(block_mask, cu_seqlens, n_docs)
+    rc = lib().usp_attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D, int(causal),
+                                   P_u, P_r, ctypes.byref(m), _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_attn_bwd_masked(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, block_mask,
+                        cu_seqlens, n_docs, workspace, ws_bytes, stream=None, check=True):
+    m = _mask(block_mask, cu_seqlens, n_docs)
+    rc = lib().usp_attn_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
+                                   _ptr(dV), B, S, Hq, Hkv, D, int(causal), P_u, P_r, ctypes.byref(m),
+                                   _ptr(workspace), ws_bytes, _stream(stream))
     return _check(rc) if check else rc
 
 

@@ -167,6 +167,16 @@ unsigned long long current_wait_ns() { return g_wait_ns; }
 }  // namespace usp
 
 namespace {
+int check_geom(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, AttnGeom* g);
+}  // namespace
+
+namespace usp {
+int validate_geom(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, AttnGeom* g) {
+  return check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, g);
+}
+}  // namespace usp
+
+namespace {
 
 size_t rows_of(const AttnGeom& g) { return static_cast<size_t>(g.B) * g.S * g.Hq; }
 
@@ -246,12 +256,34 @@ size_t usp_attn_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal,
   return fwd_ws(g, mode);
 }
 
-int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
-                 int Hkv, int D, int causal, int P_u, int P_r, int mode, void* workspace, size_t ws_bytes,
-                 void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The masks of usp_attn_*_masked as kernel arguments; validates them against
+// the geometry (masks need chunks that are whole tiles).
+int mask_args(const usp_attn_mask* m, const AttnGeom& g, MaskArgs* out) {
+  *out = MaskArgs{};
+  if (!m || (!m->block_mask && !m->cu_seqlens)) return USP_OK;
+  if (g.c % 128 != 0)
+    return fail(USP_ERR_UNSUPPORTED, "masks need zigzag chunks of a multiple of 128 tokens (S/(2 P) = %d)", g.c);
+  if (m->cu_seqlens && m->n_docs < 1) return fail(USP_ERR_INVALID_ARG, "n_docs must be >= 1 with cu_seqlens");
+  out->bm = m->block_mask;
+  out->cu = m->cu_seqlens;
+  out->n_docs = m->cu_seqlens ? m->n_docs : 0;
+  out->nb = g.S / 128;
+  out->Hq = g.Hq;
+  return USP_OK;
+}
+
+int attn_fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq, int Hkv,
+                  int D, int causal, int P_u, int P_r, int mode, const usp_attn_mask* mask, void* workspace,
+                  size_t ws_bytes, void* stream) {
   AttnGeom g{};
   int rc = check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
   if (rc != USP_OK) return rc;
+  MaskArgs mk{};
+  if ((rc = mask_args(mask, g, &mk)) != USP_OK) return rc;
   if (mode != USP_MODE_FUSED && mode != USP_MODE_STEPWISE) return fail(USP_ERR_INVALID_ARG, "bad mode %d", mode);
   if (!q || !k || !v || !out || !lse) return fail(USP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
@@ -267,6 +299,7 @@ int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
   if ((rc = make_tmap(&L.tm_v, v, D, g.Hkv_l, g.L, g.n_ranks * B)) != USP_OK) return rc;
   L.status = static_cast<int*>(workspace);
   L.wait_ns = g_wait_ns;
+  L.mask = mk;
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
   if (e != cudaSuccess) return cuda_fail(e, "status reset");
   if (mode == USP_MODE_FUSED) {
@@ -299,6 +332,24 @@ int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
   return USP_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int usp_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
+                 int Hkv, int D, int causal, int P_u, int P_r, int mode, void* workspace, size_t ws_bytes,
+                 void* stream) {
+  return attn_fwd_impl(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, P_u, P_r, mode, nullptr, workspace, ws_bytes,
+                       stream);
+}
+
+int usp_attn_fwd_masked(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
+                        int Hkv, int D, int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  return attn_fwd_impl(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, P_u, P_r, USP_MODE_FUSED, mask, workspace,
+                       ws_bytes, stream);
+}
+
 int usp_attn_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,
                          int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream) {
   AttnGeom g{};
@@ -321,14 +372,18 @@ int usp_attn_bwd_prepare(const void* out, const float* lse, const void* dO, int 
   return e == cudaSuccess ? USP_OK : cuda_fail(e, "preprocess launch");
 }
 
+}  // extern "C"
+
 namespace {
 // Validation and TMA maps shared by the two backward kernels (workspace prepared
 // by usp_attn_bwd_prepare).
 int bwd_launch_setup(const void* q, const void* k, const void* v, const void* dO, int B, int S, int Hq, int Hkv,
-                     int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, BwdLaunch* L) {
+                     int D, int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace,
+                     size_t ws_bytes, BwdLaunch* L) {
   AttnGeom g{};
   int rc = check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
   if (rc != USP_OK) return rc;
+  if ((rc = mask_args(mask, g, &L->mask)) != USP_OK) return rc;
   if (!q || !k || !v || !dO) return fail(USP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO))
     return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
@@ -349,15 +404,14 @@ int bwd_launch_setup(const void* q, const void* k, const void* v, const void* dO
   L->wait_ns = g_wait_ns;
   return USP_OK;
 }
-}  // namespace
 
-int usp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, float* dK, float* dV, int B,
-                      int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes,
-                      void* stream) {
+int bwd_dkdv_impl(const void* q, const void* k, const void* v, const void* dO, float* dK, float* dV, int B, int S,
+                  int Hq, int Hkv, int D, int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace,
+                  size_t ws_bytes, void* stream) {
   if (!dK || !dV) return fail(USP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(dK) || !aligned16(dV)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   BwdLaunch L{};
-  const int rc = bwd_launch_setup(q, k, v, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, &L);
+  const int rc = bwd_launch_setup(q, k, v, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes, &L);
   if (rc != USP_OK) return rc;
   L.dk = dK;
   L.dv = dV;
@@ -365,24 +419,27 @@ int usp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* d
   return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention backward (dK, dV) launch");
 }
 
-int usp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dQ, int B, int S, int Hq,
-                    int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream) {
+int bwd_dq_impl(const void* q, const void* k, const void* v, const void* dO, void* dQ, int B, int S, int Hq, int Hkv,
+                int D, int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace, size_t ws_bytes,
+                void* stream) {
   if (!dQ) return fail(USP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(dQ)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   BwdLaunch L{};
-  const int rc = bwd_launch_setup(q, k, v, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, &L);
+  const int rc = bwd_launch_setup(q, k, v, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes, &L);
   if (rc != USP_OK) return rc;
   L.dq = dQ;
   const cudaError_t e = launch_attn_bwd_dq(L, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention backward (dQ) launch");
 }
 
-int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dO,
-                 void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D, int causal, int P_u,
-                 int P_r, void* workspace, size_t ws_bytes, void* stream) {
+int attn_bwd_impl(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dO,
+                  void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r,
+                  const usp_attn_mask* mask, void* workspace, size_t ws_bytes, void* stream) {
   AttnGeom g{};
   int rc = check_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
   if (rc != USP_OK) return rc;
+  MaskArgs mk{};
+  if ((rc = mask_args(mask, g, &mk)) != USP_OK) return rc;
   if (!q || !k || !v || !out || !lse || !dO || !dQ || !dK || !dV) return fail(USP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dO) ||
       !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
@@ -390,10 +447,40 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   if ((rc = usp_attn_bwd_prepare(out, lse, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream)) !=
       USP_OK)
     return rc;
-  if ((rc = usp_attn_bwd_dkdv(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes,
-                              stream)) != USP_OK)
+  if ((rc = bwd_dkdv_impl(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes,
+                          stream)) != USP_OK)
     return rc;
-  return usp_attn_bwd_dq(q, k, v, dO, dQ, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream);
+  return bwd_dq_impl(q, k, v, dO, dQ, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes, stream);
+}
+}  // namespace
+
+extern "C" {
+
+int usp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, float* dK, float* dV, int B,
+                      int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes,
+                      void* stream) {
+  return bwd_dkdv_impl(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, nullptr, workspace, ws_bytes,
+                       stream);
+}
+
+int usp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dQ, int B, int S, int Hq,
+                    int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream) {
+  return bwd_dq_impl(q, k, v, dO, dQ, B, S, Hq, Hkv, D, causal, P_u, P_r, nullptr, workspace, ws_bytes, stream);
+}
+
+int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dO,
+                 void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D, int causal, int P_u,
+                 int P_r, void* workspace, size_t ws_bytes, void* stream) {
+  return attn_bwd_impl(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, nullptr, workspace,
+                       ws_bytes, stream);
+}
+
+int usp_attn_bwd_masked(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                        const void* dO, void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D,
+                        int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  return attn_bwd_impl(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace,
+                       ws_bytes, stream);
 }
 
 int usp_lse_merge(const float* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,

@@ -68,6 +68,7 @@ struct BwdArgs {
   float* dv;
   int* status;
   unsigned long long wait_ns;
+  int loc_i, loc_u, loc_j;  // local mode: query rank (i, u), KV block of ring rank j
 };
 
 struct BwdBars {
@@ -103,12 +104,29 @@ __device__ __forceinline__ int classify_q(const Geo& g, int i, int m, int kmin, 
   return kMasked;
 }
 
-__device__ __forceinline__ void qwalk_settle(const Geo& g, int j, int kmin, int kmax, QWalk& w) {
+// Masked variant: the causal kind narrowed by the block / document masks (the
+// query tile of ring rank i, tile m, head hh of the group of kv-head gl).
+struct MaskedQ {
+  const Geo& g;
+  int b, u, gl, kmin, kmax;
+  __device__ __forceinline__ int operator()(int hh, int i, int m) const {
+    const int kind = classify_q(g, i, m, kmin, kmax);
+    int qmin, qmax;
+    pos_range(g, i, m * kBM, m * kBM + kBM, qmin, qmax);
+    return mask_tile(g.mask, kind, b, u * g.Hq_l + gl * g.G + hh, qmin, qmax, kmin, kmax);
+  }
+};
+
+// Steps t in [t_lo, t_hi) of the walk: all ring ranks i = (j + t) mod P_r, or
+// in the local mode the one rank that computes.
+template <bool kMask>
+__device__ __forceinline__ void qwalk_settle(const Geo& g, int j, int kmin, int kmax, QWalk& w, const MaskedQ& mq,
+                                             int t_lo, int t_hi) {
   while (w.hh < g.G) {
-    while (w.t < g.P_r) {
+    while (w.t < t_hi) {
       w.i = (j + w.t) % g.P_r;
       while (w.m < g.n_qtiles) {
-        w.kind = classify_q(g, w.i, w.m, kmin, kmax);
+        w.kind = kMask ? mq(w.hh, w.i, w.m) : classify_q(g, w.i, w.m, kmin, kmax);
         if (w.kind != kSkip) {
           w.valid = true;
           return;
@@ -119,23 +137,31 @@ __device__ __forceinline__ void qwalk_settle(const Geo& g, int j, int kmin, int 
       w.m = 0;
     }
     ++w.hh;
-    w.t = 0;
+    w.t = t_lo;
   }
   w.valid = false;
 }
 
-__device__ __forceinline__ QWalk qwalk_begin(const Geo& g, int j, int kmin, int kmax) {
-  QWalk w{0, 0, 0, 0, 0, false};
-  qwalk_settle(g, j, kmin, kmax, w);
+template <bool kMask>
+__device__ __forceinline__ QWalk qwalk_begin(const Geo& g, int j, int kmin, int kmax, const MaskedQ& mq, int t_lo,
+                                             int t_hi) {
+  QWalk w{0, t_lo, 0, 0, 0, false};
+  qwalk_settle<kMask>(g, j, kmin, kmax, w, mq, t_lo, t_hi);
   return w;
 }
 
-__device__ __forceinline__ void qwalk_next(const Geo& g, int j, int kmin, int kmax, QWalk& w) {
+template <bool kMask>
+__device__ __forceinline__ void qwalk_next(const Geo& g, int j, int kmin, int kmax, QWalk& w, const MaskedQ& mq,
+                                           int t_lo, int t_hi) {
   ++w.m;
-  qwalk_settle(g, j, kmin, kmax, w);
+  qwalk_settle<kMask>(g, j, kmin, kmax, w, mq, t_lo, t_hi);
 }
 
-template <int D>
+// kLocal: ONE rank of a real multi-GPU mesh -- the KV block of ring rank loc_j
+// it holds (its own buffers, [B][L][Hkv/P_u][D]) against the queries of rank
+// (loc_i, loc_u) only; dK and dV are ADDED to the given fp32 buffers (the
+// gradients travelling with the block around the ring).
+template <int D, bool kMask, bool kLocal>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -160,17 +186,30 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
   // Work item: CTAs of one (b, Ulysses rank, kv-head) run together; inside it,
   // key tiles in increasing original position (the causally heaviest first).
-  const int n_kt = g.P_r * g.n_ktiles;
-  int wi = blockIdx.x;
-  const int order = wi % n_kt;
-  wi /= n_kt;
-  const int gl = wi % g.Hkv_l;
-  wi /= g.Hkv_l;
-  const int u = wi % g.P_u;
-  const int b = wi / g.P_u;
-  int j, n;
-  tile_in_position_order(g, order, j, n);
-  const int jrank = j * g.P_u + u;
+  int gl, u, b, j, n;
+  if constexpr (kLocal) {
+    int wi = blockIdx.x;
+    n = wi % g.n_ktiles;
+    wi /= g.n_ktiles;
+    gl = wi % g.Hkv_l;
+    b = wi / g.Hkv_l;
+    u = a.loc_u;
+    j = a.loc_j;
+  } else {
+    const int n_kt = g.P_r * g.n_ktiles;
+    int wi = blockIdx.x;
+    const int order = wi % n_kt;
+    wi /= n_kt;
+    gl = wi % g.Hkv_l;
+    wi /= g.Hkv_l;
+    u = wi % g.P_u;
+    b = wi / g.P_u;
+    tile_in_position_order(g, order, j, n);
+  }
+  const int jrank = kLocal ? 0 : j * g.P_u + u;  // local buffers hold one rank
+  // ring steps walked: every rank's queries, or those of the one local rank
+  const int t_lo = kLocal ? (a.loc_i - j + g.P_r) % g.P_r : 0;
+  const int t_hi = kLocal ? t_lo + 1 : g.P_r;
   const int k0 = n * kBN;
   int kmin, kmax;
   pos_range(g, j, k0, k0 + kBN, kmin, kmax);
@@ -220,7 +259,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         tma_load_4d_w(&tm_v, &bars->kv_full, sV + p * C::kPanelBytes, p * 64, gl, k0, krb);
       }
       int issued = 0;
-      QWalk qw = qwalk_begin(g, j, kmin, kmax);
+      const MaskedQ mq{g, b, u, gl, kmin, kmax};
+      QWalk qw = qwalk_begin<kMask>(g, j, kmin, kmax, mq, t_lo, t_hi);
       while (true) {
         const int s = issued % C::kStages;
         if (issued >= C::kStages &&
@@ -241,7 +281,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         }
         __syncwarp();
         const int h = gl * g.G + qw.hh;
-        const int qrb = (qw.i * g.P_u + u) * g.B + b;
+        const int qrb = kLocal ? b : (qw.i * g.P_u + u) * g.B + b;
         const int q0 = qw.m * kBM;
         mbar_expect_tx_w(&bars->qd_full[s], 2 * C::kTileBytes + 1024);
         for (int p = 0; p < C::kPanels; ++p) {
@@ -253,7 +293,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         bulk_load_1d_w(sRow + s * 256, a.lse2 + rowbase, 512, &bars->qd_full[s]);
         bulk_load_1d_w(sRow + s * 256 + 128, a.delta + rowbase, 512, &bars->qd_full[s]);
         ++issued;
-        qwalk_next(g, j, kmin, kmax, qw);
+        qwalk_next<kMask>(g, j, kmin, kmax, qw, mq, t_lo, t_hi);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         mbar_wait_drain(&bars->kv_full, 0, a.wait_ns);
@@ -352,6 +392,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const int tau_k = k0 + row;
     const int pos_k = tau_k < g.L ? token_pos(g, j, tau_k) : INT_MAX;  // padding keys see no query
+    int doc_lo = 0, doc_hi = INT_MAX;  // the key's document [lo, hi) (masked variant)
+    if constexpr (kMask) doc_span(g.mask, pos_k, doc_lo, doc_hi);
     const bool aligned = (g.c % kBM) == 0;
     const int cbase = wg * 64;
     bool ok = true;
@@ -373,7 +415,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       if (st_kind == kMasked) {
         // causal: rewrite S^T of this key row to -inf where the query does not see
         // the key, so the main pass carries no masking (P = 0 there)
-        const int lo = pos_k == INT_MAX ? kBM : pos_k - token_pos(g, st_i, q0);  // aligned: cols >= lo see it
+        int lo = pos_k == INT_MAX ? kBM : pos_k - token_pos(g, st_i, q0);  // aligned: cols >= lo see it
+        int hi_c = kBM;                                                      // and cols < hi_c
+        if constexpr (kMask) {
+          // masked variant (tiles contiguous): the key's document bounds the columns too
+          const int qpos0 = token_pos(g, st_i, q0);
+          if (!g.causal && pos_k != INT_MAX) lo = 0;
+          if (pos_k != INT_MAX) {
+            lo = max(lo, doc_lo - qpos0);
+            if (doc_hi != INT_MAX) hi_c = doc_hi - qpos0;
+          }
+        }
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           const int c0 = cbase + half * 32;
@@ -381,6 +433,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           if (aligned) {
             const int nb = min(max(lo - c0, 0), 32);  // leading invisible columns
             vis = nb >= 32 ? 0u : (0xFFFFFFFFu << nb);
+            if constexpr (kMask) {
+              const int nt = min(max(hi_c - c0, 0), 32);  // columns below hi_c
+              vis &= nt >= 32 ? 0xFFFFFFFFu : ((1u << nt) - 1u);
+            }
           } else {
             vis = 0u;
             for (int c = 0; c < 32; ++c) {
@@ -480,10 +536,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           float4* dvp = reinterpret_cast<float4*>(a.dv + kr * D + c0);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            dkp[q] = make_float4(__uint_as_float(rk[4 * q]) * g.scale, __uint_as_float(rk[4 * q + 1]) * g.scale,
-                                 __uint_as_float(rk[4 * q + 2]) * g.scale, __uint_as_float(rk[4 * q + 3]) * g.scale);
-            dvp[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
-                                 __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
+            float4 nk = make_float4(__uint_as_float(rk[4 * q]) * g.scale, __uint_as_float(rk[4 * q + 1]) * g.scale,
+                                    __uint_as_float(rk[4 * q + 2]) * g.scale, __uint_as_float(rk[4 * q + 3]) * g.scale);
+            float4 nv = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
+                                    __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
+            if constexpr (kLocal) {  // add to the gradients travelling with the block
+              const float4 ok_ = dkp[q], ov = dvp[q];
+              nk = make_float4(nk.x + ok_.x, nk.y + ok_.y, nk.z + ok_.z, nk.w + ok_.w);
+              nv = make_float4(nv.x + ov.x, nv.y + ov.y, nv.z + ov.z, nv.w + ov.w);
+            }
+            dkp[q] = nk;
+            dvp[q] = nv;
           }
         }
       }
@@ -498,15 +561,16 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   }
 }
 
-template <int D>
+template <int D, bool kMask, bool kLocal>
 cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   using C = BwdCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, kMask, kLocal>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   BwdArgs a{};
   a.g = make_geo(L.g);
+  a.g.mask = L.mask;
   a.lse2 = L.lse2;
   a.delta = L.delta;
   a.Lp = L.Lp;
@@ -514,10 +578,14 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   a.dv = L.dv;
   a.status = L.status;
   a.wait_ns = L.wait_ns;
-  const long long blocks = static_cast<long long>(a.g.n_ktiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hkv_l;
+  a.loc_i = L.loc_i;
+  a.loc_u = L.loc_u;
+  a.loc_j = L.loc_j;
+  const long long blocks = kLocal ? static_cast<long long>(a.g.n_ktiles) * a.g.B * a.g.Hkv_l
+                                  : static_cast<long long>(a.g.n_ktiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hkv_l;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  attn_bwd_kernel<D><<<static_cast<unsigned>(blocks), kThreadsBwd, C::kSmemBytes, stream>>>(
+  attn_bwd_kernel<D, kMask, kLocal><<<static_cast<unsigned>(blocks), kThreadsBwd, C::kSmemBytes, stream>>>(
       L.tm_q, L.tm_k, L.tm_v, L.tm_do, a);
   note_launch();
   return cudaGetLastError();
@@ -526,8 +594,20 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_attn_bwd(const BwdLaunch& L, cudaStream_t stream) {
-  if (L.g.D == 128) return launch_bwd_d<128>(L, stream);
-  if (L.g.D == 64) return launch_bwd_d<64>(L, stream);
+  const bool masked = L.mask.bm != nullptr || L.mask.cu != nullptr;
+  if (masked && L.local) return cudaErrorInvalidValue;
+  if (L.local) {
+    if (L.g.D == 128) return launch_bwd_d<128, false, true>(L, stream);
+    if (L.g.D == 64) return launch_bwd_d<64, false, true>(L, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (masked) {
+    if (L.g.D == 128) return launch_bwd_d<128, true, false>(L, stream);
+    if (L.g.D == 64) return launch_bwd_d<64, true, false>(L, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (L.g.D == 128) return launch_bwd_d<128, false, false>(L, stream);
+  if (L.g.D == 64) return launch_bwd_d<64, false, false>(L, stream);
   return cudaErrorInvalidValue;
 }
 

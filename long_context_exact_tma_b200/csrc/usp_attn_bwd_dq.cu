@@ -61,6 +61,8 @@ struct DqArgs {
   const float* ndelta;  // [n_ranks*B*Hq_l][Lp]: -Delta (0 on padding rows)
   int Lp;
   __nv_bfloat16* dq;    // bf16 [n_ranks][B][L][Hq_l][D]
+  float* dq_acc;        // local mode: fp32 [B][L][Hq_l][D], this step's dQ is added to it
+  int loc_i, loc_u, loc_t;  // local mode: the rank (i, u) and its ring step t
   int* status;
   unsigned long long wait_ns;
 };
@@ -82,7 +84,10 @@ enum : int {
   kSiteQDp = 0x323, kSiteQEpi = 0x324, kSiteQAlign = 0x3FF
 };
 
-template <int D>
+// kLocal: ONE rank (loc_i, loc_u) of a real multi-GPU mesh at ring step loc_t:
+// its own Q and dO against the KV block it holds (owner (i - t) mod P_r), its
+// own buffers ([B][L][H/P_u][D]); dQ is ADDED to the fp32 dq_acc.
+template <int D, bool kMask, bool kLocal>
 __global__ void __launch_bounds__(kThreadsDq, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -106,17 +111,30 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
 
   // Work item: CTAs of one (b, Ulysses rank, head) run together so that its K/V
   // stay in L2; inside it, query tiles in decreasing original position.
-  const int n_qt = g.P_r * g.n_qtiles;
-  int wi = blockIdx.x;
-  const int order = n_qt - 1 - wi % n_qt;
-  wi /= n_qt;
-  const int h = wi % g.Hq_l;
-  wi /= g.Hq_l;
-  const int u = wi % g.P_u;
-  const int b = wi / g.P_u;
-  int i, m;
-  tile_in_position_order(g, order, i, m);
-  const int rank = i * g.P_u + u;
+  int h, u, b, i, m;
+  if constexpr (kLocal) {
+    int wi = blockIdx.x;
+    m = g.n_qtiles - 1 - wi % g.n_qtiles;
+    wi /= g.n_qtiles;
+    h = wi % g.Hq_l;
+    b = wi / g.Hq_l;
+    i = a.loc_i;
+    u = a.loc_u;
+  } else {
+    const int n_qt = g.P_r * g.n_qtiles;
+    int wi = blockIdx.x;
+    const int order = n_qt - 1 - wi % n_qt;
+    wi /= n_qt;
+    h = wi % g.Hq_l;
+    wi /= g.Hq_l;
+    u = wi % g.P_u;
+    b = wi / g.P_u;
+    tile_in_position_order(g, order, i, m);
+  }
+  const int rank = kLocal ? 0 : i * g.P_u + u;  // local buffers hold one rank
+  // ring steps walked: all of them, or the local rank's one step
+  const int t_lo = kLocal ? a.loc_t : 0;
+  const int t_hi = kLocal ? a.loc_t + 1 : g.P_r;
   const int kvh = h / g.G;
   const int q0 = m * kBM;
 
@@ -158,7 +176,17 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     {
       int qmin, qmax;
       pos_range(g, i, q0, q0 + kBM, qmin, qmax);
-      KvWalk kw = kv_walk_begin(g, i, qmin, qmax, 0, g.P_r);
+      // masked variant: the causal kind narrowed by the block / document masks
+      auto kind_of = [&](int j, int n) {
+        int kmin, kmax;
+        pos_range(g, j, n * kBN, n * kBN + kBN, kmin, kmax);
+        return mask_tile(g.mask, classify_tile(g, qmin, qmax, j, n), b, u * g.Hq_l + h, qmin, qmax, kmin, kmax);
+      };
+      KvWalk kw;
+      if constexpr (kMask)
+        kw = kv_walk_begin_by(g, i, t_lo, t_hi, kind_of);
+      else
+        kw = kv_walk_begin(g, i, qmin, qmax, t_lo, t_hi);
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -193,7 +221,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
           slot[3] = kw.kind;
         }
         __syncwarp();
-        const int krb = (kw.j * g.P_u + u) * g.B + b;
+        const int krb = kLocal ? b : (kw.j * g.P_u + u) * g.B + b;
         mbar_expect_tx_w(&bars->k_full[sk], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_4d_w(&tm_k, &bars->k_full[sk], sK + sk * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
@@ -207,7 +235,10 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
           tma_load_4d_w(&tm_v, &bars->v_full[sv], sV + sv * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
                         kw.n * kBN, krb);
         ++v_issued;
-        kv_walk_next(g, i, qmin, qmax, g.P_r, kw);
+        if constexpr (kMask)
+          kv_walk_next_by(g, i, t_hi, kw, kind_of);
+        else
+          kv_walk_next(g, i, qmin, qmax, t_hi, kw);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         // Let every copy this warp started land before the CTA exits.
@@ -324,6 +355,8 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     const int tau_q = q0 + row;
     const int pos_q = tau_q < g.L ? token_pos(g, i, tau_q) : INT_MAX;
     const bool aligned = (g.c % kBN) == 0;
+    int doc_lo = 0, doc_hi = INT_MAX;  // the row's document [lo, hi) (masked variant)
+    if constexpr (kMask) doc_span(g.mask, pos_q, doc_lo, doc_hi);
     const size_t tab = (static_cast<size_t>(rank * g.B + b) * g.Hq_l + h) * a.Lp + tau_q;
     const float nl = __ldg(a.nlse2 + tab);   // -inf on padding rows: their P is 0
     const float nd = __ldg(a.ndelta + tab);
@@ -348,6 +381,12 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
         const int k0 = kn * kBN;
         int lim = min(127, g.L - k0 - 1);  // keys at or past L are padding
         if (aligned && g.causal) lim = min(lim, pos_q - token_pos(g, kj, k0));
+        int first = 0;  // first visible column (documents: keys from the row's document start)
+        if constexpr (kMask) {
+          const int kpos0 = token_pos(g, kj, k0);  // tiles are contiguous under a mask
+          if (doc_hi != INT_MAX) lim = min(lim, doc_hi - 1 - kpos0);
+          first = max(0, doc_lo - kpos0);
+        }
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           const int c0 = cbase + half * 32;
@@ -355,6 +394,10 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
           if (aligned) {
             const int nb = min(max(lim - c0 + 1, 0), 32);
             vis = nb >= 32 ? 0xFFFFFFFFu : ((1u << nb) - 1u);
+            if constexpr (kMask) {
+              const int nlo = min(max(first - c0, 0), 32);  // leading invisible columns
+              vis &= nlo >= 32 ? 0u : (0xFFFFFFFFu << nlo);
+            }
           } else {
             vis = 0u;
             for (int c = 0; c < 32; ++c) {
@@ -420,7 +463,37 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = 0u;
         }
-        if (store) {
+        if (store && kLocal) {
+          // add this step's dQ to the fp32 accumulator; on the last step (a bf16
+          // output given) write the sum as bf16 instead
+          const float4* acc = reinterpret_cast<const float4*>(a.dq_acc + qr * D + c0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 ov = acc[q];
+            o[q * 4 + 0] = __float_as_uint(ov.x + __uint_as_float(o[q * 4 + 0]) * g.scale);
+            o[q * 4 + 1] = __float_as_uint(ov.y + __uint_as_float(o[q * 4 + 1]) * g.scale);
+            o[q * 4 + 2] = __float_as_uint(ov.z + __uint_as_float(o[q * 4 + 2]) * g.scale);
+            o[q * 4 + 3] = __float_as_uint(ov.w + __uint_as_float(o[q * 4 + 3]) * g.scale);
+          }
+          if (a.dq == nullptr) {
+            float4* dst = reinterpret_cast<float4*>(a.dq_acc + qr * D + c0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(__uint_as_float(o[q * 4]), __uint_as_float(o[q * 4 + 1]),
+                                   __uint_as_float(o[q * 4 + 2]), __uint_as_float(o[q * 4 + 3]));
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(a.dq + qr * D + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(o[q * 8 + 0]), __uint_as_float(o[q * 8 + 1]));
+              v.y = pack_bf16x2(__uint_as_float(o[q * 8 + 2]), __uint_as_float(o[q * 8 + 3]));
+              v.z = pack_bf16x2(__uint_as_float(o[q * 8 + 4]), __uint_as_float(o[q * 8 + 5]));
+              v.w = pack_bf16x2(__uint_as_float(o[q * 8 + 6]), __uint_as_float(o[q * 8 + 7]));
+              dst[q] = v;
+            }
+          }
+        } else if (store) {
           uint4* dst = reinterpret_cast<uint4*>(a.dq + qr * D + c0);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -444,25 +517,31 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
   }
 }
 
-template <int D>
+template <int D, bool kMask, bool kLocal>
 cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
   using C = DqCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kMask, kLocal>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   DqArgs a{};
   a.g = make_geo(L.g);
+  a.g.mask = L.mask;
   a.nlse2 = L.lse2;
   a.ndelta = L.delta;
   a.Lp = L.Lp;
   a.dq = static_cast<__nv_bfloat16*>(L.dq);
+  a.dq_acc = L.dq_acc;
+  a.loc_i = L.loc_i;
+  a.loc_u = L.loc_u;
+  a.loc_t = L.loc_t;
   a.status = L.status;
   a.wait_ns = L.wait_ns;
-  const long long blocks = static_cast<long long>(a.g.n_qtiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;
+  const long long blocks = kLocal ? static_cast<long long>(a.g.n_qtiles) * a.g.B * a.g.Hq_l
+                                  : static_cast<long long>(a.g.n_qtiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  attn_bwd_dq_kernel<D><<<static_cast<unsigned>(blocks), kThreadsDq, C::kSmemBytes, stream>>>(
+  attn_bwd_dq_kernel<D, kMask, kLocal><<<static_cast<unsigned>(blocks), kThreadsDq, C::kSmemBytes, stream>>>(
       L.tm_q, L.tm_k, L.tm_v, L.tm_do, a);
   note_launch();
   return cudaGetLastError();
@@ -471,8 +550,20 @@ cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_attn_bwd_dq(const BwdLaunch& L, cudaStream_t stream) {
-  if (L.g.D == 128) return launch_dq_d<128>(L, stream);
-  if (L.g.D == 64) return launch_dq_d<64>(L, stream);
+  const bool masked = L.mask.bm != nullptr || L.mask.cu != nullptr;
+  if (masked && L.local) return cudaErrorInvalidValue;
+  if (L.local) {
+    if (L.g.D == 128) return launch_dq_d<128, false, true>(L, stream);
+    if (L.g.D == 64) return launch_dq_d<64, false, true>(L, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (masked) {
+    if (L.g.D == 128) return launch_dq_d<128, true, false>(L, stream);
+    if (L.g.D == 64) return launch_dq_d<64, true, false>(L, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (L.g.D == 128) return launch_dq_d<128, false, false>(L, stream);
+  if (L.g.D == 64) return launch_dq_d<64, false, false>(L, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -40,6 +40,7 @@ namespace usp {
 namespace {
 
 constexpr int kThreadsFwd = 320;
+enum : int { kModeUsp = 0, kModeSub = 1, kModeLocal = 2 };
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThresh = 8.0f;  // log2 units: rescale O only if the max grows by > 256x
 
@@ -69,6 +70,7 @@ struct FwdArgs {
   int* status;
   unsigned long long wait_ns;
   FwdSub sub;  // sub-problem mode (kSub): see usp_internal.h
+  int loc_i, loc_u;  // local mode: the one rank (ring i, Ulysses u) this launch computes
 };
 
 struct FwdBars {
@@ -103,10 +105,17 @@ __device__ __forceinline__ void pair_in_position_order(const Geo& g, int o, int&
   }
 }
 
-template <int D, bool kSub>
+// kMode: kModeUsp -- every virtual rank of the mesh, Q/K/V of all ranks in one
+// head-sharded tensor; kModeSub -- independent one-rank problems (dilated
+// attention); kModeLocal -- ONE rank (i, u) of a real multi-GPU mesh: its own Q
+// ([B][L][Hq/P_u][D]) against the one KV block it holds at ring step `step`
+// (owner j = (i - step) mod P_r, [B][L][Hkv/P_u][D]), positions as in the mesh.
+template <int D, int kMode, bool kMask>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+  constexpr bool kSub = kMode == kModeSub;
+  constexpr bool kLocal = kMode == kModeLocal;
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -130,6 +139,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     qc4 = wi / a.sub.n_heads;  // the problem
     u = b = i = 0;
     m = 2 * order;
+  } else if constexpr (kLocal) {
+    // work item: (b, head, pair of query tiles) of the one rank, heaviest first
+    const int np = (g.n_qtiles + 1) / 2;
+    int wi = blockIdx.x;
+    const int order = np - 1 - wi % np;
+    wi /= np;
+    h = wi % g.Hq_l;
+    b = wi / g.Hq_l;
+    i = a.loc_i;
+    u = a.loc_u;
+    m = 2 * order;
+    qc4 = 0;
   } else {
     // Work item: CTAs of one (b, Ulysses rank, head) run together so that its K/V
     // stay in L2; inside it, query-tile pairs in decreasing original position
@@ -146,7 +167,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     pair_in_position_order(g, order, i, m);
     qc4 = 0;
   }
-  const int rank = kSub ? 0 : i * g.P_u + u;
+  const int rank = (kSub || kLocal) ? 0 : i * g.P_u + u;  // local buffers hold one rank
   const int kvh = h / g.G;
   const int q0 = m * kBM;
   const int t_begin = a.step < 0 ? 0 : a.step;
@@ -188,7 +209,22 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       pos_range<kSub>(g, i, q0, q0 + kBM, qmin0, qmax0);
       pos_range<kSub>(g, i, q0 + kBM, q0 + 2 * kBM, qmin1, qmax1);
       const int qmin = min(qmin0, qmin1), qmax = max(qmax0, qmax1);
-      KvWalk kw = kv_walk_begin<kSub>(g, i, qmin, qmax, t_begin, t_end);
+      // masked variant: both query tiles' kinds narrowed by the block / document
+      // masks; a key tile is walked when either query tile attends it
+      const int hg = u * g.Hq_l + h;
+      auto kinds_of = [&](int j, int n) {
+        int k0c = classify_tile<kSub>(g, qmin0, qmax0, j, n), k1c = classify_tile<kSub>(g, qmin1, qmax1, j, n);
+        int kmin, kmax;
+        pos_range<kSub>(g, j, n * kBN, n * kBN + kBN, kmin, kmax);
+        k0c = mask_tile(g.mask, k0c, b, hg, qmin0, qmax0, kmin, kmax);
+        k1c = mask_tile(g.mask, k1c, b, hg, qmin1, qmax1, kmin, kmax);
+        return k0c | (k1c << 4);
+      };
+      KvWalk kw;
+      if constexpr (kMask)
+        kw = kv_walk_begin_by(g, i, t_begin, t_end, kinds_of);
+      else
+        kw = kv_walk_begin<kSub>(g, i, qmin, qmax, t_begin, t_end);
       int issued = 0;
       const bool any = kw.valid;
       if (any) {
@@ -216,8 +252,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           mbar_arrive_w(&bars->k_full[s]);
           break;
         }
-        const int kinds =
-            classify_tile<kSub>(g, qmin0, qmax0, kw.j, kw.n) | (classify_tile<kSub>(g, qmin1, qmax1, kw.j, kw.n) << 4);
+        const int kinds = kMask ? kw.kind
+                                : classify_tile<kSub>(g, qmin0, qmax0, kw.j, kw.n) |
+                                      (classify_tile<kSub>(g, qmin1, qmax1, kw.j, kw.n) << 4);
         if (lane == 0) {
           slot[0] = 1;
           slot[1] = kw.j;
@@ -225,7 +262,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           slot[3] = kinds;
         }
         __syncwarp();
-        const int krb = kSub ? qc4 : (kw.j * g.P_u + u) * g.B + b;
+        const int krb = kSub ? qc4 : kLocal ? b : (kw.j * g.P_u + u) * g.B + b;
         mbar_expect_tx_w(&bars->k_full[s], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_4d_w(&tm_k, &bars->k_full[s], sK + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
@@ -235,7 +272,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           tma_load_4d_w(&tm_v, &bars->v_full[s], sV + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
                         kw.n * kBN, krb);
         ++issued;
-        kv_walk_next<kSub>(g, i, qmin, qmax, t_end, kw);
+        if constexpr (kMask)
+          kv_walk_next_by(g, i, t_end, kw, kinds_of);
+        else
+          kv_walk_next<kSub>(g, i, qmin, qmax, t_end, kw);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         // Let every copy this warp started land before the CTA exits.
@@ -323,6 +363,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const int tau_q = q0 + t * kBM + row;
     const int pos_q = tau_q < g.L ? token_pos<kSub>(g, i, tau_q) : INT_MAX;
     const bool aligned = (g.c % kBN) == 0;
+    int doc_lo = 0, doc_hi = INT_MAX;  // the row's document [lo, hi) (masked variant)
+    if constexpr (kMask) doc_span(g.mask, pos_q, doc_lo, doc_hi);
     // l_run: sum of the fp32 weights (for LSE); lb_run: sum of the bf16-rounded
     // weights the PV UMMA consumes (normalises O, so O stays a convex combination
     // of V rows even when one key dominates).
@@ -344,6 +386,14 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         const int k0 = kn * kBN;
         int lim = kkind == kSkip ? -1 : min(127, g.L - k0 - 1);  // keys at or past L are padding
         if (kkind == kMasked && aligned && g.causal) lim = min(lim, pos_q - token_pos<kSub>(g, kj, k0));
+        int first = 0;  // first visible column (documents: keys from the row's document start)
+        if constexpr (kMask) {
+          if (kkind == kMasked) {
+            const int kpos0 = token_pos<kSub>(g, kj, k0);  // tiles are contiguous under a mask
+            lim = min(lim, doc_hi == INT_MAX ? 127 : doc_hi - 1 - kpos0);
+            first = max(0, doc_lo - kpos0);
+          }
+        }
         const bool per_key = kkind == kMasked && !aligned;  // chunks shorter than a tile
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -351,6 +401,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           if (!per_key) {
             const int nb = min(max(lim - c0 + 1, 0), 32);
             vis = nb >= 32 ? 0xFFFFFFFFu : ((1u << nb) - 1u);
+            if constexpr (kMask) {
+              const int nlo = min(max(first - c0, 0), 32);  // leading invisible columns
+              vis &= nlo >= 32 ? 0u : (0xFFFFFFFFu << nlo);
+            }
           } else {
             vis = 0u;
             for (int c = 0; c < 32; ++c) {
@@ -551,12 +605,13 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   }
 }
 
-template <int D, bool kSub>
+template <int D, int kMode, bool kMask>
 cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
+  constexpr bool kSub = kMode == kModeSub;
   using C = FwdCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, kSub>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, kMode, kMask>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a{};
   a.g = make_geo(L.g);
@@ -568,6 +623,7 @@ cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
   a.status = L.status;
   a.wait_ns = L.wait_ns;
   a.sub = L.sub;
+  a.g.mask = L.mask;
   long long blocks;
   if (kSub) {
     // every problem: one rank, L = sub.L rows whose local index is the position
@@ -577,13 +633,17 @@ cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
     a.g.c = kBN;
     a.g.n_qtiles = a.g.n_ktiles = (L.sub.L + kBM - 1) / kBM;
     blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * L.sub.n_heads * L.sub.n_prob;
+  } else if (kMode == kModeLocal) {
+    a.loc_i = L.loc_i;
+    a.loc_u = L.loc_u;
+    blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * a.g.B * a.g.Hq_l;
   } else {
     blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;
   }
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  attn_fwd_kernel<D, kSub><<<static_cast<unsigned>(blocks), kThreadsFwd, C::kSmemBytes, stream>>>(L.tm_q, L.tm_k,
-                                                                                                 L.tm_v, a);
+  attn_fwd_kernel<D, kMode, kMask><<<static_cast<unsigned>(blocks), kThreadsFwd, C::kSmemBytes, stream>>>(
+      L.tm_q, L.tm_k, L.tm_v, a);
   note_launch();
   return cudaGetLastError();
 }
@@ -591,13 +651,25 @@ cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_attn_fwd(const FwdLaunch& L, cudaStream_t stream) {
+  const bool masked = L.mask.bm != nullptr || L.mask.cu != nullptr;
+  if ((L.sub.active || L.local) && masked) return cudaErrorInvalidValue;  // masks: emulated mesh only
   if (L.sub.active) {
-    if (L.g.D == 128) return launch_fwd_d<128, true>(L, stream);
-    if (L.g.D == 64) return launch_fwd_d<64, true>(L, stream);
+    if (L.g.D == 128) return launch_fwd_d<128, kModeSub, false>(L, stream);
+    if (L.g.D == 64) return launch_fwd_d<64, kModeSub, false>(L, stream);
     return cudaErrorInvalidValue;
   }
-  if (L.g.D == 128) return launch_fwd_d<128, false>(L, stream);
-  if (L.g.D == 64) return launch_fwd_d<64, false>(L, stream);
+  if (L.local) {
+    if (L.g.D == 128) return launch_fwd_d<128, kModeLocal, false>(L, stream);
+    if (L.g.D == 64) return launch_fwd_d<64, kModeLocal, false>(L, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (masked) {
+    if (L.g.D == 128) return launch_fwd_d<128, kModeUsp, true>(L, stream);
+    if (L.g.D == 64) return launch_fwd_d<64, kModeUsp, true>(L, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (L.g.D == 128) return launch_fwd_d<128, kModeUsp, false>(L, stream);
+  if (L.g.D == 64) return launch_fwd_d<64, kModeUsp, false>(L, stream);
   return cudaErrorInvalidValue;
 }
 

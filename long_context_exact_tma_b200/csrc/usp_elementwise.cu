@@ -178,7 +178,10 @@ __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16*
       const long long h = r % Hl, rt = r / Hl, tau = rt % L, rb = rt / L;
       const long long dst = (rb * Hl + h) * Lp + tau;
       delta_t[dst] = -acc;
-      lse2_t[dst] = -lse[r] * 1.4426950408889634f;
+      // a row that saw no key (LSE = -inf, O = 0; masked attention) must give
+      // P = 0, as the padding rows do, not exp2(+inf)
+      const float l = lse[r];
+      lse2_t[dst] = l == -INFINITY ? -INFINITY : -l * 1.4426950408889634f;
     }
   }
   // Padding rows [L, Lp) of every head: LSE = +inf and Delta = 0, so a padded

@@ -18,6 +18,10 @@ void note_launch();
 // The calling thread's bounded-wait limit (usp_set_wait_limit_ns).
 unsigned long long current_wait_ns();
 
+struct AttnGeom;
+// The shape checks of the attention calls; fills g; usp_status (message recorded).
+int validate_geom(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, AttnGeom* g);
+
 // Tensor map of a bf16 tensor viewed as {D, H, rows, n4} with the given row and
 // block strides in bytes (box 64 x 1 x 128 x 1, 128-byte swizzle); usp_status.
 int make_tmap_strided(CUtensorMap* m, const void* base, int D, int H, long long rows, long long n4,
@@ -27,7 +31,17 @@ int make_tmap_strided(CUtensorMap* m, const void* base, int D, int H, long long 
 cudaError_t launch_fill_running(float* o, float* lse, long long rows, int D, cudaStream_t stream);
 
 // Layout maps of the gather kernel (see usp_layout.cu).
-enum LayoutMap { kZigzagShard = 0, kZigzagUnshard = 1, kSeq2Head = 2, kHead2Seq = 3 };
+// The last four are the local halves of a real Ulysses all-to-all between G
+// ranks holding T tokens each (run = the H/G heads of a group):
+//   kPackHeads    [B][T][G][run] -> [G][B][T][run]  (send buffer of seq->head)
+//   kUnpackTokens [G][B][T][run] -> [B][G][T][run]  (receive buffer of seq->head)
+//   kPackTokens   [B][G][T][run] -> [G][B][T][run]  (send buffer of head->seq)
+//   kUnpackHeads  [G][B][T][run] -> [B][T][G][run]  (receive buffer of head->seq)
+// For these, LayoutArgs.S is T, P_u is G and P_r is 1.
+enum LayoutMap {
+  kZigzagShard = 0, kZigzagUnshard = 1, kSeq2Head = 2, kHead2Seq = 3,
+  kPackHeads = 4, kUnpackTokens = 5, kPackTokens = 6, kUnpackHeads = 7
+};
 
 struct LayoutArgs {
   const uint8_t* src;
@@ -47,6 +61,14 @@ cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n
 cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D,
                                   cudaStream_t stream);
 cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
+
+// Block-sparse / document masks of the masked attention variants (see
+// usp_attn_common.cuh); all null for plain causal or full attention.
+struct MaskArgs {
+  const uint8_t* bm;  // [B][Hq][nb][nb] block mask over 128-position blocks, or null
+  const int* cu;      // [n_docs + 1] document boundaries, or null
+  int nb, n_docs, Hq;
+};
 
 // Geometry of one attention problem in the head-sharded layout.
 struct AttnGeom {
@@ -81,6 +103,9 @@ struct FwdLaunch {
   int* status;
   unsigned long long wait_ns;
   FwdSub sub;         // sub-problem mode when sub.active
+  MaskArgs mask;      // masked variant when mask.bm or mask.cu is set
+  int local;          // local mode: one rank (loc_i, loc_u) of a real mesh, its own buffers (B in dim 4)
+  int loc_i, loc_u;
 };
 cudaError_t launch_attn_fwd(const FwdLaunch& a, cudaStream_t stream);
 
@@ -101,6 +126,12 @@ struct BwdLaunch {
   float* dv;           // fp32, v layout
   int* status;
   unsigned long long wait_ns;
+  MaskArgs mask;       // masked variant when mask.bm or mask.cu is set
+  // local mode: one rank (loc_i, loc_u) of a real mesh at ring step loc_t, whose
+  // KV block belongs to ring rank loc_j = (loc_i - loc_t) mod P_r; its own buffers
+  // (B in dim 4); dK, dV and the fp32 dq_acc are accumulated into
+  int local, loc_i, loc_u, loc_t, loc_j;
+  float* dq_acc;
 };
 cudaError_t launch_attn_bwd(const BwdLaunch& a, cudaStream_t stream);     // dK, dV (key-major)
 cudaError_t launch_attn_bwd_dq(const BwdLaunch& a, cudaStream_t stream);  // dQ (query-major)

@@ -79,6 +79,30 @@ __device__ __forceinline__ void run_offsets(const RunMap& m, uint32_t q, uint64_
       dof = static_cast<uint64_t>(q) * m.run_bytes;
       break;
     }
+    case kPackHeads: {  // dst (g, b, t) <- src (b, t, g)
+      const uint32_t t = q % m.S, q1 = q / m.S, b = q1 % m.B, gg = q1 / m.B;
+      so = (static_cast<uint64_t>(b * m.S + t) * m.P_u + gg) * m.run_bytes;
+      dof = static_cast<uint64_t>(q) * m.run_bytes;
+      break;
+    }
+    case kUnpackHeads: {  // dst (b, t, g) <- src (g, b, t)
+      const uint32_t gg = q % m.P_u, q1 = q / m.P_u, t = q1 % m.S, b = q1 / m.S;
+      so = (static_cast<uint64_t>(gg * m.B + b) * m.S + t) * m.run_bytes;
+      dof = static_cast<uint64_t>(q) * m.run_bytes;
+      break;
+    }
+    case kPackTokens: {  // dst (g, b, t) <- src (b, g, t)
+      const uint32_t t = q % m.S, q1 = q / m.S, b = q1 % m.B, gg = q1 / m.B;
+      so = (static_cast<uint64_t>(b * m.P_u + gg) * m.S + t) * m.run_bytes;
+      dof = static_cast<uint64_t>(q) * m.run_bytes;
+      break;
+    }
+    case kUnpackTokens: {  // dst (b, g, t) <- src (g, b, t)
+      const uint32_t t = q % m.S, q1 = q / m.S, gg = q1 % m.P_u, b = q1 / m.P_u;
+      so = (static_cast<uint64_t>(gg * m.B + b) * m.S + t) * m.run_bytes;
+      dof = static_cast<uint64_t>(q) * m.run_bytes;
+      break;
+    }
     default: {  // kHead2Seq: dst rank (r), b, t, head group u <- (i,u,b,tau)
       const uint32_t u = q % m.P_u, q1 = q / m.P_u, t = q1 % m.c2, rb = q1 / m.c2;
       const uint32_t b = rb % m.B, r = rb / m.B;
@@ -212,6 +236,9 @@ RunMap make_map(int map, uint32_t B, uint32_t S, uint32_t H, uint32_t P_u, uint3
   if (map == kZigzagShard || map == kZigzagUnshard) {
     m.run_bytes = H * row_bytes;
     m.n_runs = B * S;
+  } else if (map >= kPackHeads) {  // S = T tokens per rank, P_u = G ranks
+    m.run_bytes = m.Hl * row_bytes;
+    m.n_runs = B * S * P_u;
   } else {
     m.run_bytes = m.Hl * row_bytes;
     m.n_runs = B * S * P_u;
@@ -248,6 +275,10 @@ cudaError_t launch_layout_batch(const LayoutArgs* a, int n, cudaStream_t stream)
       case kZigzagShard:
       case kZigzagUnshard: jb.seg = m.c; jb.src_step = m.run_bytes; break;
       case kSeq2Head: jb.seg = m.c2; jb.src_step = static_cast<uint64_t>(m.H) * m.row_bytes; break;
+      case kPackHeads: jb.seg = m.S; jb.src_step = static_cast<uint64_t>(m.P_u) * m.run_bytes; break;
+      case kUnpackHeads: jb.seg = m.P_u; jb.src_step = static_cast<uint64_t>(m.B) * m.S * m.run_bytes; break;
+      case kPackTokens:
+      case kUnpackTokens: jb.seg = m.S; jb.src_step = m.run_bytes; break;
       default: jb.seg = m.P_u; jb.src_step = static_cast<uint64_t>(m.B) * m.L * m.run_bytes; break;
     }
     if (jb.nvec >= 32 * kSlots) {

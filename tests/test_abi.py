@@ -166,3 +166,16 @@ def test_dilated_rejects_bad_arguments():
     assert call(ww=zero_w) == B_.USP_ERR_INVALID_ARG
     assert B_.usp_dilated_workspace_size(1, 1024, 4, 128) == 256 + 1024 * 4 * (4 * 128 + 4)
     assert B_.usp_dilated_workspace_size(1, 1024, 4, 96) == 0
+
+
+def test_masked_rejects_unaligned_chunks_and_bad_docs():
+    L = B_.lib()
+    m = B_.AttnMask(FAKE, None, 0)
+    # S=768, P=4: chunks of 96 tokens are not whole tiles
+    rc = L.usp_attn_fwd_masked(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 768, 4, 4, 128, 1, 2, 2, m, FAKE, 256, None)
+    assert rc == B_.USP_ERR_UNSUPPORTED and "128" in B_.usp_last_error()
+    m2 = B_.AttnMask(None, FAKE, 0)
+    rc = L.usp_attn_fwd_masked(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 2, 2, m2, FAKE, 256, None)
+    assert rc == B_.USP_ERR_INVALID_ARG
+    rc = L.usp_attn_bwd_masked(*([FAKE] * 9), 1, 768, 4, 4, 128, 1, 2, 2, m, FAKE, 1 << 30, None)
+    assert rc == B_.USP_ERR_UNSUPPORTED
