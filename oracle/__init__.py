@@ -17,6 +17,10 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
       example (tests/golden/dilated_tiny_closed_form.json), one pair (w = S,
       r = 1) against torch's fp64 scaled_dot_product_attention, and torch's fp64
       SDPA with the log of the key multiplicities as an additive mask.
+  dilated_attn_full (forward and backward) -- pinned: its forward against the
+      pinned dilated_fwd_rows, its gradients against central finite
+      differences and against torch fp64 autograd of SDPA with the
+      key-multiplicity mask.
   masked_fwd_rows / masked_attn_full (block-sparse and document masks) --
       pinned: a hand-derived worked example (tests/golden/masked_tiny_closed_form.json),
       the all-ones mask against the unmasked pinned oracle, torch fp64 SDPA with
@@ -51,6 +55,8 @@ def lib():
         L.oracle_attn_dkdv_cols.argtypes = [P, P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, P, P, P, P, i_]
         L.oracle_lse_merge.argtypes = [l_, l_, l_, P, P, P, P, i_]
         L.oracle_dilated_fwd_rows.argtypes = [P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, l_, P, P, P, i_]
+        L.oracle_dilated_attn_full.argtypes = [P, P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, l_, P, P, P, P, P, P,
+                                               i_]
         L.oracle_masked_fwd_rows.argtypes = [P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, P, l_, P, l_, l_, P, P, P,
                                              i_]
         L.oracle_masked_attn_full.argtypes = [P, P, P, P, i_, l_, l_, l_, l_, l_, i_, d_, P, l_, P, l_, P, P, P,
@@ -62,7 +68,8 @@ def lib():
         for name in ("oracle_attn_fwd_rows", "oracle_attn_full", "oracle_attn_dq_rows",
                      "oracle_attn_dkdv_cols", "oracle_lse_merge", "oracle_zigzag_shard",
                      "oracle_zigzag_unshard", "oracle_seq2head", "oracle_head2seq",
-                     "oracle_dilated_fwd_rows", "oracle_masked_fwd_rows", "oracle_masked_attn_full"):
+                     "oracle_dilated_fwd_rows", "oracle_masked_fwd_rows", "oracle_masked_attn_full",
+                     "oracle_dilated_attn_full"):
             getattr(L, name).restype = ctypes.c_int
         L.oracle_max_threads.restype = ctypes.c_int
         _lib = L
@@ -133,6 +140,23 @@ def dilated_fwd_rows(q, k, v, causal, pairs, rows, scale=None, threads=0):
     if rc != 0:
         raise ValueError(f"oracle_dilated_fwd_rows failed ({rc})")
     return o, lse
+
+
+def dilated_attn_full(q, k, v, do, causal, pairs, scale=None, threads=0):
+    """Whole-tensor LongNet dilated attention forward and backward: dict of
+    float64 o, lse, dq, dk, dv (global layouts)."""
+    B, S, Hq, Hkv, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    (qa, ka, va, da), f64 = _inputs(q, k, v, do)
+    pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    o = np.zeros((B, S, Hq, D)); lse = np.zeros((B, S, Hq)); dq = np.zeros((B, S, Hq, D))
+    dk = np.zeros((B, S, Hkv, D)); dv = np.zeros((B, S, Hkv, D))
+    rc = lib().oracle_dilated_attn_full(_ptr(qa), _ptr(ka), _ptr(va), _ptr(da), f64, B, S, Hq, Hkv, D, int(causal),
+                                        scale, pr.shape[0], _ptr(pr), _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk),
+                                        _ptr(dv), threads)
+    if rc != 0:
+        raise ValueError(f"oracle_dilated_attn_full failed ({rc})")
+    return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv)
 
 
 def _mask_args(block_mask, block, cu_seqlens):

@@ -689,3 +689,102 @@ int oracle_masked_attn_full(const void *q, const void *k, const void *v, const v
     }
     return 0;
 }
+
+/*
+ * LongNet dilated attention, whole-tensor forward AND backward (small shapes).
+ * The forward is that of oracle_dilated_fwd_rows written over the multiset of
+ * keys the pairs show a row: key j counts C_ij times, C_ij = the number of
+ * pairs (w, r) that keep both i and j in one segment (with j <= i if causal);
+ * then O_i = sum_j C_ij e^{s_ij} V_j / sum_j C_ij e^{s_ij} -- the same result as
+ * combining the pairs by their softmax denominators. The backward is the
+ * calculus of that expression: P_ij = C_ij exp(s_ij - LSE_i),
+ * Delta_i = dO_i . O_i, dS_ij = P_ij (dO_i . V_j - Delta_i),
+ * dQ_i = scale sum_j dS_ij K_j, dK_j = scale sum dS_ij Q_i, dV_j = sum P_ij dO_i.
+ * Work is split over (b, kv-head) so that each task owns its dK/dV rows.
+ */
+static long dilated_count(long i, long j, long h, long S, int causal, long n_pairs, const long *pairs) {
+    if (causal && j > i) return 0;
+    long n = 0;
+    for (long p = 0; p < n_pairs; p++) {
+        long w = pairs[2 * p], r = pairs[2 * p + 1], off = h % r;
+        long si = i / w, sj = j / w;
+        if (si != sj) continue;
+        long ri = i - si * w, rj = j - sj * w;
+        if (ri >= off && (ri - off) % r == 0 && rj >= off && (rj - off) % r == 0) n++;
+    }
+    (void)S;
+    return n;
+}
+
+int oracle_dilated_attn_full(const void *q, const void *k, const void *v, const void *dO, int f64,
+                             long B, long S, long Hq, long Hkv, long D, int causal, double scale,
+                             long n_pairs, const long *pairs, double *o, double *lse, double *dq,
+                             double *dk, double *dv, int n_threads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || n_pairs <= 0) return -1;
+    for (long p = 0; p < n_pairs; p++)
+        if (pairs[2 * p] < 1 || pairs[2 * p + 1] < 1) return -1;
+    long G = Hq / Hkv;
+    set_threads(n_threads);
+    memset(dk, 0, sizeof(double) * (size_t)(B * S * Hkv * D));
+    memset(dv, 0, sizeof(double) * (size_t)(B * S * Hkv * D));
+#pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)S);
+        long *cnt = (long *)malloc(sizeof(long) * (size_t)S);
+#pragma omp for schedule(dynamic, 1)
+        for (long bg = 0; bg < B * Hkv; bg++) {
+            long b = bg / Hkv, g = bg % Hkv;
+            for (long hh = 0; hh < G; hh++) {
+                long h = g * G + hh;
+                for (long i = 0; i < S; i++) {
+                    long qi = idx4(b, i, h, 0, S, Hq, D);
+                    double *oi = o + qi, *dqi = dq + qi;
+                    double m = -INFINITY;
+                    for (long j = 0; j < S; j++) {
+                        cnt[j] = dilated_count(i, j, h, S, causal, n_pairs, pairs);
+                        if (!cnt[j]) continue;
+                        long kj = idx4(b, j, g, 0, S, Hkv, D);
+                        double acc = 0.0;
+                        for (long d = 0; d < D; d++) acc += ld(q, qi + d, f64) * ld(k, kj + d, f64);
+                        s_buf[j] = scale * acc;
+                        if (s_buf[j] > m) m = s_buf[j];
+                    }
+                    for (long d = 0; d < D; d++) oi[d] = dqi[d] = 0.0;
+                    if (m == -INFINITY) {
+                        lse[(b * S + i) * Hq + h] = -INFINITY;
+                        continue;
+                    }
+                    double l = 0.0;
+                    for (long j = 0; j < S; j++)
+                        if (cnt[j]) l += (double)cnt[j] * exp(s_buf[j] - m);
+                    double L = m + log(l);
+                    lse[(b * S + i) * Hq + h] = L;
+                    for (long j = 0; j < S; j++) {
+                        if (!cnt[j]) continue;
+                        double p = (double)cnt[j] * exp(s_buf[j] - L);
+                        long vj = idx4(b, j, g, 0, S, Hkv, D);
+                        for (long d = 0; d < D; d++) oi[d] += p * ld(v, vj + d, f64);
+                    }
+                    double delta = 0.0;
+                    for (long d = 0; d < D; d++) delta += ld(dO, qi + d, f64) * oi[d];
+                    for (long j = 0; j < S; j++) {
+                        if (!cnt[j]) continue;
+                        double p = (double)cnt[j] * exp(s_buf[j] - L);
+                        long kj = idx4(b, j, g, 0, S, Hkv, D);
+                        double dp = 0.0;
+                        for (long d = 0; d < D; d++) dp += ld(dO, qi + d, f64) * ld(v, kj + d, f64);
+                        double ds = p * (dp - delta);
+                        for (long d = 0; d < D; d++) {
+                            dqi[d] += scale * ds * ld(k, kj + d, f64);
+                            dk[kj + d] += scale * ds * ld(q, qi + d, f64);
+                            dv[kj + d] += p * ld(dO, qi + d, f64);
+                        }
+                    }
+                }
+            }
+        }
+        free(s_buf);
+        free(cnt);
+    }
+    return 0;
+}

@@ -480,3 +480,53 @@ def test_masked_matches_sdpa_forward_and_autograd(causal, kind):
     np.testing.assert_allclose(m["o"][~e_bsh], on[~e_bsh], rtol=0, atol=1e-12)
     for n, t in (("dq", qr), ("dk", kr), ("dv", vr)):
         np.testing.assert_allclose(m[n], t.grad.numpy(), rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_dilated_full_forward_matches_rows_and_grads_match_autograd(causal):
+    """The whole-tensor dilated oracle: its forward equals the row form (pinned
+    above); its gradients equal torch fp64 autograd of SDPA with the additive
+    log-multiplicity mask."""
+    B, S, Hq, Hkv, D = 1, 24, 4, 2, 8
+    pairs = [(6, 1), (12, 2), (24, 4)]
+    q, k, v, do = (_rand(120 + n, (B, S, h, D)).double() for n, h in enumerate((Hq, Hkv, Hkv, Hq)))
+    full = oracle.dilated_attn_full(q, k, v, do, causal, pairs)
+    rows = _all_rows(B, S, Hq)
+    o_r, l_r = oracle.dilated_fwd_rows(q, k, v, causal, pairs, rows)
+    idx = np.array(rows)
+    np.testing.assert_allclose(full["o"][idx[:, 0], idx[:, 2], idx[:, 1]], o_r, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(full["lse"][idx[:, 0], idx[:, 2], idx[:, 1]], l_r, rtol=0, atol=1e-12)
+    C = _multiplicity_mask(S, Hq, pairs, causal)
+    with np.errstate(divide="ignore"):
+        mask = torch.tensor(np.log(C)).unsqueeze(0)
+    G = Hq // Hkv
+    qr, kr, vr = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = F.scaled_dot_product_attention(qr.transpose(1, 2), kr.repeat_interleave(G, dim=2).transpose(1, 2),
+                                       vr.repeat_interleave(G, dim=2).transpose(1, 2), attn_mask=mask).transpose(1, 2)
+    (o * do).sum().backward()
+    for n, t in (("dq", qr), ("dk", kr), ("dv", vr)):
+        np.testing.assert_allclose(full[n], t.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def test_dilated_full_backward_central_finite_differences():
+    B, S, Hq, Hkv, D = 1, 12, 2, 1, 4
+    pairs = [(4, 1), (12, 3)]
+    q, k, v = (_rand(130 + n, (B, S, h, D)).double() for n, h in enumerate((Hq, Hkv, Hkv)))
+    wgt = _rand(133, (B, S, Hq, D)).double()
+    full = oracle.dilated_attn_full(q, k, v, wgt, True, pairs)
+
+    def loss(q_, k_, v_):
+        return float((oracle.dilated_attn_full(q_, k_, v_, wgt, True, pairs)["o"] * wgt.numpy()).sum())
+
+    h = 1e-6
+    rng = np.random.default_rng(2)
+    for name, t in (("dq", q), ("dk", k), ("dv", v)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(n)) for n in t.shape)
+            tp, tm = t.clone(), t.clone()
+            tp[idx] += h
+            tm[idx] -= h
+            args_p = [tp if x is t else x for x in (q, k, v)]
+            args_m = [tm if x is t else x for x in (q, k, v)]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - full[name][idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, full[name][idx])
