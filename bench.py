@@ -456,6 +456,70 @@ def per_workload(dev, peak_tf, peak_hbm):
         res[f"cfg{cfg}"] = rec
         del rm, hs
         torch.cuda.empty_cache()
+    res.update(variants_per_workload(dev, peak_tf))
+    return res
+
+
+def _time_pair(fwd, bwd, reps=3):
+    ms_f = _time_ms(fwd, reps)
+    ms_b = _time_ms(bwd, reps)
+    return ms_f, ms_b
+
+
+def variants_per_workload(dev, peak_tf):
+    """Event-timed forward and backward of the attention variants on workloads
+    of the pages' shapes: LongNet dilated attention with its segment/dilation
+    schedule (w = 2048..32768, r = 1, 2, 4, 6, 12) on a 32K sequence, and a
+    block-sparse (half the 128 x 128 blocks, seeded) causal attention on the
+    S=16K ring-8 workload. FLOPs are the algorithmic ones of the visible
+    (query, key) pairs: 4*D per pair forward, 2.5x that backward."""
+    from long_context_exact_tma_b200 import api
+    import numpy as np
+    from usp_inputs import normal_bf16
+    res = {}
+    # LongNet dilated attention
+    B, S, H, D = 1, 32768, 16, 128
+    pairs = [(2048, 1), (4096, 2), (8192, 4), (16384, 6), (32768, 12)]
+    q, k, v, do = (normal_bf16(900 + x, (B, S, H, D), device=dev) for x in range(4))
+    vis = 0
+    for w, r in pairs:
+        for h in range(H):
+            kept = (w - h % r + r - 1) // r
+            vis += (S // w) * kept * (kept + 1) // 2
+    fl = 4.0 * D * B * vis
+    o, l = api.dilated_attn_fwd(q, k, v, True, pairs)
+    ms_f, ms_b = _time_pair(lambda: api.dilated_attn_fwd(q, k, v, True, pairs),
+                            lambda: api.dilated_attn_bwd(q, k, v, o, l, do, True, pairs))
+    res["dilated_longnet_s32k"] = {
+        "shape": "B=1 S=32768 H=16 D=128 causal, (w, r) = (2048,1) (4096,2) (8192,4) (16384,6) (32768,12)",
+        "fwd": {"TFLOP/s": round(fl / ms_f / 1e9, 1), "frac_of_peak": round(fl / ms_f / 1e9 / peak_tf, 4),
+                "ms": round(ms_f, 3)},
+        "bwd": {"TFLOP/s": round(2.5 * fl / ms_b / 1e9, 1), "frac_of_peak": round(2.5 * fl / ms_b / 1e9 / peak_tf, 4),
+                "ms": round(ms_b, 3)}}
+    del q, k, v, do, o, l
+    # block-sparse causal attention, S=16K ring 8
+    w = dict(WORKLOADS[2])
+    P_u, P_r = w["P_u"], w["P_r"]
+    t = workload(w, device=dev, which=("q", "k", "v", "do"))
+    qh, kh, vh, doh = (api.to_head_sharded(t[n], P_u, P_r) for n in ("q", "k", "v", "do"))
+    del t
+    nb = w["S"] // 128
+    rng = np.random.default_rng(17)
+    bm = (rng.random((w["B"], w["Hq"], nb, nb)) < 0.5).astype(np.uint8)
+    causal_blocks = np.tril(np.ones((nb, nb), np.int64), -1) * 128 * 128 + np.eye(nb, dtype=np.int64) * (128 * 129 // 2)
+    fl = 4.0 * w["D"] * float((bm.astype(np.int64) * causal_blocks).sum())
+    bmd = torch.tensor(bm, device=dev)
+    o, l = api.attn_fwd_masked(qh, kh, vh, True, P_u, P_r, block_mask=bmd)
+    ms_f, ms_b = _time_pair(lambda: api.attn_fwd_masked(qh, kh, vh, True, P_u, P_r, block_mask=bmd),
+                            lambda: api.attn_bwd_masked(qh, kh, vh, o, l, doh, True, P_u, P_r, block_mask=bmd))
+    res["block_sparse_s16k_ring8"] = {
+        "shape": "the S=16K ring-8 workload with a seeded half-dense 128x128 block mask, causal",
+        "fwd": {"TFLOP/s": round(fl / ms_f / 1e9, 1), "frac_of_peak": round(fl / ms_f / 1e9 / peak_tf, 4),
+                "ms": round(ms_f, 3)},
+        "bwd": {"TFLOP/s": round(2.5 * fl / ms_b / 1e9, 1), "frac_of_peak": round(2.5 * fl / ms_b / 1e9 / peak_tf, 4),
+                "ms": round(ms_b, 3)}}
+    del qh, kh, vh, doh, o, l, bmd
+    torch.cuda.empty_cache()
     return res
 
 

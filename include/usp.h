@@ -354,6 +354,24 @@ int usp_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
  */
 #define USP_DILATED_MAX_PAIRS 16
 size_t usp_dilated_workspace_size(int B, int S, int Hq, int D);
+/*
+ * usp_dilated_attn_bwd: the backward of usp_dilated_attn_fwd. With the final
+ * (merged) LSE and Delta_i = dO_i . O_i, every pair contributes at its kept
+ * rows the attention backward of its segments -- P_ij = exp(s_ij - LSE_i),
+ * dS_ij = P_ij (dO_i . V_j - Delta_i), dQ = scale dS K, dK = scale dS^T Q,
+ * dV = P^T dO -- and the pairs' contributions are summed (a key shown to a
+ * query by two pairs counts twice, as in the forward).
+ *   out, lse   the forward's outputs;  dO [B][S][Hq][D] bf16
+ *   dQ         [B][S][Hq][D] bf16;  dK, dV [B][S][Hkv][D] fp32 (overwritten)
+ *   workspace  usp_dilated_bwd_workspace_size(B, S, Hq, D, n_pairs, w, r)
+ *              bytes (status, Delta of every row, an fp32 dQ, the row tables
+ *              of the largest launch); 0 for an unsupported shape.
+ */
+size_t usp_dilated_bwd_workspace_size(int B, int S, int Hq, int D, int n_pairs, const int* w, const int* r);
+int usp_dilated_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                         const void* dO, void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv, int D,
+                         int causal, int n_pairs, const int* w, const int* r, void* workspace, size_t ws_bytes,
+                         void* stream);
 int usp_dilated_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int S, int Hq,
                          int Hkv, int D, int causal, int n_pairs, const int* w, const int* r, void* workspace,
                          size_t ws_bytes, void* stream);

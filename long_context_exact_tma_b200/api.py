@@ -224,6 +224,22 @@ def dilated_attn_fwd(q, k, v, causal: bool, pairs, ws=None, out=None, lse=None, 
     return out, lse
 
 
+def dilated_attn_bwd(q, k, v, out, lse, dO, causal: bool, pairs, ws=None, stream=None, check_status: bool = False):
+    """Backward of dilated_attn_fwd; returns (dQ bf16 like q, dK fp32 like k, dV fp32 like v)."""
+    _require_cuda(q, k, v, out, lse, dO)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if ws is None:
+        ws = workspace(B_.usp_dilated_bwd_workspace_size(B, S, Hq, D, pairs), q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=k.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=v.device)
+    B_.usp_dilated_attn_bwd(q, k, v, out, lse, dO, dq, dk, dv, B, S, Hq, Hkv, D, causal, pairs, ws, ws.numel(), stream)
+    if check_status:
+        check_workspace(ws, stream)
+    return dq, dk, dv
+
+
 def lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out_dtype=torch.bfloat16, stream=None):
     """o_parts [n, rows, D] fp32, lse_parts [n, rows] fp32 -> (out [rows, D], lse [rows])."""
     _require_cuda(o_parts, lse_parts)

@@ -70,6 +70,8 @@ SIGNATURES = {
     "usp_ring_bwd_step": (_I, [_P] * 8 + [_I] * 11 + [_P, _SZ, _P]),
     "usp_dilated_workspace_size": (_SZ, [_I] * 4),
     "usp_dilated_attn_fwd": (_I, [_P] * 5 + [_I] * 7 + [_P, _P, _P, _SZ, _P]),
+    "usp_dilated_bwd_workspace_size": (_SZ, [_I] * 5 + [_P, _P]),
+    "usp_dilated_attn_bwd": (_I, [_P] * 9 + [_I] * 7 + [_P, _P, _P, _SZ, _P]),
     "usp_attn_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_P, _SZ, _P]),
     "usp_attn_bwd": (_I, [_P] * 9 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_fwd_masked": (_I, [_P] * 5 + [_I] * 8 + [ctypes.POINTER(AttnMask), _P, _SZ, _P]),
@@ -225,6 +227,26 @@ def usp_dilated_attn_fwd(q, k, v, out, lse, B, S, Hq, Hkv, D, causal, pairs, wor
     r = (ctypes.c_int * max(n, 1))(*[int(p[1]) for p in pairs])
     rc = lib().usp_dilated_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, Hq, Hkv, D, int(causal),
                                     n, w, r, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def _pairs(pairs):
+    n = len(pairs)
+    return (n, (ctypes.c_int * max(n, 1))(*[int(p[0]) for p in pairs]),
+            (ctypes.c_int * max(n, 1))(*[int(p[1]) for p in pairs]))
+
+
+def usp_dilated_bwd_workspace_size(B, S, Hq, D, pairs) -> int:
+    n, w, r = _pairs(pairs)
+    return int(lib().usp_dilated_bwd_workspace_size(B, S, Hq, D, n, w, r))
+
+
+def usp_dilated_attn_bwd(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, causal, pairs, workspace, ws_bytes,
+                         stream=None, check=True):
+    n, w, r = _pairs(pairs)
+    rc = lib().usp_dilated_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
+                                    _ptr(dV), B, S, Hq, Hkv, D, int(causal), n, w, r, _ptr(workspace), ws_bytes,
+                                    _stream(stream))
     return _check(rc) if check else rc
 
 

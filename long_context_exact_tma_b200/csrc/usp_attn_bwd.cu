@@ -69,6 +69,7 @@ struct BwdArgs {
   int* status;
   unsigned long long wait_ns;
   int loc_i, loc_u, loc_j;  // local mode: query rank (i, u), KV block of ring rank j
+  FwdSub sub;               // sub-problem mode (dilated attention): see usp_internal.h
 };
 
 struct BwdBars {
@@ -94,10 +95,11 @@ struct QWalk {
   bool valid;
 };
 
+template <bool kPlain = false>
 __device__ __forceinline__ int classify_q(const Geo& g, int i, int m, int kmin, int kmax) {
   const int q0 = m * kBM;
   int qmin, qmax;
-  pos_range(g, i, q0, q0 + kBM, qmin, qmax);
+  pos_range<kPlain>(g, i, q0, q0 + kBM, qmin, qmax);
   // Padded query columns need no mask: their LSE is +inf, so P = 0 there.
   if (g.causal && qmax < kmin) return kSkip;
   if (!g.causal || qmin >= kmax) return kFull;
@@ -119,14 +121,20 @@ struct MaskedQ {
 
 // Steps t in [t_lo, t_hi) of the walk: all ring ranks i = (j + t) mod P_r, or
 // in the local mode the one rank that computes.
-template <bool kMask>
+// In the sub-problem mode (kPlain) only the q-heads of the group that belong to
+// the launch (hbase + hh congruent to hoff mod hstep) are walked.
+template <bool kMask, bool kPlain = false>
 __device__ __forceinline__ void qwalk_settle(const Geo& g, int j, int kmin, int kmax, QWalk& w, const MaskedQ& mq,
-                                             int t_lo, int t_hi) {
+                                             int t_lo, int t_hi, int hbase = 0, int hoff = 0, int hstep = 1) {
   while (w.hh < g.G) {
+    if (kPlain && (hbase + w.hh - hoff) % hstep != 0) {
+      ++w.hh;
+      continue;
+    }
     while (w.t < t_hi) {
       w.i = (j + w.t) % g.P_r;
       while (w.m < g.n_qtiles) {
-        w.kind = kMask ? mq(w.hh, w.i, w.m) : classify_q(g, w.i, w.m, kmin, kmax);
+        w.kind = kMask ? mq(w.hh, w.i, w.m) : classify_q<kPlain>(g, w.i, w.m, kmin, kmax);
         if (w.kind != kSkip) {
           w.valid = true;
           return;
@@ -142,30 +150,37 @@ __device__ __forceinline__ void qwalk_settle(const Geo& g, int j, int kmin, int 
   w.valid = false;
 }
 
-template <bool kMask>
+template <bool kMask, bool kPlain = false>
 __device__ __forceinline__ QWalk qwalk_begin(const Geo& g, int j, int kmin, int kmax, const MaskedQ& mq, int t_lo,
-                                             int t_hi) {
+                                             int t_hi, int hbase = 0, int hoff = 0, int hstep = 1) {
   QWalk w{0, t_lo, 0, 0, 0, false};
-  qwalk_settle<kMask>(g, j, kmin, kmax, w, mq, t_lo, t_hi);
+  qwalk_settle<kMask, kPlain>(g, j, kmin, kmax, w, mq, t_lo, t_hi, hbase, hoff, hstep);
   return w;
 }
 
-template <bool kMask>
+template <bool kMask, bool kPlain = false>
 __device__ __forceinline__ void qwalk_next(const Geo& g, int j, int kmin, int kmax, QWalk& w, const MaskedQ& mq,
-                                           int t_lo, int t_hi) {
+                                           int t_lo, int t_hi, int hbase = 0, int hoff = 0, int hstep = 1) {
   ++w.m;
-  qwalk_settle<kMask>(g, j, kmin, kmax, w, mq, t_lo, t_hi);
+  qwalk_settle<kMask, kPlain>(g, j, kmin, kmax, w, mq, t_lo, t_hi, hbase, hoff, hstep);
 }
 
-// kLocal: ONE rank of a real multi-GPU mesh -- the KV block of ring rank loc_j
-// it holds (its own buffers, [B][L][Hkv/P_u][D]) against the queries of rank
-// (loc_i, loc_u) only; dK and dV are ADDED to the given fp32 buffers (the
-// gradients travelling with the block around the ring).
-template <int D, bool kMask, bool kLocal>
+enum : int { kModeUsp = 0, kModeSub = 1, kModeLocal = 2 };
+
+// kMode: kModeUsp -- every virtual rank of the mesh; kModeLocal -- ONE rank of a
+// real multi-GPU mesh: the KV block of ring rank loc_j it holds (its own
+// buffers, [B][L][Hkv/P_u][D]) against the queries of rank (loc_i, loc_u) only,
+// dK and dV ADDED to the given fp32 buffers (the gradients travelling with the
+// block around the ring); kModeSub -- the one-rank problems of a dilated
+// attention launch (a (w, r) pair and head offset; strided tensor maps), dK and
+// dV ADDED at the kept rows' original positions.
+template <int D, bool kMask, int kMode>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdArgs a) {
+  constexpr bool kLocal = kMode == kModeLocal;
+  constexpr bool kSub = kMode == kModeSub;
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_addr(smem_raw) & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -186,8 +201,15 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
   // Work item: CTAs of one (b, Ulysses rank, kv-head) run together; inside it,
   // key tiles in increasing original position (the causally heaviest first).
-  int gl, u, b, j, n;
-  if constexpr (kLocal) {
+  int gl, u, b, j, n, prob = 0;
+  if constexpr (kSub) {  // work item: (problem, kv-head, key tile)
+    int wi = blockIdx.x;
+    n = wi % g.n_ktiles;
+    wi /= g.n_ktiles;
+    gl = wi % g.Hkv_l;
+    prob = wi / g.Hkv_l;
+    u = b = j = 0;
+  } else if constexpr (kLocal) {
     int wi = blockIdx.x;
     n = wi % g.n_ktiles;
     wi /= g.n_ktiles;
@@ -206,13 +228,13 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     b = wi / g.P_u;
     tile_in_position_order(g, order, j, n);
   }
-  const int jrank = kLocal ? 0 : j * g.P_u + u;  // local buffers hold one rank
+  const int jrank = (kLocal || kSub) ? 0 : j * g.P_u + u;  // local buffers hold one rank
   // ring steps walked: every rank's queries, or those of the one local rank
   const int t_lo = kLocal ? (a.loc_i - j + g.P_r) % g.P_r : 0;
   const int t_hi = kLocal ? t_lo + 1 : g.P_r;
   const int k0 = n * kBN;
   int kmin, kmax;
-  pos_range(g, j, k0, k0 + kBN, kmin, kmax);
+  pos_range<kSub>(g, j, k0, k0 + kBN, kmin, kmax);
 
   if (threadIdx.x == 0) {
     bars->abort_flag = *reinterpret_cast<volatile int*>(a.status) != 0;
@@ -252,7 +274,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         tma_prefetch_desc(&tm_do);
       }
       __syncwarp();
-      const int krb = jrank * g.B + b;
+      const int krb = kSub ? prob : jrank * g.B + b;
       mbar_expect_tx_w(&bars->kv_full, 2 * C::kTileBytes);
       for (int p = 0; p < C::kPanels; ++p) {
         tma_load_4d_w(&tm_k, &bars->kv_full, sK + p * C::kPanelBytes, p * 64, gl, k0, krb);
@@ -260,7 +282,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       }
       int issued = 0;
       const MaskedQ mq{g, b, u, gl, kmin, kmax};
-      QWalk qw = qwalk_begin<kMask>(g, j, kmin, kmax, mq, t_lo, t_hi);
+      // sub-problem mode: the launch's q-heads are a.sub.h0 + k * a.sub.h_step
+      QWalk qw = qwalk_begin<kMask, kSub>(g, j, kmin, kmax, mq, t_lo, t_hi, gl * g.G, a.sub.h0, a.sub.h_step);
       while (true) {
         const int s = issued % C::kStages;
         if (issued >= C::kStages &&
@@ -281,7 +304,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         }
         __syncwarp();
         const int h = gl * g.G + qw.hh;
-        const int qrb = kLocal ? b : (qw.i * g.P_u + u) * g.B + b;
+        const int qrb = kSub ? prob : kLocal ? b : (qw.i * g.P_u + u) * g.B + b;
         const int q0 = qw.m * kBM;
         mbar_expect_tx_w(&bars->qd_full[s], 2 * C::kTileBytes + 1024);
         for (int p = 0; p < C::kPanels; ++p) {
@@ -289,11 +312,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           tma_load_4d_w(&tm_do, &bars->qd_full[s], sDO + s * C::kTileBytes + p * C::kPanelBytes, p * 64, h, q0,
                         qrb);
         }
-        const size_t rowbase = (static_cast<size_t>(qrb) * g.Hq_l + h) * a.Lp + q0;
+        // row tables: per (rank, head), or per (problem, launch head) in the sub-problem mode
+        const size_t rowbase =
+            kSub ? (static_cast<size_t>(prob) * a.sub.n_heads + (h - a.sub.h0) / a.sub.h_step) * a.Lp + q0
+                 : (static_cast<size_t>(qrb) * g.Hq_l + h) * a.Lp + q0;
         bulk_load_1d_w(sRow + s * 256, a.lse2 + rowbase, 512, &bars->qd_full[s]);
         bulk_load_1d_w(sRow + s * 256 + 128, a.delta + rowbase, 512, &bars->qd_full[s]);
         ++issued;
-        qwalk_next<kMask>(g, j, kmin, kmax, qw, mq, t_lo, t_hi);
+        qwalk_next<kMask, kSub>(g, j, kmin, kmax, qw, mq, t_lo, t_hi, gl * g.G, a.sub.h0, a.sub.h_step);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         mbar_wait_drain(&bars->kv_full, 0, a.wait_ns);
@@ -391,7 +417,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     const int row = wq * 32 + lane;  // key row of S^T/dP^T/dK/dV; query row of the dQ tile
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const int tau_k = k0 + row;
-    const int pos_k = tau_k < g.L ? token_pos(g, j, tau_k) : INT_MAX;  // padding keys see no query
+    const int pos_k = tau_k < g.L ? token_pos<kSub>(g, j, tau_k) : INT_MAX;  // padding keys see no query
     int doc_lo = 0, doc_hi = INT_MAX;  // the key's document [lo, hi) (masked variant)
     if constexpr (kMask) doc_span(g.mask, pos_k, doc_lo, doc_hi);
     const bool aligned = (g.c % kBM) == 0;
@@ -415,11 +441,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       if (st_kind == kMasked) {
         // causal: rewrite S^T of this key row to -inf where the query does not see
         // the key, so the main pass carries no masking (P = 0 there)
-        int lo = pos_k == INT_MAX ? kBM : pos_k - token_pos(g, st_i, q0);  // aligned: cols >= lo see it
+        int lo = pos_k == INT_MAX ? kBM : pos_k - token_pos<kSub>(g, st_i, q0);  // aligned: cols >= lo see it
         int hi_c = kBM;                                                      // and cols < hi_c
         if constexpr (kMask) {
           // masked variant (tiles contiguous): the key's document bounds the columns too
-          const int qpos0 = token_pos(g, st_i, q0);
+          const int qpos0 = token_pos<kSub>(g, st_i, q0);
           if (!g.causal && pos_k != INT_MAX) lo = 0;
           if (pos_k != INT_MAX) {
             lo = max(lo, doc_lo - qpos0);
@@ -441,7 +467,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             vis = 0u;
             for (int c = 0; c < 32; ++c) {
               const int tq = q0 + c0 + c;
-              if (tq < g.L && pos_k <= token_pos(g, st_i, tq)) vis |= 1u << c;
+              if (tq < g.L && pos_k <= token_pos<kSub>(g, st_i, tq)) vis |= 1u << c;
             }
           }
           uint32_t r[32];
@@ -516,7 +542,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     if (ok) {
       tc_fence_after();
       const bool store = tau_k < g.L;
-      const size_t kr = (static_cast<size_t>(jrank * g.B + b) * g.L + (store ? tau_k : 0)) * g.Hkv_l + gl;
+      size_t kr;
+      if constexpr (kSub) {  // the key's original position in [B][S][Hkv]
+        const int pb = prob / a.sub.n_seg, ps = prob % a.sub.n_seg;
+        kr = (static_cast<size_t>(pb) * a.sub.S + static_cast<size_t>(ps) * a.sub.w + a.sub.off +
+              static_cast<size_t>(store ? tau_k : 0) * a.sub.r) * g.Hkv_l + gl;
+      } else {
+        kr = (static_cast<size_t>(jrank * g.B + b) * g.L + (store ? tau_k : 0)) * g.Hkv_l + gl;
+      }
       // warpgroup wg writes columns [wg*D/2, wg*D/2 + D/2)
 #pragma unroll
       for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
@@ -540,7 +573,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
                                     __uint_as_float(rk[4 * q + 2]) * g.scale, __uint_as_float(rk[4 * q + 3]) * g.scale);
             float4 nv = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
                                     __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
-            if constexpr (kLocal) {  // add to the gradients travelling with the block
+            if constexpr (kLocal || kSub) {  // add (travelling ring gradients; the pairs' sum)
               const float4 ok_ = dkp[q], ov = dvp[q];
               nk = make_float4(nk.x + ok_.x, nk.y + ok_.y, nk.z + ok_.z, nk.w + ok_.w);
               nv = make_float4(nv.x + ov.x, nv.y + ov.y, nv.z + ov.z, nv.w + ov.w);
@@ -561,11 +594,13 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   }
 }
 
-template <int D, bool kMask, bool kLocal>
+template <int D, bool kMask, int kMode>
 cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
+  constexpr bool kLocal = kMode == kModeLocal;
+  constexpr bool kSub = kMode == kModeSub;
   using C = BwdCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, kMask, kLocal>,
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, kMask, kMode>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   BwdArgs a{};
@@ -581,11 +616,19 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   a.loc_i = L.loc_i;
   a.loc_u = L.loc_u;
   a.loc_j = L.loc_j;
-  const long long blocks = kLocal ? static_cast<long long>(a.g.n_ktiles) * a.g.B * a.g.Hkv_l
-                                  : static_cast<long long>(a.g.n_ktiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hkv_l;
+  a.sub = L.sub;
+  if (kSub) {  // one-rank geometry of every problem (see the forward's sub-problem mode)
+    a.g.P_u = a.g.P_r = a.g.P = a.g.n_ranks = 1;
+    a.g.L = L.sub.L;
+    a.g.c = kBN;
+    a.g.n_qtiles = a.g.n_ktiles = (L.sub.L + kBM - 1) / kBM;
+  }
+  const long long blocks = kSub     ? static_cast<long long>(a.g.n_ktiles) * a.g.Hkv_l * L.sub.n_prob
+                           : kLocal ? static_cast<long long>(a.g.n_ktiles) * a.g.B * a.g.Hkv_l
+                                    : static_cast<long long>(a.g.n_ktiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hkv_l;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  attn_bwd_kernel<D, kMask, kLocal><<<static_cast<unsigned>(blocks), kThreadsBwd, C::kSmemBytes, stream>>>(
+  attn_bwd_kernel<D, kMask, kMode><<<static_cast<unsigned>(blocks), kThreadsBwd, C::kSmemBytes, stream>>>(
       L.tm_q, L.tm_k, L.tm_v, L.tm_do, a);
   note_launch();
   return cudaGetLastError();
@@ -595,19 +638,24 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
 
 cudaError_t launch_attn_bwd(const BwdLaunch& L, cudaStream_t stream) {
   const bool masked = L.mask.bm != nullptr || L.mask.cu != nullptr;
-  if (masked && L.local) return cudaErrorInvalidValue;
+  if (masked && (L.local || L.sub.active)) return cudaErrorInvalidValue;
+  if (L.sub.active) {
+    if (L.g.D == 128) return launch_bwd_d<128, false, kModeSub>(L, stream);
+    if (L.g.D == 64) return launch_bwd_d<64, false, kModeSub>(L, stream);
+    return cudaErrorInvalidValue;
+  }
   if (L.local) {
-    if (L.g.D == 128) return launch_bwd_d<128, false, true>(L, stream);
-    if (L.g.D == 64) return launch_bwd_d<64, false, true>(L, stream);
+    if (L.g.D == 128) return launch_bwd_d<128, false, kModeLocal>(L, stream);
+    if (L.g.D == 64) return launch_bwd_d<64, false, kModeLocal>(L, stream);
     return cudaErrorInvalidValue;
   }
   if (masked) {
-    if (L.g.D == 128) return launch_bwd_d<128, true, false>(L, stream);
-    if (L.g.D == 64) return launch_bwd_d<64, true, false>(L, stream);
+    if (L.g.D == 128) return launch_bwd_d<128, true, kModeUsp>(L, stream);
+    if (L.g.D == 64) return launch_bwd_d<64, true, kModeUsp>(L, stream);
     return cudaErrorInvalidValue;
   }
-  if (L.g.D == 128) return launch_bwd_d<128, false, false>(L, stream);
-  if (L.g.D == 64) return launch_bwd_d<64, false, false>(L, stream);
+  if (L.g.D == 128) return launch_bwd_d<128, false, kModeUsp>(L, stream);
+  if (L.g.D == 64) return launch_bwd_d<64, false, kModeUsp>(L, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -63,6 +63,7 @@ struct DqArgs {
   __nv_bfloat16* dq;    // bf16 [n_ranks][B][L][Hq_l][D]
   float* dq_acc;        // local mode: fp32 [B][L][Hq_l][D], this step's dQ is added to it
   int loc_i, loc_u, loc_t;  // local mode: the rank (i, u) and its ring step t
+  FwdSub sub;               // sub-problem mode (dilated attention): see usp_internal.h
   int* status;
   unsigned long long wait_ns;
 };
@@ -87,11 +88,18 @@ enum : int {
 // kLocal: ONE rank (loc_i, loc_u) of a real multi-GPU mesh at ring step loc_t:
 // its own Q and dO against the KV block it holds (owner (i - t) mod P_r), its
 // own buffers ([B][L][H/P_u][D]); dQ is ADDED to the fp32 dq_acc.
-template <int D, bool kMask, bool kLocal>
+enum : int { kModeUsp = 0, kModeSub = 1, kModeLocal = 2 };
+
+// kModeSub: the one-rank problems of a dilated attention launch (a (w, r) pair
+// and head offset, strided tensor maps); dQ is ADDED to the fp32 dq_acc at the
+// kept rows' original positions.
+template <int D, bool kMask, int kMode>
 __global__ void __launch_bounds__(kThreadsDq, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const DqArgs a) {
+  constexpr bool kLocal = kMode == kModeLocal;
+  constexpr bool kSub = kMode == kModeSub;
   using C = DqCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_addr(smem_raw) & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -111,8 +119,15 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
 
   // Work item: CTAs of one (b, Ulysses rank, head) run together so that its K/V
   // stay in L2; inside it, query tiles in decreasing original position.
-  int h, u, b, i, m;
-  if constexpr (kLocal) {
+  int h, u, b, i, m, prob = 0;
+  if constexpr (kSub) {  // work item: (problem, launch head, query tile), heaviest first
+    int wi = blockIdx.x;
+    m = g.n_qtiles - 1 - wi % g.n_qtiles;
+    wi /= g.n_qtiles;
+    h = a.sub.h0 + (wi % a.sub.n_heads) * a.sub.h_step;
+    prob = wi / a.sub.n_heads;
+    u = b = i = 0;
+  } else if constexpr (kLocal) {
     int wi = blockIdx.x;
     m = g.n_qtiles - 1 - wi % g.n_qtiles;
     wi /= g.n_qtiles;
@@ -131,7 +146,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     b = wi / g.P_u;
     tile_in_position_order(g, order, i, m);
   }
-  const int rank = kLocal ? 0 : i * g.P_u + u;  // local buffers hold one rank
+  const int rank = (kLocal || kSub) ? 0 : i * g.P_u + u;  // local buffers hold one rank
   // ring steps walked: all of them, or the local rank's one step
   const int t_lo = kLocal ? a.loc_t : 0;
   const int t_hi = kLocal ? a.loc_t + 1 : g.P_r;
@@ -175,7 +190,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     // elected lane issues each copy and barrier operation.
     {
       int qmin, qmax;
-      pos_range(g, i, q0, q0 + kBM, qmin, qmax);
+      pos_range<kSub>(g, i, q0, q0 + kBM, qmin, qmax);
       // masked variant: the causal kind narrowed by the block / document masks
       auto kind_of = [&](int j, int n) {
         int kmin, kmax;
@@ -186,7 +201,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       if constexpr (kMask)
         kw = kv_walk_begin_by(g, i, t_lo, t_hi, kind_of);
       else
-        kw = kv_walk_begin(g, i, qmin, qmax, t_lo, t_hi);
+        kw = kv_walk_begin<kSub>(g, i, qmin, qmax, t_lo, t_hi);
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -194,7 +209,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
         tma_prefetch_desc(&tm_do);
       }
       __syncwarp();
-      const int qrb = rank * g.B + b;
+      const int qrb = kSub ? prob : rank * g.B + b;
       mbar_expect_tx_w(&bars->q_full, 2 * C::kTileBytes);
       for (int p = 0; p < C::kPanels; ++p) {
         tma_load_4d_w(&tm_q, &bars->q_full, sQ + p * C::kPanelBytes, p * 64, h, q0, qrb);
@@ -221,7 +236,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
           slot[3] = kw.kind;
         }
         __syncwarp();
-        const int krb = kLocal ? b : (kw.j * g.P_u + u) * g.B + b;
+        const int krb = kSub ? prob : kLocal ? b : (kw.j * g.P_u + u) * g.B + b;
         mbar_expect_tx_w(&bars->k_full[sk], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_4d_w(&tm_k, &bars->k_full[sk], sK + sk * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
@@ -238,7 +253,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
         if constexpr (kMask)
           kv_walk_next_by(g, i, t_hi, kw, kind_of);
         else
-          kv_walk_next(g, i, qmin, qmax, t_hi, kw);
+          kv_walk_next<kSub>(g, i, qmin, qmax, t_hi, kw);
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         // Let every copy this warp started land before the CTA exits.
@@ -353,11 +368,14 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const int cbase = wg * 64;
     const int tau_q = q0 + row;
-    const int pos_q = tau_q < g.L ? token_pos(g, i, tau_q) : INT_MAX;
+    const int pos_q = tau_q < g.L ? token_pos<kSub>(g, i, tau_q) : INT_MAX;
     const bool aligned = (g.c % kBN) == 0;
     int doc_lo = 0, doc_hi = INT_MAX;  // the row's document [lo, hi) (masked variant)
     if constexpr (kMask) doc_span(g.mask, pos_q, doc_lo, doc_hi);
-    const size_t tab = (static_cast<size_t>(rank * g.B + b) * g.Hq_l + h) * a.Lp + tau_q;
+    // row tables: per (rank, head), or per (problem, launch head) in the sub-problem mode
+    const size_t tab =
+        kSub ? (static_cast<size_t>(prob) * a.sub.n_heads + (h - a.sub.h0) / a.sub.h_step) * a.Lp + tau_q
+             : (static_cast<size_t>(rank * g.B + b) * g.Hq_l + h) * a.Lp + tau_q;
     const float nl = __ldg(a.nlse2 + tab);   // -inf on padding rows: their P is 0
     const float nd = __ldg(a.ndelta + tab);
     const float2 sl2 = make_float2(g.scale_log2, g.scale_log2);
@@ -380,10 +398,10 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
         // rewrite the scores this query does not see to -inf (P = 0 there)
         const int k0 = kn * kBN;
         int lim = min(127, g.L - k0 - 1);  // keys at or past L are padding
-        if (aligned && g.causal) lim = min(lim, pos_q - token_pos(g, kj, k0));
+        if (aligned && g.causal) lim = min(lim, pos_q - token_pos<kSub>(g, kj, k0));
         int first = 0;  // first visible column (documents: keys from the row's document start)
         if constexpr (kMask) {
-          const int kpos0 = token_pos(g, kj, k0);  // tiles are contiguous under a mask
+          const int kpos0 = token_pos<kSub>(g, kj, k0);  // tiles are contiguous under a mask
           if (doc_hi != INT_MAX) lim = min(lim, doc_hi - 1 - kpos0);
           first = max(0, doc_lo - kpos0);
         }
@@ -402,7 +420,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
             vis = 0u;
             for (int c = 0; c < 32; ++c) {
               const int tau = k0 + c0 + c;
-              if (tau < g.L && (!g.causal || token_pos(g, kj, tau) <= pos_q)) vis |= 1u << c;
+              if (tau < g.L && (!g.causal || token_pos<kSub>(g, kj, tau) <= pos_q)) vis |= 1u << c;
             }
           }
           uint32_t r[32];
@@ -451,7 +469,14 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     if (ok) {
       tc_fence_after();
       const bool store = tau_q < g.L;
-      const size_t qr = (static_cast<size_t>(rank * g.B + b) * g.L + (store ? tau_q : 0)) * g.Hq_l + h;
+      size_t qr;
+      if constexpr (kSub) {  // the query's original position in [B][S][Hq]
+        const int pb = prob / a.sub.n_seg, ps = prob % a.sub.n_seg;
+        qr = (static_cast<size_t>(pb) * a.sub.S + static_cast<size_t>(ps) * a.sub.w + a.sub.off +
+              static_cast<size_t>(store ? tau_q : 0) * a.sub.r) * a.sub.Hq + h;
+      } else {
+        qr = (static_cast<size_t>(rank * g.B + b) * g.L + (store ? tau_q : 0)) * g.Hq_l + h;
+      }
 #pragma unroll
       for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
         uint32_t o[32];
@@ -463,7 +488,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = 0u;
         }
-        if (store && kLocal) {
+        if (store && (kLocal || kSub)) {
           // add this step's dQ to the fp32 accumulator; on the last step (a bf16
           // output given) write the sum as bf16 instead
           const float4* acc = reinterpret_cast<const float4*>(a.dq_acc + qr * D + c0);
@@ -517,11 +542,13 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
   }
 }
 
-template <int D, bool kMask, bool kLocal>
+template <int D, bool kMask, int kMode>
 cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
+  constexpr bool kLocal = kMode == kModeLocal;
+  constexpr bool kSub = kMode == kModeSub;
   using C = DqCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kMask, kLocal>,
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kMask, kMode>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   DqArgs a{};
@@ -537,11 +564,19 @@ cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
   a.loc_t = L.loc_t;
   a.status = L.status;
   a.wait_ns = L.wait_ns;
-  const long long blocks = kLocal ? static_cast<long long>(a.g.n_qtiles) * a.g.B * a.g.Hq_l
-                                  : static_cast<long long>(a.g.n_qtiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;
+  a.sub = L.sub;
+  if (kSub) {  // one-rank geometry of every problem (see the forward's sub-problem mode)
+    a.g.P_u = a.g.P_r = a.g.P = a.g.n_ranks = 1;
+    a.g.L = L.sub.L;
+    a.g.c = kBN;
+    a.g.n_qtiles = a.g.n_ktiles = (L.sub.L + kBM - 1) / kBM;
+  }
+  const long long blocks = kSub     ? static_cast<long long>(a.g.n_qtiles) * L.sub.n_heads * L.sub.n_prob
+                           : kLocal ? static_cast<long long>(a.g.n_qtiles) * a.g.B * a.g.Hq_l
+                                    : static_cast<long long>(a.g.n_qtiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  attn_bwd_dq_kernel<D, kMask, kLocal><<<static_cast<unsigned>(blocks), kThreadsDq, C::kSmemBytes, stream>>>(
+  attn_bwd_dq_kernel<D, kMask, kMode><<<static_cast<unsigned>(blocks), kThreadsDq, C::kSmemBytes, stream>>>(
       L.tm_q, L.tm_k, L.tm_v, L.tm_do, a);
   note_launch();
   return cudaGetLastError();
@@ -551,19 +586,24 @@ cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
 
 cudaError_t launch_attn_bwd_dq(const BwdLaunch& L, cudaStream_t stream) {
   const bool masked = L.mask.bm != nullptr || L.mask.cu != nullptr;
-  if (masked && L.local) return cudaErrorInvalidValue;
+  if (masked && (L.local || L.sub.active)) return cudaErrorInvalidValue;
+  if (L.sub.active) {
+    if (L.g.D == 128) return launch_dq_d<128, false, kModeSub>(L, stream);
+    if (L.g.D == 64) return launch_dq_d<64, false, kModeSub>(L, stream);
+    return cudaErrorInvalidValue;
+  }
   if (L.local) {
-    if (L.g.D == 128) return launch_dq_d<128, false, true>(L, stream);
-    if (L.g.D == 64) return launch_dq_d<64, false, true>(L, stream);
+    if (L.g.D == 128) return launch_dq_d<128, false, kModeLocal>(L, stream);
+    if (L.g.D == 64) return launch_dq_d<64, false, kModeLocal>(L, stream);
     return cudaErrorInvalidValue;
   }
   if (masked) {
-    if (L.g.D == 128) return launch_dq_d<128, true, false>(L, stream);
-    if (L.g.D == 64) return launch_dq_d<64, true, false>(L, stream);
+    if (L.g.D == 128) return launch_dq_d<128, true, kModeUsp>(L, stream);
+    if (L.g.D == 64) return launch_dq_d<64, true, kModeUsp>(L, stream);
     return cudaErrorInvalidValue;
   }
-  if (L.g.D == 128) return launch_dq_d<128, false, false>(L, stream);
-  if (L.g.D == 64) return launch_dq_d<64, false, false>(L, stream);
+  if (L.g.D == 128) return launch_dq_d<128, false, kModeUsp>(L, stream);
+  if (L.g.D == 64) return launch_dq_d<64, false, kModeUsp>(L, stream);
   return cudaErrorInvalidValue;
 }
 

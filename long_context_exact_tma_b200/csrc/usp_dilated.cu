@@ -114,3 +114,158 @@ extern "C" int usp_dilated_attn_fwd(const void* q, const void* k, const void* v,
   if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "final merge launch: %s", cudaGetErrorString(e));
   return USP_OK;
 }
+
+// ---------------------------------------------------------------- backward
+//
+// The gradient of the pairs' combination: with the FINAL merged LSE and
+// Delta_i = dO_i . O_i of every row, each pair contributes, at its kept rows,
+// P_ij = exp(s_ij - LSE_i), dS_ij = P_ij (dO_i . V_j - Delta_i) -- the
+// standard attention backward of that pair's sub-problems with the final
+// LSE -- and the contributions of all pairs are summed. One launch of the
+// key-major (dK, dV) and of the query-major (dQ) kernel per (pair, head
+// offset), over the same strided tensor maps as the forward; dK and dV are
+// accumulated in place (fp32), dQ in an fp32 workspace converted to bf16 last.
+namespace {
+
+using usp::record_error;
+
+struct DilatedLaunchShape {
+  int kept, n_seg, n_heads;
+};
+
+DilatedLaunchShape launch_shape(int S, int Hq, int w, int r, int off) {
+  return DilatedLaunchShape{(w - off + r - 1) / r, S / w, (Hq - off + r - 1) / r};
+}
+
+size_t dilated_bwd_ws(int B, int S, int Hq, int D, int n_pairs, const int* w, const int* r, size_t* tbl_floats) {
+  size_t tbl = 0;  // the largest per-launch table: n_prob * n_heads * Lp floats
+  for (int p = 0; p < n_pairs; ++p)
+    for (int off = 0; off < r[p] && off < Hq; ++off) {
+      const DilatedLaunchShape sh = launch_shape(S, Hq, w[p], r[p], off);
+      const size_t Lp = static_cast<size_t>((sh.kept + 127) / 128 * 128);
+      const size_t n = static_cast<size_t>(B) * sh.n_seg * sh.n_heads * Lp;
+      if (n > tbl) tbl = n;
+    }
+  if (tbl_floats) *tbl_floats = tbl;
+  const size_t rows = static_cast<size_t>(B) * S * Hq;
+  // status | Delta of every row | fp32 dQ | two row tables
+  return usp::kStatusBytes + rows * 4 + rows * D * 4 + 2 * tbl * 4;
+}
+
+int check_pairs(int S, int n_pairs, const int* w, const int* r) {
+  if (!w || !r) return record_error(USP_ERR_INVALID_ARG, "null pair arrays");
+  if (n_pairs < 1 || n_pairs > USP_DILATED_MAX_PAIRS)
+    return record_error(USP_ERR_INVALID_ARG, "n_pairs must be 1..%d", USP_DILATED_MAX_PAIRS);
+  for (int p = 0; p < n_pairs; ++p) {
+    if (w[p] < 1 || r[p] < 1) return record_error(USP_ERR_INVALID_ARG, "pair %d: w and r must be positive", p);
+    if (S % w[p] != 0) return record_error(USP_ERR_UNSUPPORTED, "pair %d: S (%d) is not a multiple of w (%d)", p, S, w[p]);
+    if (r[p] > w[p]) return record_error(USP_ERR_UNSUPPORTED, "pair %d: r (%d) exceeds w (%d)", p, r[p], w[p]);
+  }
+  return USP_OK;
+}
+
+}  // namespace
+
+extern "C" size_t usp_dilated_bwd_workspace_size(int B, int S, int Hq, int D, int n_pairs, const int* w,
+                                                 const int* r) {
+  if (B <= 0 || S <= 0 || Hq <= 0 || (D != 64 && D != 128)) return 0;
+  if (!w || !r || n_pairs < 1 || n_pairs > USP_DILATED_MAX_PAIRS) return 0;
+  for (int p = 0; p < n_pairs; ++p)
+    if (w[p] < 1 || r[p] < 1 || r[p] > w[p] || S % w[p] != 0) return 0;
+  return dilated_bwd_ws(B, S, Hq, D, n_pairs, w, r, nullptr);
+}
+
+extern "C" int usp_dilated_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                                    const void* dO, void* dQ, float* dK, float* dV, int B, int S, int Hq, int Hkv,
+                                    int D, int causal, int n_pairs, const int* w, const int* r, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0) return record_error(USP_ERR_INVALID_ARG, "sizes must be positive");
+  if (causal != 0 && causal != 1) return record_error(USP_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (D != 64 && D != 128) return record_error(USP_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", D);
+  if (Hq % Hkv != 0) return record_error(USP_ERR_UNSUPPORTED, "Hq %% Hkv != 0");
+  if (static_cast<long long>(B) * S * Hq >= (1LL << 31)) return record_error(USP_ERR_UNSUPPORTED, "too many rows");
+  int rc = check_pairs(S, n_pairs, w, r);
+  if (rc != USP_OK) return rc;
+  if (!q || !k || !v || !out || !lse || !dO || !dQ || !dK || !dV)
+    return record_error(USP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return record_error(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  size_t tbl = 0;
+  const size_t need = dilated_bwd_ws(B, S, Hq, D, n_pairs, w, r, &tbl);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return record_error(USP_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long rows = static_cast<long long>(B) * S * Hq;
+  const long long kv_elems = static_cast<long long>(B) * S * Hkv * D;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  float* delta_all = reinterpret_cast<float*>(base + usp::kStatusBytes);
+  float* dq_acc = delta_all + rows;
+  float* lse2_t = dq_acc + rows * D;
+  float* delta_t = lse2_t + tbl;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dq_acc, 0, rows * D * sizeof(float), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dK, 0, kv_elems * sizeof(float), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, kv_elems * sizeof(float), st);
+  if (e == cudaSuccess) e = usp::launch_bwd_preprocess(out, dO, delta_all, rows, D, st);
+  if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated backward init: %s", cudaGetErrorString(e));
+
+  usp::BwdLaunch L{};
+  usp::AttnGeom& g = L.g;
+  g.B = B; g.S = S; g.Hq = Hq; g.Hkv = Hkv; g.D = D; g.causal = causal;
+  g.P_u = g.P_r = g.P = g.n_ranks = 1;
+  g.G = Hq / Hkv;
+  g.Hq_l = Hq;
+  g.Hkv_l = Hkv;
+  L.status = static_cast<int*>(workspace);
+  L.wait_ns = usp::current_wait_ns();
+  L.lse2 = lse2_t;
+  L.delta = delta_t;
+  L.dk = dK;
+  L.dv = dV;
+  L.dq = nullptr;
+  L.dq_acc = dq_acc;
+  const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;
+  for (int p = 0; p < n_pairs; ++p) {
+    const int wp = w[p], rp = r[p];
+    for (int off = 0; off < rp && off < Hq; ++off) {
+      const DilatedLaunchShape sh = launch_shape(S, Hq, wp, rp, off);
+      usp::FwdSub& sb = L.sub;
+      sb.active = 1;
+      sb.n_prob = B * sh.n_seg;
+      sb.L = sh.kept;
+      sb.h0 = off;
+      sb.h_step = rp;
+      sb.n_heads = sh.n_heads;
+      sb.n_seg = sh.n_seg;
+      sb.w = wp;
+      sb.off = off;
+      sb.r = rp;
+      sb.S = S;
+      sb.Hq = Hq;
+      g.L = sh.kept;
+      g.c = sh.kept;
+      L.Lp = (sh.kept + 127) / 128 * 128;
+      rc = usp::make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, sh.kept, sb.n_prob,
+                                  rp * tokq, wp * tokq);
+      if (rc == USP_OK)
+        rc = usp::make_tmap_strided(&L.tm_do, static_cast<const uint8_t*>(dO) + off * tokq, D, Hq, sh.kept,
+                                    sb.n_prob, rp * tokq, wp * tokq);
+      if (rc == USP_OK)
+        rc = usp::make_tmap_strided(&L.tm_k, static_cast<const uint8_t*>(k) + off * tokkv, D, Hkv, sh.kept,
+                                    sb.n_prob, rp * tokkv, wp * tokkv);
+      if (rc == USP_OK)
+        rc = usp::make_tmap_strided(&L.tm_v, static_cast<const uint8_t*>(v) + off * tokkv, D, Hkv, sh.kept,
+                                    sb.n_prob, rp * tokkv, wp * tokkv);
+      if (rc != USP_OK) return rc;
+      e = usp::launch_dilated_tables(lse, delta_all, lse2_t, delta_t, sb, L.Lp, st);
+      if (e == cudaSuccess) e = usp::launch_attn_bwd(L, st);
+      if (e == cudaSuccess) e = usp::launch_attn_bwd_dq(L, st);
+      if (e != cudaSuccess)
+        return record_error(USP_ERR_CUDA, "dilated backward launch: %s", cudaGetErrorString(e));
+    }
+  }
+  e = usp::launch_f32_to_bf16(dq_acc, dQ, rows * D, st);
+  if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dQ conversion: %s", cudaGetErrorString(e));
+  return USP_OK;
+}

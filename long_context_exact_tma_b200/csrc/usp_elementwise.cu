@@ -208,6 +208,49 @@ __global__ void __launch_bounds__(256) fill_running_kernel(float4* __restrict__ 
     lse[x] = -INFINITY;
 }
 
+// Row tables of one dilated-attention backward launch: for problem p (batch
+// p / n_seg, segment p % n_seg), launch head jh (query head h0 + jh * h_step) and
+// kept row tau < kept (position (p % n_seg) * w + off + tau * r), the
+// -LSE*log2(e) and -Delta of that row, at [(p * n_heads + jh) * Lp + tau];
+// padding rows (tau >= kept) get -inf and 0.
+__global__ void __launch_bounds__(256) dilated_tables_kernel(const float* __restrict__ lse,
+                                                             const float* __restrict__ delta_all,
+                                                             float* __restrict__ lse2_t, float* __restrict__ delta_t,
+                                                             long long n, int Lp, int kept, int n_heads, int h0,
+                                                             int h_step, int n_seg, int w, int off, int r, int S,
+                                                             int Hq) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += stride) {
+    const int tau = static_cast<int>(e % Lp);
+    const long long pj = e / Lp;
+    const int jh = static_cast<int>(pj % n_heads);
+    const long long p = pj / n_heads;
+    if (tau >= kept) {
+      lse2_t[e] = -INFINITY;
+      delta_t[e] = 0.f;
+      continue;
+    }
+    const long long row = ((p / n_seg) * S + (p % n_seg) * w + off + static_cast<long long>(tau) * r) * Hq +
+                          h0 + static_cast<long long>(jh) * h_step;
+    const float l = lse[row];
+    lse2_t[e] = l == -INFINITY ? -INFINITY : -l * 1.4426950408889634f;
+    delta_t[e] = -delta_all[row];
+  }
+}
+
+// fp32 -> bf16, n elements (n a multiple of 4, both 16-byte aligned).
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ x, uint2* __restrict__ y,
+                                                          long long n4) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n4; e += stride) {
+    const float4 v = __ldcs(x + e);
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    y[e] = o;
+  }
+}
+
 // Waits on an mbarrier that nothing completes; the bounded wait must give up.
 __global__ void wait_selftest_kernel(int* status, unsigned long long limit_ns) {
   __shared__ uint64_t bar;
@@ -288,6 +331,26 @@ cudaError_t launch_fill_running(float* o, float* lse, long long rows, int D, cud
   if (rows == 0) return cudaSuccess;
   const long long n4 = rows * D / 4;
   fill_running_kernel<<<grid_for(256 * 4, n4), 256, 0, stream>>>(reinterpret_cast<float4*>(o), lse, n4, rows);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dilated_tables(const float* lse, const float* delta_all, float* lse2_t, float* delta_t,
+                                  const FwdSub& sb, int Lp, cudaStream_t stream) {
+  const long long n = static_cast<long long>(sb.n_prob) * sb.n_heads * Lp;
+  if (n == 0) return cudaSuccess;
+  dilated_tables_kernel<<<grid_for(256, n), 256, 0, stream>>>(lse, delta_all, lse2_t, delta_t, n, Lp, sb.L,
+                                                              sb.n_heads, sb.h0, sb.h_step, sb.n_seg, sb.w, sb.off,
+                                                              sb.r, sb.S, sb.Hq);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float* x, void* y, long long n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const long long n4 = n / 4;
+  f32_to_bf16_kernel<<<grid_for(256, n4), 256, 0, stream>>>(reinterpret_cast<const float4*>(x),
+                                                            static_cast<uint2*>(y), n4);
   note_launch();
   return cudaGetLastError();
 }

@@ -115,6 +115,14 @@ cudaError_t launch_attn_fwd(const FwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* lse, float* delta_t, float* lse2_t,
                                  int n_rb, int L, int Hl, int D, int Lp, cudaStream_t stream);
 
+// Row tables (-LSE*log2(e), -Delta) of one dilated-attention backward launch,
+// gathered from the final LSE and Delta of every row ([B*S*Hq]); see
+// usp_elementwise.cu.
+cudaError_t launch_dilated_tables(const float* lse, const float* delta_all, float* lse2_t, float* delta_t,
+                                  const FwdSub& sb, int Lp, cudaStream_t stream);
+// fp32 -> bf16 of n elements (n % 4 == 0, 16-byte aligned).
+cudaError_t launch_f32_to_bf16(const float* x, void* y, long long n, cudaStream_t stream);
+
 struct BwdLaunch {
   AttnGeom g;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
@@ -131,7 +139,8 @@ struct BwdLaunch {
   // KV block belongs to ring rank loc_j = (loc_i - loc_t) mod P_r; its own buffers
   // (B in dim 4); dK, dV and the fp32 dq_acc are accumulated into
   int local, loc_i, loc_u, loc_t, loc_j;
-  float* dq_acc;
+  float* dq_acc;       // local and sub-problem modes: fp32 dQ accumulator
+  FwdSub sub;          // sub-problem mode (dilated attention) when sub.active
 };
 cudaError_t launch_attn_bwd(const BwdLaunch& a, cudaStream_t stream);     // dK, dV (key-major)
 cudaError_t launch_attn_bwd_dq(const BwdLaunch& a, cudaStream_t stream);  // dQ (query-major)

@@ -76,3 +76,26 @@ def test_dilated_two_calls_reuse_workspace(cuda):
     o1, l1 = api.dilated_attn_fwd(q, k, v, causal, pairs, ws=ws)
     o2, l2 = api.dilated_attn_fwd(q, k, v, causal, pairs, ws=ws, check_status=True)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+BWD_CASES = {
+    # name: (B, S, Hq, Hkv, D, causal, pairs) -- whole-tensor oracle in seconds
+    "longnet_scaled_s768": (1, 768, 4, 4, 128, True, [(64, 1), (128, 2), (256, 4), (384, 6), (768, 12)]),
+    "noncausal_gqa_d64": (2, 512, 8, 2, 64, False, [(128, 1), (256, 3), (512, 8)]),
+    "tiny_segments_gqa": (1, 384, 4, 2, 128, True, [(96, 1), (192, 5), (384, 7)]),
+}
+
+
+@pytest.mark.parametrize("name", list(BWD_CASES))
+def test_dilated_backward_full_tensors(cuda, name):
+    from helpers import GRAD_REL_L2, GRAD_STATS, rel_l2
+    B, S, Hq, Hkv, D, causal, pairs = BWD_CASES[name]
+    q, k, v = _inputs(B, S, Hq, Hkv, D, 770 + len(name), cuda)
+    do = normal_bf16(790 + len(name), (B, S, Hq, D), device=cuda)
+    o, lse = api.dilated_attn_fwd(q, k, v, causal, pairs, check_status=True)
+    dq, dk, dv = api.dilated_attn_bwd(q, k, v, o, lse, do, causal, pairs, check_status=True)
+    torch.cuda.synchronize()
+    ref = oracle.dilated_attn_full(q.cpu(), k.cpu(), v.cpu(), do.cpu(), causal, pairs)
+    errs = {n: rel_l2(g.double().cpu().numpy(), ref[n]) for n, g in (("dq", dq), ("dk", dk), ("dv", dv))}
+    GRAD_STATS.append((f"dilated/{name}", errs))
+    assert all(e <= GRAD_REL_L2 for e in errs.values()), errs

@@ -45,6 +45,7 @@ def test_ulysses_pack_around_all_to_all_bit_exact(cuda):
                 s = torch.empty((G, B, T, Hl, D), dtype=dt, device=cuda)
                 B_.usp_ulysses_pack(B_.USP_MAP_PACK_HEADS, [(rm[i * P_u + u], s, H, D, _dt(s))], B, T, G)
                 sends.append(s)
+            backs = []
             for u in range(P_u):
                 recv = torch.stack([sends[up][u] for up in range(P_u)])  # the all-to-all
                 got = torch.empty((B, G * T, Hl, D), dtype=dt, device=cuda)
@@ -53,9 +54,9 @@ def test_ulysses_pack_around_all_to_all_bit_exact(cuda):
                 # and back: pack tokens, all-to-all, unpack heads
                 back_s = torch.empty((G, B, T, Hl, D), dtype=dt, device=cuda)
                 B_.usp_ulysses_pack(B_.USP_MAP_PACK_TOKENS, [(got, back_s, H, D, _dt(got))], B, T, G)
-                sends[u] = back_s
+                backs.append(back_s)
             for u in range(P_u):
-                recv = torch.stack([sends[up][u] for up in range(P_u)])
+                recv = torch.stack([backs[up][u] for up in range(P_u)])
                 out = torch.empty((B, T, H, D), dtype=dt, device=cuda)
                 B_.usp_ulysses_pack(B_.USP_MAP_UNPACK_HEADS, [(recv, out, H, D, _dt(out))], B, T, G)
                 assert torch.equal(out, rm[i * P_u + u])
