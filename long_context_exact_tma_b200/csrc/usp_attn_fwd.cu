@@ -11,16 +11,21 @@
 // step and writes the fp32 partial (O_t, LSE_t) for usp_lse_merge.
 //
 // CTA = two consecutive 128-row query tiles of one (rank, batch, head) that
-// share every K/V tile (320 threads):
-//   warp 0      TMA producer: Q0, Q1 once, then K and V tiles into a kStages ring;
-//               it alone walks the key tiles and publishes one descriptor per tile.
+// share every K/V tile (352 threads):
+//   warp 0      TMA producer of Q0, Q1 (once) and of the K tiles (3 stages); it
+//               walks the key tiles and publishes one descriptor per tile.
+//   warp 10     TMA producer of the V tiles of the same walk (2 stages at D=128).
+//               A K stage is released when both S of its tile have completed, a
+//               V stage when both PV have: K runs ahead of the S it feeds instead
+//               of waiting behind the previous tile's PV.
 //   warp 1      TMEM allocator and UMMA issuer (one thread), per key tile and
 //               query tile t = 0, 1 in turn:
 //                 O_t += P_t V    (M=128 N=D; A = P_t read from TMEM)
 //                 S_t  = Q_t K^T  of the next key tile (M=128 N=128, fp32 in TMEM;
 //                                 it overwrites P_t, so it waits for that PV)
 //               so the tensor core runs tile 1's PV and S while softmax 0 works
-//               and the other way round.
+//               and the other way round. Before each S_t it hands that tile's
+//               descriptor to softmax t (desc_full[t]).
 //   warps 2..5  softmax of tile 0, warps 6..9 softmax of tile 1: thread = query
 //               row = TMEM lane. tcgen05.ld of S, mask by original positions,
 //               online max/sum in the exp2 domain with lazy rescaling of O (only
@@ -39,7 +44,8 @@
 namespace usp {
 namespace {
 
-constexpr int kThreadsFwd = 320;
+constexpr int kThreadsFwd = 352;
+constexpr int kWarpV = 10;  // V producer
 enum : int { kModeUsp = 0, kModeSub = 1, kModeLocal = 2 };
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThresh = 8.0f;  // log2 units: rescale O only if the max grows by > 256x
@@ -52,12 +58,13 @@ struct FwdCfg {
   static constexpr int kPanels = D / 64;          // 128-byte (64 x bf16) swizzle panels along D
   static constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes
   static constexpr int kTileBytes = kPanels * kPanelBytes;
-  static constexpr int kStages = D == 128 ? 2 : 3;
+  static constexpr int kKSt = 3;                  // K stages
+  static constexpr int kVSt = D == 128 ? 2 : 3;   // V stages
   static constexpr int kOffQ = 0;                 // two query tiles
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr int kOffV = kOffK + kKSt * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVSt * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 320 + 1024;
 };
 
 struct FwdArgs {
@@ -75,21 +82,24 @@ struct FwdArgs {
 
 struct FwdBars {
   uint64_t q_full;
-  uint64_t k_full[3], v_full[3], kv_empty[3];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
+  uint64_t s_full[2], p_full[2], pv_done[2], desc_full[2];
   uint64_t drain;
   // Key-tile descriptors published by the producer with k_full of that tile:
   // {1, or -1 = no more tiles; ring rank j of the key owner; key tile n;
   //  kind for query tile 0 | kind for query tile 1 << 4}.
   int step[4][4];
+  // The descriptor of the tile whose S the MMA warp issues next for query tile
+  // t, handed to that tile's softmax warps with desc_full[t].
+  int sdesc[2][4];
   uint32_t tmem_base;
   int abort_flag;
 };
 
 // Wait-site codes recorded in the status word: 0x100 | role << 4 | which.
 enum : int {
-  kSiteQ = 0x101, kSiteKvEmpty = 0x102, kSiteK = 0x111, kSitePvDone = 0x112, kSiteP = 0x113, kSiteV = 0x114,
-  kSiteS = 0x121, kSiteO = 0x122, kSiteKs = 0x123
+  kSiteQ = 0x101, kSiteKEmpty = 0x102, kSiteVEmpty = 0x103, kSiteK = 0x111, kSitePvDone = 0x112, kSiteP = 0x113,
+  kSiteV = 0x114, kSiteS = 0x121, kSiteO = 0x122, kSiteDesc = 0x123
 };
 
 // The pair of consecutive query tiles (i, m, m+1) handled by CTA-order index o
@@ -120,7 +130,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::kOffBar);
-  static_assert(sizeof(FwdBars) <= 256, "barrier block");
+  static_assert(sizeof(FwdBars) <= 320, "barrier block");
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
@@ -177,15 +187,17 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     // A CTA that starts after another one gave up does no work at all.
     bars->abort_flag = *reinterpret_cast<volatile int*>(a.status) != 0;
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], 4);  // one arrival per softmax warp
       mbar_init(&bars->pv_done[t], 1);
+      mbar_init(&bars->desc_full[t], 1);
     }
     mbar_init(&bars->drain, 1);
     fence_mbar_init();
@@ -200,11 +212,16 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
 
   if (skip) {
     // nothing issued, nothing to drain
-  } else if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    // The whole warp walks the tiles (the same values in every lane); one elected
-    // lane issues each copy and barrier operation.
+  } else if (warp == 0 || warp == kWarpV) {
+    // ------------------------------------------------------------ TMA producers
+    // Warp 0 loads Q0, Q1 and the K tiles and publishes one descriptor per key
+    // tile; warp kWarpV loads the V tiles of the same walk. K and V have their
+    // own rings: a K stage is released as soon as both S of its tile have
+    // completed, a V stage only after both PV, so K runs up to kKSt tiles ahead
+    // of the S it feeds. The whole warp walks the tiles (the same values in
+    // every lane); one elected lane issues each copy and barrier operation.
     {
+      const bool kside = warp == 0;
       int qmin0, qmax0, qmin1, qmax1;
       pos_range<kSub>(g, i, q0, q0 + kBM, qmin0, qmax0);
       pos_range<kSub>(g, i, q0 + kBM, q0 + 2 * kBM, qmin1, qmax1);
@@ -227,50 +244,54 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         kw = kv_walk_begin<kSub>(g, i, qmin, qmax, t_begin, t_end);
       int issued = 0;
       const bool any = kw.valid;
+      const int n_st = kside ? C::kKSt : C::kVSt;
+      uint64_t* full = kside ? bars->k_full : bars->v_full;
+      uint64_t* empty = kside ? bars->k_empty : bars->v_empty;
+      const CUtensorMap* tm = kside ? &tm_k : &tm_v;
+      uint8_t* sbuf = kside ? sK : sV;
       if (any) {
         if (lane == 0) {
-          tma_prefetch_desc(&tm_q);
-          tma_prefetch_desc(&tm_k);
-          tma_prefetch_desc(&tm_v);
+          if (kside) tma_prefetch_desc(&tm_q);
+          tma_prefetch_desc(tm);
         }
         __syncwarp();
-        mbar_expect_tx_w(&bars->q_full, 2 * C::kTileBytes);
-        for (int t = 0; t < 2; ++t)
-          for (int p = 0; p < C::kPanels; ++p)
-            tma_load_4d_w(&tm_q, &bars->q_full, sQ + t * C::kTileBytes + p * C::kPanelBytes, p * 64, h,
-                          q0 + t * kBM, kSub ? qc4 : rank * g.B + b);
+        if (kside) {
+          mbar_expect_tx_w(&bars->q_full, 2 * C::kTileBytes);
+          for (int t = 0; t < 2; ++t)
+            for (int p = 0; p < C::kPanels; ++p)
+              tma_load_4d_w(&tm_q, &bars->q_full, sQ + t * C::kTileBytes + p * C::kPanelBytes, p * 64, h,
+                            q0 + t * kBM, kSub ? qc4 : rank * g.B + b);
+        }
       }
       while (true) {
-        const int s = issued % C::kStages;
-        if (issued >= C::kStages &&
-            !mbar_wait_w(&bars->kv_empty[s], ((issued / C::kStages) - 1) & 1, w, kSiteKvEmpty))
+        const int s = issued % n_st;
+        if (!kside && !kw.valid) break;
+        if (issued >= n_st &&
+            !mbar_wait_w(&empty[s], ((issued / n_st) - 1) & 1, w, kside ? kSiteKEmpty : kSiteVEmpty))
           break;
-        int* slot = bars->step[issued & 3];
-        if (!kw.valid) {  // publish the end of the walk on this stage's barrier
-          if (lane == 0) slot[0] = -1;
+        if (kside) {
+          int* slot = bars->step[issued & 3];
+          if (!kw.valid) {  // publish the end of the walk on this stage's barrier
+            if (lane == 0) slot[0] = -1;
+            __syncwarp();
+            mbar_arrive_w(&full[s]);
+            break;
+          }
+          const int kinds = kMask ? kw.kind
+                                  : classify_tile<kSub>(g, qmin0, qmax0, kw.j, kw.n) |
+                                        (classify_tile<kSub>(g, qmin1, qmax1, kw.j, kw.n) << 4);
+          if (lane == 0) {
+            slot[0] = 1;
+            slot[1] = kw.j;
+            slot[2] = kw.n;
+            slot[3] = kinds;
+          }
           __syncwarp();
-          mbar_arrive_w(&bars->k_full[s]);
-          break;
         }
-        const int kinds = kMask ? kw.kind
-                                : classify_tile<kSub>(g, qmin0, qmax0, kw.j, kw.n) |
-                                      (classify_tile<kSub>(g, qmin1, qmax1, kw.j, kw.n) << 4);
-        if (lane == 0) {
-          slot[0] = 1;
-          slot[1] = kw.j;
-          slot[2] = kw.n;
-          slot[3] = kinds;
-        }
-        __syncwarp();
         const int krb = kSub ? qc4 : kLocal ? b : (kw.j * g.P_u + u) * g.B + b;
-        mbar_expect_tx_w(&bars->k_full[s], C::kTileBytes);
+        mbar_expect_tx_w(&full[s], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_4d_w(&tm_k, &bars->k_full[s], sK + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
-                        kw.n * kBN, krb);
-        mbar_expect_tx_w(&bars->v_full[s], C::kTileBytes);
-        for (int p = 0; p < C::kPanels; ++p)
-          tma_load_4d_w(&tm_v, &bars->v_full[s], sV + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh,
-                        kw.n * kBN, krb);
+          tma_load_4d_w(tm, &full[s], sbuf + s * C::kTileBytes + p * C::kPanelBytes, p * 64, kvh, kw.n * kBN, krb);
         ++issued;
         if constexpr (kMask)
           kv_walk_next_by(g, i, t_end, kw, kinds_of);
@@ -279,11 +300,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       }
       if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) {
         // Let every copy this warp started land before the CTA exits.
-        if (any) mbar_wait_drain(&bars->q_full, 0, a.wait_ns);
-        for (int it = issued - C::kStages < 0 ? 0 : issued - C::kStages; it < issued; ++it) {
-          mbar_wait_drain(&bars->k_full[it % C::kStages], (it / C::kStages) & 1, a.wait_ns);
-          mbar_wait_drain(&bars->v_full[it % C::kStages], (it / C::kStages) & 1, a.wait_ns);
-        }
+        if (any && kside) mbar_wait_drain(&bars->q_full, 0, a.wait_ns);
+        for (int it = issued - n_st < 0 ? 0 : issued - n_st; it < issued; ++it)
+          mbar_wait_drain(&full[it % n_st], (it / n_st) & 1, a.wait_ns);
       }
     }
     __syncwarp();
@@ -307,23 +326,45 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         }
         umma_commit_w(&bars->s_full[t]);
       };
+      // Hands the descriptor of key-tile slot `slot` (or the end of the walk) to
+      // the softmax warps of query tile t.
+      auto publish = [&](int t, const int* slot) {
+        if (lane == 0) {
+          int* sd = bars->sdesc[t];
+          sd[0] = slot ? slot[0] : -1;
+          if (slot) {
+            sd[1] = slot[1];
+            sd[2] = slot[2];
+            sd[3] = slot[3];
+          }
+        }
+        __syncwarp();
+        mbar_arrive_w(&bars->desc_full[t]);
+      };
       bool ok = mbar_wait_w(&bars->k_full[0], 0, w, kSiteK);
       const bool have = ok && bars->step[0][0] >= 0;
       bool issued_any = false;
+      if (ok && !have) {
+        publish(0, nullptr);
+        publish(1, nullptr);
+      }
       if (have) ok = mbar_wait_w(&bars->q_full, 0, w, kSiteQ);
       if (ok && have) {
         tc_fence_after();
+        publish(0, bars->step[0]);
+        publish(1, bars->step[0]);
         issue_s(0, 0);
         issue_s(1, 0);
+        umma_commit_w(&bars->k_empty[0]);
         issued_any = true;
       }
       // Per key tile `it`, per query tile t in turn: O_t += P_t V, then S_t of
       // tile it+1 (which overwrites P_t, so it waits for that PV to land). The
       // softmax of one query tile thus overlaps the other tile's PV and S.
       for (int it = 0; ok && have; ++it) {
-        const int s = it % C::kStages;
-        const int s1 = (it + 1) % C::kStages;
-        if (!mbar_wait_w(&bars->v_full[s], (it / C::kStages) & 1, w, kSiteV)) { ok = false; break; }
+        const int s = it % C::kVSt;
+        const int s1 = (it + 1) % C::kKSt;
+        if (!mbar_wait_w(&bars->v_full[s], (it / C::kVSt) & 1, w, kSiteV)) { ok = false; break; }
         const uint64_t vd = dV0 + ((s * C::kTileBytes) >> 4);
         bool next = false;
         for (int t = 0; t < 2 && ok; ++t) {
@@ -334,15 +375,19 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
             umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
                                (it > 0 || kk > 0) ? 1u : 0u);
           umma_commit_w(&bars->pv_done[t]);
-          if (t == 1) umma_commit_w(&bars->kv_empty[s]);
+          if (t == 1) umma_commit_w(&bars->v_empty[s]);
           if (t == 0) {
-            if (!mbar_wait_w(&bars->k_full[s1], ((it + 1) / C::kStages) & 1, w, kSiteK)) { ok = false; break; }
+            if (!mbar_wait_w(&bars->k_full[s1], ((it + 1) / C::kKSt) & 1, w, kSiteK)) { ok = false; break; }
             next = bars->step[(it + 1) & 3][0] >= 0;
           }
           if (next) {
             if (!mbar_wait_w(&bars->pv_done[t], it & 1, w, kSitePvDone)) { ok = false; break; }
             tc_fence_after();
+            publish(t, bars->step[(it + 1) & 3]);
             issue_s(t, s1);
+            if (t == 1) umma_commit_w(&bars->k_empty[s1]);
+          } else {
+            publish(t, nullptr);
           }
         }
         if (!ok || !next) break;
@@ -372,9 +417,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     int it = 0;
     bool ok = true;
     for (;; ++it) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->k_full[it % C::kStages], (it / C::kStages) & 1, w, kSiteKs));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->desc_full[t], it & 1, w, kSiteDesc));
       if (!ok) break;
-      const int* slot = bars->step[it & 3];
+      const int* slot = bars->sdesc[t];
       if (slot[0] < 0) break;
       const int kj = slot[1], kn = slot[2], kkind = (slot[3] >> (4 * t)) & 15;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], it & 1, w, kSiteS));
@@ -472,7 +517,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], pv);
           pk[c >> 1] = pack_bf16x2(pv.x, pv.y);
-          accb[(c >> 1) & 3] = fadd2(accb[(c >> 1) & 3], bf16x2_unpack(pk[c >> 1]));
+          accb[(c >> 1) & 3] = add_bf16x2_f32(accb[(c >> 1) & 3], pk[c >> 1]);
         }
         tmem_st16(trow + cS + col, pk);
       };
