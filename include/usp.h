@@ -377,6 +377,95 @@ int usp_dilated_attn_fwd(const void* q, const void* k, const void* v, void* out,
                          size_t ws_bytes, void* stream);
 
 /*
+ * usp_rows_copy: up to USP_MAX_ROWS_JOBS affine row copies in one launch, the
+ * data movement around the LongNet collectives below (packing the kept rows of
+ * a rank before an all-gather, compacting the gathered blocks, and the reverse
+ * for the reduce-scatter of their gradients). Job x copies, for b < n_b,
+ * k < n_k, j < n_j, one row of D elements
+ *   src[b * s_b + (s_k0 + k * s_kstep) * s_k + ((s_h0 + j * s_hstep) / s_hdiv) * s_h]
+ *   -> dst[b * d_b + (d_k0 + k * d_kstep) * d_k + ((d_h0 + j * d_hstep) / d_hdiv) * d_h]
+ * (strides in elements), assigning, or adding when `add` (USP_F32 only; the
+ * rows of one (b, k) are added in j order, so several j may share a
+ * destination row). dtype USP_BF16 or USP_F32 for both sides; D * element size
+ * a multiple of 16 bytes and every row 16-byte aligned. Different jobs of one
+ * call must not write the same destination row. USP_ERR_INVALID_ARG otherwise.
+ */
+#define USP_MAX_ROWS_JOBS 16
+typedef struct {
+  const void* src;
+  void* dst;
+  int dtype;
+  int add;
+  int n_b, n_k, n_j, D;
+  long long s_b, s_k, s_h;
+  int s_k0, s_kstep, s_h0, s_hstep, s_hdiv;
+  long long d_b, d_k, d_h;
+  int d_k0, d_kstep, d_h0, d_hstep, d_hdiv;
+} usp_rows_job;
+int usp_rows_copy(const usp_rows_job* jobs, int n_jobs, void* stream);
+
+/*
+ * LongNet's distributed layout, per rank (LongNet slides, "LONGNET as a
+ * Distributed Trainer": a segment no longer than a device's slice is computed
+ * locally; a longer one has its key/value rows brought together by an
+ * all-gather, and the local queries attend those global rows; in the backward
+ * the all-gather becomes a reduce-scatter). The sequence of S tokens is split
+ * into M contiguous slices of T = S / M tokens, rank d holding positions
+ * [d*T, (d+1)*T) of q [B][T][Hq][D], k, v [B][T][Hkv][D] (bf16). Each (w, r)
+ * pair of usp_dilated_attn_fwd is then either
+ *   local     w <= T (T % w == 0): usp_longnet_fwd_local / _bwd_local, the
+ *             dilated attention of the rank's own segments;
+ *   gathered  w > T (w % T == 0): the segment spans G = w / T ranks; the rank
+ *             is number g = d mod G in it. For every head offset o < min(r, Hq)
+ *             the query heads o, o + r, ... (n_sel of them) keep the segment
+ *             rows at positions = o (mod r). usp_longnet_rows gives this rank's
+ *             share of those rows: the first kept local row lp0, its index k_lo
+ *             among the segment's kept rows, their count n_rows (local rows
+ *             lp0, lp0 + r, ...), and the segment's total n_kept. The caller
+ *             packs the rank's kept K/V rows of the kv heads of those query
+ *             heads (usp_rows_copy), all-gathers them over the segment's G
+ *             ranks, compacts them in kept order into kc, vc
+ *             [B][n_kept][n_sel][D] bf16 (head j = the kv head of query head
+ *             o + j r) and calls usp_longnet_fwd_cross: the rank's n_rows
+ *             kept query rows (kept indices k_lo ...) against all n_kept rows,
+ *             causal by kept index.
+ * Every call folds into a running fp32 (O, LSE) in the workspace
+ * (usp_longnet_fwd_begin resets it, usp_longnet_fwd_end writes out [B][T][Hq][D]
+ * bf16 and lse [B][T][Hq] fp32 with the pairs combined as in
+ * usp_dilated_attn_fwd), so the rank's result equals rows [d*T, (d+1)*T) of
+ * usp_dilated_attn_fwd on the whole sequence.
+ * Backward: usp_longnet_bwd_begin (Delta of every row; dQ accumulator, dK and
+ * dV zeroed) with the final out and lse; per local pair usp_longnet_bwd_local
+ * (adds to dK, dV [B][T][Hkv][D] fp32); per gathered (pair, offset)
+ * usp_longnet_bwd_cross with the same kc, vc: writes this rank's queries'
+ * contribution to the gathered rows' gradients dkc, dvc [B][n_kept][n_sel][D]
+ * fp32 (overwritten), which the caller reduce-scatters over the segment and
+ * adds at its own kept rows (usp_rows_copy with add); usp_longnet_bwd_end
+ * writes dQ [B][T][Hq][D] bf16.
+ * Workspace: usp_longnet_workspace_size(B, T, Hq, D, n_pairs, w, r, bwd) for
+ * the pairs that will be passed (0 for an unsupported shape). D in {64, 128},
+ * Hq % Hkv == 0, 1 <= r <= w.
+ */
+int usp_longnet_rows(int T, int w, int r, int o, int g, int* lp0, int* k_lo, int* n_rows, int* n_kept);
+size_t usp_longnet_workspace_size(int B, int T, int Hq, int D, int n_pairs, const int* w, const int* r, int bwd);
+int usp_longnet_fwd_begin(int B, int T, int Hq, int D, void* workspace, size_t ws_bytes, void* stream);
+int usp_longnet_fwd_local(const void* q, const void* k, const void* v, int B, int T, int Hq, int Hkv, int D,
+                          int causal, int w, int r, void* workspace, size_t ws_bytes, void* stream);
+int usp_longnet_fwd_cross(const void* q, const void* kc, const void* vc, int B, int T, int Hq, int Hkv, int D,
+                          int causal, int w, int r, int o, int g, void* workspace, size_t ws_bytes, void* stream);
+int usp_longnet_fwd_end(void* out, float* lse, int B, int T, int Hq, int D, void* workspace, size_t ws_bytes,
+                        void* stream);
+int usp_longnet_bwd_begin(const void* out, const float* lse, const void* dO, float* dK, float* dV, int B, int T,
+                          int Hq, int Hkv, int D, void* workspace, size_t ws_bytes, void* stream);
+int usp_longnet_bwd_local(const void* q, const void* k, const void* v, const void* dO, const float* lse, float* dK,
+                          float* dV, int B, int T, int Hq, int Hkv, int D, int causal, int w, int r, void* workspace,
+                          size_t ws_bytes, void* stream);
+int usp_longnet_bwd_cross(const void* q, const void* kc, const void* vc, const void* dO, const float* lse,
+                          float* dkc, float* dvc, int B, int T, int Hq, int Hkv, int D, int causal, int w, int r,
+                          int o, int g, void* workspace, size_t ws_bytes, void* stream);
+int usp_longnet_bwd_end(void* dQ, int B, int T, int Hq, int D, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * usp_workspace_status for the static scratch of usp_attn_bwd_noalloc (which a
  * caller cannot name): synchronises `stream`, returns USP_ERR_TIMEOUT if a
  * kernel of an earlier usp_attn_bwd_noalloc call on the current device recorded

@@ -34,11 +34,24 @@ USP_MAP_UNPACK_TOKENS = 5
 USP_MAP_PACK_TOKENS = 6
 USP_MAP_UNPACK_HEADS = 7
 USP_DILATED_MAX_PAIRS = 16
+USP_MAX_ROWS_JOBS = 16
 
 
 class AttnMask(ctypes.Structure):
     """usp_attn_mask of include/usp.h."""
     _fields_ = [("block_mask", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p), ("n_docs", ctypes.c_int)]
+
+
+class RowsJob(ctypes.Structure):
+    """usp_rows_job of include/usp.h."""
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("dtype", ctypes.c_int), ("add", ctypes.c_int),
+                ("n_b", ctypes.c_int), ("n_k", ctypes.c_int), ("n_j", ctypes.c_int), ("D", ctypes.c_int),
+                ("s_b", ctypes.c_longlong), ("s_k", ctypes.c_longlong), ("s_h", ctypes.c_longlong),
+                ("s_k0", ctypes.c_int), ("s_kstep", ctypes.c_int), ("s_h0", ctypes.c_int), ("s_hstep", ctypes.c_int),
+                ("s_hdiv", ctypes.c_int),
+                ("d_b", ctypes.c_longlong), ("d_k", ctypes.c_longlong), ("d_h", ctypes.c_longlong),
+                ("d_k0", ctypes.c_int), ("d_kstep", ctypes.c_int), ("d_h0", ctypes.c_int), ("d_hstep", ctypes.c_int),
+                ("d_hdiv", ctypes.c_int)]
 
 
 class PermuteJob(ctypes.Structure):
@@ -72,6 +85,17 @@ SIGNATURES = {
     "usp_dilated_attn_fwd": (_I, [_P] * 5 + [_I] * 7 + [_P, _P, _P, _SZ, _P]),
     "usp_dilated_bwd_workspace_size": (_SZ, [_I] * 5 + [_P, _P]),
     "usp_dilated_attn_bwd": (_I, [_P] * 9 + [_I] * 7 + [_P, _P, _P, _SZ, _P]),
+    "usp_rows_copy": (_I, [ctypes.POINTER(RowsJob), _I, _P]),
+    "usp_longnet_rows": (_I, [_I] * 5 + [_P] * 4),
+    "usp_longnet_workspace_size": (_SZ, [_I] * 5 + [_P, _P, _I]),
+    "usp_longnet_fwd_begin": (_I, [_I] * 4 + [_P, _SZ, _P]),
+    "usp_longnet_fwd_local": (_I, [_P] * 3 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_longnet_fwd_cross": (_I, [_P] * 3 + [_I] * 10 + [_P, _SZ, _P]),
+    "usp_longnet_fwd_end": (_I, [_P, _P] + [_I] * 4 + [_P, _SZ, _P]),
+    "usp_longnet_bwd_begin": (_I, [_P] * 5 + [_I] * 5 + [_P, _SZ, _P]),
+    "usp_longnet_bwd_local": (_I, [_P] * 7 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_longnet_bwd_cross": (_I, [_P] * 7 + [_I] * 10 + [_P, _SZ, _P]),
+    "usp_longnet_bwd_end": (_I, [_P] + [_I] * 4 + [_P, _SZ, _P]),
     "usp_attn_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 9 + [_P, _SZ, _P]),
     "usp_attn_bwd": (_I, [_P] * 9 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_fwd_masked": (_I, [_P] * 5 + [_I] * 8 + [ctypes.POINTER(AttnMask), _P, _SZ, _P]),
@@ -247,6 +271,80 @@ def usp_dilated_attn_bwd(q, k, v, out, lse, dO, dQ, dK, dV, B, S, Hq, Hkv, D, ca
     rc = lib().usp_dilated_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
                                     _ptr(dV), B, S, Hq, Hkv, D, int(causal), n, w, r, _ptr(workspace), ws_bytes,
                                     _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_rows_copy(jobs, stream=None, check=True):
+    """jobs: sequence of dicts with the usp_rows_job fields (src/dst tensors or pointers; omitted strides and
+    offsets default to 0, steps and divisors to 1)."""
+    arr = (RowsJob * max(len(jobs), 1))()
+    for x, j in enumerate(jobs):
+        f = dict(add=0, s_k0=0, s_kstep=1, s_h0=0, s_hstep=1, s_hdiv=1, d_k0=0, d_kstep=1, d_h0=0, d_hstep=1,
+                 d_hdiv=1, s_b=0, s_k=0, s_h=0, d_b=0, d_k=0, d_h=0)
+        f.update(j)
+        f["src"], f["dst"] = _ptr(f["src"]), _ptr(f["dst"])
+        arr[x] = RowsJob(**f)
+    rc = lib().usp_rows_copy(arr, len(jobs), _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_rows(T, w, r, o, g):
+    """(lp0, k_lo, n_rows, n_kept) of rank g of a segment at head offset o."""
+    out = [ctypes.c_int() for _ in range(4)]
+    _check(lib().usp_longnet_rows(T, w, r, o, g, *[ctypes.addressof(x) for x in out]))
+    return tuple(x.value for x in out)
+
+
+def usp_longnet_workspace_size(B, T, Hq, D, pairs, bwd) -> int:
+    n, w, r = _pairs(pairs)
+    return int(lib().usp_longnet_workspace_size(B, T, Hq, D, n, w, r, int(bwd)))
+
+
+def usp_longnet_fwd_begin(B, T, Hq, D, workspace, ws_bytes, stream=None, check=True):
+    rc = lib().usp_longnet_fwd_begin(B, T, Hq, D, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_fwd_local(q, k, v, B, T, Hq, Hkv, D, causal, w, r, workspace, ws_bytes, stream=None, check=True):
+    rc = lib().usp_longnet_fwd_local(_ptr(q), _ptr(k), _ptr(v), B, T, Hq, Hkv, D, int(causal), w, r, _ptr(workspace),
+                                     ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_fwd_cross(q, kc, vc, B, T, Hq, Hkv, D, causal, w, r, o, g, workspace, ws_bytes, stream=None,
+                          check=True):
+    rc = lib().usp_longnet_fwd_cross(_ptr(q), _ptr(kc), _ptr(vc), B, T, Hq, Hkv, D, int(causal), w, r, o, g,
+                                     _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_fwd_end(out, lse, B, T, Hq, D, workspace, ws_bytes, stream=None, check=True):
+    rc = lib().usp_longnet_fwd_end(_ptr(out), _ptr(lse), B, T, Hq, D, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_bwd_begin(out, lse, dO, dK, dV, B, T, Hq, Hkv, D, workspace, ws_bytes, stream=None, check=True):
+    rc = lib().usp_longnet_bwd_begin(_ptr(out), _ptr(lse), _ptr(dO), _ptr(dK), _ptr(dV), B, T, Hq, Hkv, D,
+                                     _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_bwd_local(q, k, v, dO, lse, dK, dV, B, T, Hq, Hkv, D, causal, w, r, workspace, ws_bytes, stream=None,
+                          check=True):
+    rc = lib().usp_longnet_bwd_local(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(lse), _ptr(dK), _ptr(dV), B, T, Hq,
+                                     Hkv, D, int(causal), w, r, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_bwd_cross(q, kc, vc, dO, lse, dkc, dvc, B, T, Hq, Hkv, D, causal, w, r, o, g, workspace, ws_bytes,
+                          stream=None, check=True):
+    rc = lib().usp_longnet_bwd_cross(_ptr(q), _ptr(kc), _ptr(vc), _ptr(dO), _ptr(lse), _ptr(dkc), _ptr(dvc), B, T,
+                                     Hq, Hkv, D, int(causal), w, r, o, g, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_longnet_bwd_end(dQ, B, T, Hq, D, workspace, ws_bytes, stream=None, check=True):
+    rc = lib().usp_longnet_bwd_end(_ptr(dQ), B, T, Hq, D, _ptr(workspace), ws_bytes, _stream(stream))
     return _check(rc) if check else rc
 
 

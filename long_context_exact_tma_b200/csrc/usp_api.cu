@@ -150,11 +150,15 @@ namespace usp {
 // stride4 bytes apart; box 64 x 1 x 128 x 1, 128-byte swizzle.
 int make_tmap_strided(CUtensorMap* m, const void* base, int D, int H, long long rows, long long n4,
                       unsigned long long row_stride, unsigned long long stride4) {
+  return make_tmap_strided_h(m, base, D, H, rows, n4, static_cast<unsigned long long>(D) * 2, row_stride, stride4);
+}
+int make_tmap_strided_h(CUtensorMap* m, const void* base, int D, int H, long long rows, long long n4,
+                        unsigned long long head_stride, unsigned long long row_stride, unsigned long long stride4) {
   auto fn = encode_fn();
   if (!fn) return record_error(USP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(n4)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, row_stride, stride4};
+  cuuint64_t strides[3] = {head_stride, row_stride, stride4};
   cuuint32_t box[4] = {64, 1, 128, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,

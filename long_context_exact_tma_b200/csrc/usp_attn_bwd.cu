@@ -99,7 +99,7 @@ template <bool kPlain = false>
 __device__ __forceinline__ int classify_q(const Geo& g, int i, int m, int kmin, int kmax) {
   const int q0 = m * kBM;
   int qmin, qmax;
-  pos_range<kPlain>(g, i, q0, q0 + kBM, qmin, qmax);
+  qpos_range<kPlain>(g, i, q0, q0 + kBM, qmin, qmax);
   // Padded query columns need no mask: their LSE is +inf, so P = 0 there.
   if (g.causal && qmax < kmin) return kSkip;
   if (!g.causal || qmin >= kmax) return kFull;
@@ -441,11 +441,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       if (st_kind == kMasked) {
         // causal: rewrite S^T of this key row to -inf where the query does not see
         // the key, so the main pass carries no masking (P = 0 there)
-        int lo = pos_k == INT_MAX ? kBM : pos_k - token_pos<kSub>(g, st_i, q0);  // aligned: cols >= lo see it
+        int lo = pos_k == INT_MAX ? kBM : pos_k - qtoken_pos<kSub>(g, st_i, q0);  // aligned: cols >= lo see it
         int hi_c = kBM;                                                      // and cols < hi_c
         if constexpr (kMask) {
           // masked variant (tiles contiguous): the key's document bounds the columns too
-          const int qpos0 = token_pos<kSub>(g, st_i, q0);
+          const int qpos0 = qtoken_pos<kSub>(g, st_i, q0);
           if (!g.causal && pos_k != INT_MAX) lo = 0;
           if (pos_k != INT_MAX) {
             lo = max(lo, doc_lo - qpos0);
@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             vis = 0u;
             for (int c = 0; c < 32; ++c) {
               const int tq = q0 + c0 + c;
-              if (tq < g.L && pos_k <= token_pos<kSub>(g, st_i, tq)) vis |= 1u << c;
+              if (tq < g.Lq && pos_k <= qtoken_pos<kSub>(g, st_i, tq)) vis |= 1u << c;
             }
           }
           uint32_t r[32];
@@ -543,10 +543,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       tc_fence_after();
       const bool store = tau_k < g.L;
       size_t kr;
-      if constexpr (kSub) {  // the key's original position in [B][S][Hkv]
+      if constexpr (kSub) {  // the key's row in the dK/dV buffers (its original position, or a gathered row)
         const int pb = prob / a.sub.n_seg, ps = prob % a.sub.n_seg;
-        kr = (static_cast<size_t>(pb) * a.sub.S + static_cast<size_t>(ps) * a.sub.w + a.sub.off +
-              static_cast<size_t>(store ? tau_k : 0) * a.sub.r) * g.Hkv_l + gl;
+        kr = (static_cast<size_t>(pb) * a.sub.kS + static_cast<size_t>(ps) * a.sub.kw + a.sub.koff +
+              static_cast<size_t>(store ? tau_k : 0) * a.sub.kstep) * a.sub.kH + gl;
       } else {
         kr = (static_cast<size_t>(jrank * g.B + b) * g.L + (store ? tau_k : 0)) * g.Hkv_l + gl;
       }
@@ -621,7 +621,10 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
     a.g.P_u = a.g.P_r = a.g.P = a.g.n_ranks = 1;
     a.g.L = L.sub.L;
     a.g.c = kBN;
-    a.g.n_qtiles = a.g.n_ktiles = (L.sub.L + kBM - 1) / kBM;
+    a.g.Lq = L.sub.Lq;
+    a.g.q_off = L.sub.q_off;
+    a.g.n_qtiles = (L.sub.Lq + kBM - 1) / kBM;
+    a.g.n_ktiles = (L.sub.L + kBN - 1) / kBN;
   }
   const long long blocks = kSub     ? static_cast<long long>(a.g.n_ktiles) * a.g.Hkv_l * L.sub.n_prob
                            : kLocal ? static_cast<long long>(a.g.n_ktiles) * a.g.B * a.g.Hkv_l

@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     // elected lane issues each copy and barrier operation.
     {
       int qmin, qmax;
-      pos_range<kSub>(g, i, q0, q0 + kBM, qmin, qmax);
+      qpos_range<kSub>(g, i, q0, q0 + kBM, qmin, qmax);
       // masked variant: the causal kind narrowed by the block / document masks
       auto kind_of = [&](int j, int n) {
         int kmin, kmax;
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const int cbase = wg * 64;
     const int tau_q = q0 + row;
-    const int pos_q = tau_q < g.L ? token_pos<kSub>(g, i, tau_q) : INT_MAX;
+    const int pos_q = tau_q < g.Lq ? qtoken_pos<kSub>(g, i, tau_q) : INT_MAX;
     const bool aligned = (g.c % kBN) == 0;
     int doc_lo = 0, doc_hi = INT_MAX;  // the row's document [lo, hi) (masked variant)
     if constexpr (kMask) doc_span(g.mask, pos_q, doc_lo, doc_hi);
@@ -468,12 +468,12 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_done[(it - 1) & 1], ((it - 1) >> 1) & 1, w, kSiteQEpi));
     if (ok) {
       tc_fence_after();
-      const bool store = tau_q < g.L;
+      const bool store = tau_q < g.Lq;
       size_t qr;
       if constexpr (kSub) {  // the query's original position in [B][S][Hq]
         const int pb = prob / a.sub.n_seg, ps = prob % a.sub.n_seg;
         qr = (static_cast<size_t>(pb) * a.sub.S + static_cast<size_t>(ps) * a.sub.w + a.sub.off +
-              static_cast<size_t>(store ? tau_q : 0) * a.sub.r) * a.sub.Hq + h;
+              static_cast<size_t>(store ? tau_q : 0) * a.sub.r) * a.sub.Hq + (a.sub.out_h0 + h * a.sub.out_hstep);
       } else {
         qr = (static_cast<size_t>(rank * g.B + b) * g.L + (store ? tau_q : 0)) * g.Hq_l + h;
       }
@@ -569,7 +569,10 @@ cudaError_t launch_dq_d(const BwdLaunch& L, cudaStream_t stream) {
     a.g.P_u = a.g.P_r = a.g.P = a.g.n_ranks = 1;
     a.g.L = L.sub.L;
     a.g.c = kBN;
-    a.g.n_qtiles = a.g.n_ktiles = (L.sub.L + kBM - 1) / kBM;
+    a.g.Lq = L.sub.Lq;
+    a.g.q_off = L.sub.q_off;
+    a.g.n_qtiles = (L.sub.Lq + kBM - 1) / kBM;
+    a.g.n_ktiles = (L.sub.L + kBN - 1) / kBN;
   }
   const long long blocks = kSub     ? static_cast<long long>(a.g.n_qtiles) * L.sub.n_heads * L.sub.n_prob
                            : kLocal ? static_cast<long long>(a.g.n_qtiles) * a.g.B * a.g.Hq_l

@@ -30,6 +30,7 @@ constexpr int kBN = 128;  // keys per tile
 
 struct Geo {
   int B, L, Hq_l, Hkv_l, G, P_u, P_r, P, c, causal, n_ranks, n_qtiles, n_ktiles;
+  int Lq, q_off;     // query rows and the position of the first (L and 0 but in a query window)
   MaskArgs mask;     // read only by the masked kernel variants
   float scale_log2;  // softmax scale * log2(e)
   float scale;       // softmax scale
@@ -41,6 +42,8 @@ inline Geo make_geo(const AttnGeom& a) {
   g.P = a.P; g.c = a.c; g.causal = a.causal; g.n_ranks = a.n_ranks;
   g.n_qtiles = (a.L + kBM - 1) / kBM;
   g.n_ktiles = (a.L + kBN - 1) / kBN;
+  g.Lq = a.L;
+  g.q_off = 0;
   g.scale = 1.0f / sqrtf(static_cast<float>(a.D));
   g.scale_log2 = g.scale * 1.4426950408889634f;
   return g;
@@ -74,6 +77,27 @@ __device__ __forceinline__ void pos_range(const Geo& g, int i, int t0, int t1, i
       pmin = min(pmin, token_pos(g, i, a));
       pmax = max(pmax, token_pos(g, i, e));
     }
+  }
+}
+
+// Query-side forms: the same positions, except in the sub-problem mode, where
+// the g.Lq query rows of a launch are a window whose positions start at g.q_off.
+template <bool kPlain = false>
+__device__ __forceinline__ int qtoken_pos(const Geo& g, int i, int tau) {
+  if constexpr (kPlain) return g.q_off + tau;
+  return token_pos(g, i, tau);
+}
+template <bool kPlain = false>
+__device__ __forceinline__ void qpos_range(const Geo& g, int i, int t0, int t1, int& pmin, int& pmax) {
+  if constexpr (kPlain) {
+    if (t1 > g.Lq) t1 = g.Lq;
+    pmin = INT_MAX;
+    pmax = -1;
+    if (t0 >= t1) return;
+    pmin = g.q_off + t0;
+    pmax = g.q_off + t1 - 1;
+  } else {
+    pos_range(g, i, t0, t1, pmin, pmax);
   }
 }
 

@@ -223,8 +223,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     {
       const bool kside = warp == 0;
       int qmin0, qmax0, qmin1, qmax1;
-      pos_range<kSub>(g, i, q0, q0 + kBM, qmin0, qmax0);
-      pos_range<kSub>(g, i, q0 + kBM, q0 + 2 * kBM, qmin1, qmax1);
+      qpos_range<kSub>(g, i, q0, q0 + kBM, qmin0, qmax0);
+      qpos_range<kSub>(g, i, q0 + kBM, q0 + 2 * kBM, qmin1, qmax1);
       const int qmin = min(qmin0, qmin1), qmax = max(qmax0, qmax1);
       // masked variant: both query tiles' kinds narrowed by the block / document
       // masks; a key tile is walked when either query tile attends it
@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t cS = col_s(t), cO = col_o(t);
     const int tau_q = q0 + t * kBM + row;
-    const int pos_q = tau_q < g.L ? token_pos<kSub>(g, i, tau_q) : INT_MAX;
+    const int pos_q = tau_q < g.Lq ? qtoken_pos<kSub>(g, i, tau_q) : INT_MAX;
     const bool aligned = (g.c % kBN) == 0;
     int doc_lo = 0, doc_hi = INT_MAX;  // the row's document [lo, hi) (masked variant)
     if constexpr (kMask) doc_span(g.mask, pos_q, doc_lo, doc_hi);
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     if (ok && it >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done[t], (it - 1) & 1, w, kSiteO));
     if (ok) {
       tc_fence_after();
-      const bool store = tau_q < g.L;
+      const bool store = tau_q < g.Lq;
       const float inv_l = lb_run > 0.f ? 1.f / lb_run : 0.f;
       const float lse_val = l_run > 0.f ? (m_use + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
       if constexpr (kSub) {
@@ -561,7 +561,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         const int pb = qc4 / a.sub.n_seg, ps = qc4 % a.sub.n_seg;
         const size_t orow = static_cast<size_t>(pb) * a.sub.S + static_cast<size_t>(ps) * a.sub.w + a.sub.off +
                             static_cast<size_t>(store ? tau_q : 0) * a.sub.r;
-        const size_t ridx = orow * a.sub.Hq + h;
+        const size_t ridx = orow * a.sub.Hq + (a.sub.out_h0 + h * a.sub.out_hstep);
         float lse_old = -INFINITY;
         if (store) lse_old = a.sub.lse_run[ridx];
         const float mx = fmaxf(lse_old, lse_val);
@@ -676,7 +676,10 @@ cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
     a.g.P_u = a.g.P_r = a.g.P = a.g.n_ranks = 1;
     a.g.L = L.sub.L;
     a.g.c = kBN;
-    a.g.n_qtiles = a.g.n_ktiles = (L.sub.L + kBM - 1) / kBM;
+    a.g.Lq = L.sub.Lq;
+    a.g.q_off = L.sub.q_off;
+    a.g.n_qtiles = (L.sub.Lq + kBM - 1) / kBM;
+    a.g.n_ktiles = (L.sub.L + kBN - 1) / kBN;
     blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * L.sub.n_heads * L.sub.n_prob;
   } else if (kMode == kModeLocal) {
     a.loc_i = L.loc_i;

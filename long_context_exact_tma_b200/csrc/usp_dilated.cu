@@ -34,6 +34,59 @@ extern "C" size_t usp_dilated_workspace_size(int B, int S, int Hq, int D) {
   return dilated_ws(B, S, Hq, D);
 }
 
+namespace usp {
+
+int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S, int Hq, int Hkv, int D, int causal,
+                      int wp, int rp, float* o_run, float* lse_run, int* status, cudaStream_t st) {
+  FwdLaunch L{};
+  AttnGeom& g = L.g;
+  g.B = B; g.S = S; g.Hq = Hq; g.Hkv = Hkv; g.D = D; g.causal = causal;
+  g.P_u = g.P_r = g.P = g.n_ranks = 1;
+  g.G = Hq / Hkv;
+  g.Hq_l = Hq;
+  g.Hkv_l = Hkv;
+  L.status = status;
+  L.wait_ns = current_wait_ns();
+  L.step = -1;
+  const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;  // bytes per token row
+  const int n_seg = S / wp;
+  for (int off = 0; off < rp && off < Hq; ++off) {
+    const int kept = (wp - off + rp - 1) / rp;  // rows of a segment at offset off
+    g.L = kept;
+    g.c = kept;  // unused in the sub-problem mode
+    FwdSub& sb = L.sub;
+    sb.active = 1;
+    sb.n_prob = B * n_seg;
+    sb.L = kept;
+    sb.h0 = off;
+    sb.h_step = rp;
+    sb.n_heads = (Hq - off + rp - 1) / rp;
+    sb.n_seg = n_seg;
+    sb.w = wp;
+    sb.off = off;
+    sb.r = rp;
+    sb.S = S;
+    sb.Hq = Hq;
+    sb.o_run = o_run;
+    sb.lse_run = lse_run;
+    sub_defaults(sb, Hkv);
+    int rc = make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, kept, sb.n_prob,
+                               rp * tokq, wp * tokq);
+    if (rc == USP_OK)
+      rc = make_tmap_strided(&L.tm_k, static_cast<const uint8_t*>(k) + off * tokkv, D, Hkv, kept, sb.n_prob,
+                             rp * tokkv, wp * tokkv);
+    if (rc == USP_OK)
+      rc = make_tmap_strided(&L.tm_v, static_cast<const uint8_t*>(v) + off * tokkv, D, Hkv, kept, sb.n_prob,
+                             rp * tokkv, wp * tokkv);
+    if (rc != USP_OK) return rc;
+    const cudaError_t e = launch_attn_fwd(L, st);
+    if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated attention launch: %s", cudaGetErrorString(e));
+  }
+  return USP_OK;
+}
+
+}  // namespace usp
+
 extern "C" int usp_dilated_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                                     int S, int Hq, int Hkv, int D, int causal, int n_pairs, const int* w,
                                     const int* r, void* workspace, size_t ws_bytes, void* stream) {
@@ -64,51 +117,10 @@ extern "C" int usp_dilated_attn_fwd(const void* q, const void* k, const void* v,
   if (e == cudaSuccess) e = usp::launch_fill_running(o_run, lse_run, rows, D, st);
   if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "running-result init: %s", cudaGetErrorString(e));
 
-  usp::FwdLaunch L{};
-  usp::AttnGeom& g = L.g;
-  g.B = B; g.S = S; g.Hq = Hq; g.Hkv = Hkv; g.D = D; g.causal = causal;
-  g.P_u = g.P_r = g.P = g.n_ranks = 1;
-  g.G = Hq / Hkv;
-  g.Hq_l = Hq;
-  g.Hkv_l = Hkv;
-  L.status = static_cast<int*>(workspace);
-  L.wait_ns = usp::current_wait_ns();
-  L.step = -1;
-  const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;  // bytes per token row
   for (int p = 0; p < n_pairs; ++p) {
-    const int wp = w[p], rp = r[p];
-    const int n_seg = S / wp;
-    for (int off = 0; off < rp && off < Hq; ++off) {
-      const int kept = (wp - off + rp - 1) / rp;  // rows of a segment at offset off
-      g.L = kept;
-      g.c = kept;  // unused in the sub-problem mode
-      usp::FwdSub& sb = L.sub;
-      sb.active = 1;
-      sb.n_prob = B * n_seg;
-      sb.L = kept;
-      sb.h0 = off;
-      sb.h_step = rp;
-      sb.n_heads = (Hq - off + rp - 1) / rp;
-      sb.n_seg = n_seg;
-      sb.w = wp;
-      sb.off = off;
-      sb.r = rp;
-      sb.S = S;
-      sb.Hq = Hq;
-      sb.o_run = o_run;
-      sb.lse_run = lse_run;
-      int rc = usp::make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, kept,
-                                      sb.n_prob, rp * tokq, wp * tokq);
-      if (rc == USP_OK)
-        rc = usp::make_tmap_strided(&L.tm_k, static_cast<const uint8_t*>(k) + off * tokkv, D, Hkv, kept,
-                                    sb.n_prob, rp * tokkv, wp * tokkv);
-      if (rc == USP_OK)
-        rc = usp::make_tmap_strided(&L.tm_v, static_cast<const uint8_t*>(v) + off * tokkv, D, Hkv, kept,
-                                    sb.n_prob, rp * tokkv, wp * tokkv);
-      if (rc != USP_OK) return rc;
-      e = usp::launch_attn_fwd(L, st);
-      if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated attention launch: %s", cudaGetErrorString(e));
-    }
+    const int rc = usp::dilated_fold_pair(q, k, v, B, S, Hq, Hkv, D, causal, w[p], r[p], o_run, lse_run,
+                                          static_cast<int*>(workspace), st);
+    if (rc != USP_OK) return rc;
   }
   e = usp::launch_lse_merge(o_run, lse_run, 1, rows, D, out, 0, lse, st);
   if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "final merge launch: %s", cudaGetErrorString(e));
@@ -137,15 +149,91 @@ DilatedLaunchShape launch_shape(int S, int Hq, int w, int r, int off) {
   return DilatedLaunchShape{(w - off + r - 1) / r, S / w, (Hq - off + r - 1) / r};
 }
 
+}  // namespace
+
+namespace usp {
+
+size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r) {
+  size_t tbl = 0;  // the largest per-launch table: n_prob * n_heads * Lp floats
+  for (int off = 0; off < r && off < Hq; ++off) {
+    const DilatedLaunchShape sh = launch_shape(S, Hq, w, r, off);
+    const size_t Lp = static_cast<size_t>((sh.kept + 127) / 128 * 128);
+    const size_t n = static_cast<size_t>(B) * sh.n_seg * sh.n_heads * Lp;
+    if (n > tbl) tbl = n;
+  }
+  return tbl;
+}
+
+int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO, const float* lse,
+                     const float* delta_all, float* dq_acc, float* dK, float* dV, float* lse2_t, float* delta_t, int B,
+                     int S, int Hq, int Hkv, int D, int causal, int wp, int rp, int* status, cudaStream_t st) {
+  BwdLaunch L{};
+  AttnGeom& g = L.g;
+  g.B = B; g.S = S; g.Hq = Hq; g.Hkv = Hkv; g.D = D; g.causal = causal;
+  g.P_u = g.P_r = g.P = g.n_ranks = 1;
+  g.G = Hq / Hkv;
+  g.Hq_l = Hq;
+  g.Hkv_l = Hkv;
+  L.status = status;
+  L.wait_ns = current_wait_ns();
+  L.lse2 = lse2_t;
+  L.delta = delta_t;
+  L.dk = dK;
+  L.dv = dV;
+  L.dq = nullptr;
+  L.dq_acc = dq_acc;
+  const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;
+  for (int off = 0; off < rp && off < Hq; ++off) {
+    const DilatedLaunchShape sh = launch_shape(S, Hq, wp, rp, off);
+    FwdSub& sb = L.sub;
+    sb.active = 1;
+    sb.n_prob = B * sh.n_seg;
+    sb.L = sh.kept;
+    sb.h0 = off;
+    sb.h_step = rp;
+    sb.n_heads = sh.n_heads;
+    sb.n_seg = sh.n_seg;
+    sb.w = wp;
+    sb.off = off;
+    sb.r = rp;
+    sb.S = S;
+    sb.Hq = Hq;
+    sub_defaults(sb, Hkv);
+    g.L = sh.kept;
+    g.c = sh.kept;
+    L.Lp = (sh.kept + 127) / 128 * 128;
+    int rc = make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, sh.kept, sb.n_prob,
+                               rp * tokq, wp * tokq);
+    if (rc == USP_OK)
+      rc = make_tmap_strided(&L.tm_do, static_cast<const uint8_t*>(dO) + off * tokq, D, Hq, sh.kept, sb.n_prob,
+                             rp * tokq, wp * tokq);
+    if (rc == USP_OK)
+      rc = make_tmap_strided(&L.tm_k, static_cast<const uint8_t*>(k) + off * tokkv, D, Hkv, sh.kept, sb.n_prob,
+                             rp * tokkv, wp * tokkv);
+    if (rc == USP_OK)
+      rc = make_tmap_strided(&L.tm_v, static_cast<const uint8_t*>(v) + off * tokkv, D, Hkv, sh.kept, sb.n_prob,
+                             rp * tokkv, wp * tokkv);
+    if (rc != USP_OK) return rc;
+    cudaError_t e = launch_dilated_tables(lse, delta_all, lse2_t, delta_t, sb, L.Lp, st);
+    if (e == cudaSuccess) e = launch_attn_bwd(L, st);
+    if (e == cudaSuccess) e = launch_attn_bwd_dq(L, st);
+    if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated backward launch: %s", cudaGetErrorString(e));
+  }
+  return USP_OK;
+}
+
+}  // namespace usp
+
+namespace {
+
+using usp::record_error;
+
 size_t dilated_bwd_ws(int B, int S, int Hq, int D, int n_pairs, const int* w, const int* r, size_t* tbl_floats) {
   size_t tbl = 0;  // the largest per-launch table: n_prob * n_heads * Lp floats
-  for (int p = 0; p < n_pairs; ++p)
-    for (int off = 0; off < r[p] && off < Hq; ++off) {
-      const DilatedLaunchShape sh = launch_shape(S, Hq, w[p], r[p], off);
-      const size_t Lp = static_cast<size_t>((sh.kept + 127) / 128 * 128);
-      const size_t n = static_cast<size_t>(B) * sh.n_seg * sh.n_heads * Lp;
-      if (n > tbl) tbl = n;
-    }
+  for (int p = 0; p < n_pairs; ++p) {
+    const size_t n = usp::dilated_pair_table_floats(B, S, Hq, w[p], r[p]);
+    if (n > tbl) tbl = n;
+  }
   if (tbl_floats) *tbl_floats = tbl;
   const size_t rows = static_cast<size_t>(B) * S * Hq;
   // status | Delta of every row | fp32 dQ | two row tables
@@ -210,60 +298,10 @@ extern "C" int usp_dilated_attn_bwd(const void* q, const void* k, const void* v,
   if (e == cudaSuccess) e = usp::launch_bwd_preprocess(out, dO, delta_all, rows, D, st);
   if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated backward init: %s", cudaGetErrorString(e));
 
-  usp::BwdLaunch L{};
-  usp::AttnGeom& g = L.g;
-  g.B = B; g.S = S; g.Hq = Hq; g.Hkv = Hkv; g.D = D; g.causal = causal;
-  g.P_u = g.P_r = g.P = g.n_ranks = 1;
-  g.G = Hq / Hkv;
-  g.Hq_l = Hq;
-  g.Hkv_l = Hkv;
-  L.status = static_cast<int*>(workspace);
-  L.wait_ns = usp::current_wait_ns();
-  L.lse2 = lse2_t;
-  L.delta = delta_t;
-  L.dk = dK;
-  L.dv = dV;
-  L.dq = nullptr;
-  L.dq_acc = dq_acc;
-  const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;
   for (int p = 0; p < n_pairs; ++p) {
-    const int wp = w[p], rp = r[p];
-    for (int off = 0; off < rp && off < Hq; ++off) {
-      const DilatedLaunchShape sh = launch_shape(S, Hq, wp, rp, off);
-      usp::FwdSub& sb = L.sub;
-      sb.active = 1;
-      sb.n_prob = B * sh.n_seg;
-      sb.L = sh.kept;
-      sb.h0 = off;
-      sb.h_step = rp;
-      sb.n_heads = sh.n_heads;
-      sb.n_seg = sh.n_seg;
-      sb.w = wp;
-      sb.off = off;
-      sb.r = rp;
-      sb.S = S;
-      sb.Hq = Hq;
-      g.L = sh.kept;
-      g.c = sh.kept;
-      L.Lp = (sh.kept + 127) / 128 * 128;
-      rc = usp::make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, sh.kept, sb.n_prob,
-                                  rp * tokq, wp * tokq);
-      if (rc == USP_OK)
-        rc = usp::make_tmap_strided(&L.tm_do, static_cast<const uint8_t*>(dO) + off * tokq, D, Hq, sh.kept,
-                                    sb.n_prob, rp * tokq, wp * tokq);
-      if (rc == USP_OK)
-        rc = usp::make_tmap_strided(&L.tm_k, static_cast<const uint8_t*>(k) + off * tokkv, D, Hkv, sh.kept,
-                                    sb.n_prob, rp * tokkv, wp * tokkv);
-      if (rc == USP_OK)
-        rc = usp::make_tmap_strided(&L.tm_v, static_cast<const uint8_t*>(v) + off * tokkv, D, Hkv, sh.kept,
-                                    sb.n_prob, rp * tokkv, wp * tokkv);
-      if (rc != USP_OK) return rc;
-      e = usp::launch_dilated_tables(lse, delta_all, lse2_t, delta_t, sb, L.Lp, st);
-      if (e == cudaSuccess) e = usp::launch_attn_bwd(L, st);
-      if (e == cudaSuccess) e = usp::launch_attn_bwd_dq(L, st);
-      if (e != cudaSuccess)
-        return record_error(USP_ERR_CUDA, "dilated backward launch: %s", cudaGetErrorString(e));
-    }
+    rc = usp::dilated_bwd_pair(q, k, v, dO, lse, delta_all, dq_acc, dK, dV, lse2_t, delta_t, B, S, Hq, Hkv, D,
+                               causal, w[p], r[p], static_cast<int*>(workspace), st);
+    if (rc != USP_OK) return rc;
   }
   e = usp::launch_f32_to_bf16(dq_acc, dQ, rows * D, st);
   if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dQ conversion: %s", cudaGetErrorString(e));

@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(256) dilated_tables_kernel(const float* __rest
                                                              float* __restrict__ lse2_t, float* __restrict__ delta_t,
                                                              long long n, int Lp, int kept, int n_heads, int h0,
                                                              int h_step, int n_seg, int w, int off, int r, int S,
-                                                             int Hq) {
+                                                             int Hq, int out_h0, int out_hstep) {
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += stride) {
     const int tau = static_cast<int>(e % Lp);
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(256) dilated_tables_kernel(const float* __rest
       continue;
     }
     const long long row = ((p / n_seg) * S + (p % n_seg) * w + off + static_cast<long long>(tau) * r) * Hq +
-                          h0 + static_cast<long long>(jh) * h_step;
+                          out_h0 + (h0 + static_cast<long long>(jh) * h_step) * out_hstep;
     const float l = lse[row];
     lse2_t[e] = l == -INFINITY ? -INFINITY : -l * 1.4426950408889634f;
     delta_t[e] = -delta_all[row];
@@ -339,9 +339,9 @@ cudaError_t launch_dilated_tables(const float* lse, const float* delta_all, floa
                                   const FwdSub& sb, int Lp, cudaStream_t stream) {
   const long long n = static_cast<long long>(sb.n_prob) * sb.n_heads * Lp;
   if (n == 0) return cudaSuccess;
-  dilated_tables_kernel<<<grid_for(256, n), 256, 0, stream>>>(lse, delta_all, lse2_t, delta_t, n, Lp, sb.L,
+  dilated_tables_kernel<<<grid_for(256, n), 256, 0, stream>>>(lse, delta_all, lse2_t, delta_t, n, Lp, sb.Lq,
                                                               sb.n_heads, sb.h0, sb.h_step, sb.n_seg, sb.w, sb.off,
-                                                              sb.r, sb.S, sb.Hq);
+                                                              sb.r, sb.S, sb.Hq, sb.out_h0, sb.out_hstep);
   note_launch();
   return cudaGetLastError();
 }

@@ -26,6 +26,9 @@ int validate_geom(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int
 // block strides in bytes (box 64 x 1 x 128 x 1, 128-byte swizzle); usp_status.
 int make_tmap_strided(CUtensorMap* m, const void* base, int D, int H, long long rows, long long n4,
                       unsigned long long row_stride, unsigned long long stride4);
+// The same with an explicit head stride in bytes (a multiple of 16).
+int make_tmap_strided_h(CUtensorMap* m, const void* base, int D, int H, long long rows, long long n4,
+                        unsigned long long head_stride, unsigned long long row_stride, unsigned long long stride4);
 
 // Fills a running fp32 (O, LSE) with the empty result: O = 0, LSE = -inf.
 cudaError_t launch_fill_running(float* o, float* lse, long long rows, int D, cudaStream_t stream);
@@ -84,13 +87,36 @@ struct AttnGeom {
 // (p / n_seg) * S + (p % n_seg) * w + off + tau * r by the log-sum-exp merge.
 // LongNet's dilated attention runs one such launch per (w, r) pair and head
 // offset off, with tensor maps that step r rows from the offset.
+// A query window makes a launch a cross-attention of some rows to the whole
+// problem: Lq query rows whose kept indices (positions) start at q_off, against
+// all L key rows (one rank's kept rows of a segment gathered from several
+// ranks, LongNet's distributed layout). Query-side outputs (O, LSE, dQ, the row
+// tables) use the mapping above with the output head out_h0 + h * out_hstep of
+// the launch's head index h; the key-side outputs of the backward (dK, dV) use
+// row (p / n_seg) * kS + (p % n_seg) * kw + koff + tau * kstep with kH heads a
+// row. sub_defaults() makes a plain dilated launch: the window is all L rows,
+// the output head is h, and keys map like queries.
 struct FwdSub {
   int active;
   int n_prob, L, h0, h_step, n_heads;
   int n_seg, w, off, r, S, Hq;
   float* o_run;    // fp32 [B*S][Hq][D]
   float* lse_run;  // fp32 [B*S][Hq]
+  int Lq, q_off;
+  int out_h0, out_hstep;
+  int kS, kw, koff, kstep, kH;
 };
+inline void sub_defaults(FwdSub& sb, int Hkv) {
+  sb.Lq = sb.L;
+  sb.q_off = 0;
+  sb.out_h0 = 0;
+  sb.out_hstep = 1;
+  sb.kS = sb.S;
+  sb.kw = sb.w;
+  sb.koff = sb.off;
+  sb.kstep = sb.r;
+  sb.kH = Hkv;
+}
 
 struct FwdLaunch {
   AttnGeom g;
@@ -144,5 +170,18 @@ struct BwdLaunch {
 };
 cudaError_t launch_attn_bwd(const BwdLaunch& a, cudaStream_t stream);     // dK, dV (key-major)
 cudaError_t launch_attn_bwd_dq(const BwdLaunch& a, cudaStream_t stream);  // dQ (query-major)
+
+// LongNet dilated attention of one (w, r) pair over B sequences of S tokens
+// (global layout [B][S][H][D]), every head offset (usp_dilated.cu): the forward
+// folds the pair's result into the running fp32 (O, LSE); the backward adds the
+// pair's dQ (into the fp32 dq_acc), dK and dV (fp32), with the final LSE and
+// Delta of every row and two row-table buffers of dilated_pair_table_floats
+// floats each. usp_status.
+int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S, int Hq, int Hkv, int D, int causal,
+                      int w, int r, float* o_run, float* lse_run, int* status, cudaStream_t st);
+size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r);
+int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO, const float* lse,
+                     const float* delta_all, float* dq_acc, float* dK, float* dV, float* lse2_t, float* delta_t, int B,
+                     int S, int Hq, int Hkv, int D, int causal, int w, int r, int* status, cudaStream_t st);
 
 }  // namespace usp

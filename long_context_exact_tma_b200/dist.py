@@ -250,3 +250,244 @@ def usp_attention_bwd(dout, saved, geo: Geometry, mesh: Mesh, ops=None):
     (doh,) = seq2head([dout], geo, mesh, ops)
     dqh, dkh, dvh = ring_attn_bwd(qh, kh, vh, out_h, lse_h, doh, geo, mesh, ops)
     return tuple(head2seq([dqh, dkh, dvh], geo, mesh, ops))
+
+
+# ---------------------------------------------------------------- LongNet's distributed layout
+#
+# LongNet slides, "LONGNET as a Distributed Trainer": the sequence is split
+# into M contiguous slices of T = S / M tokens, one per rank. A dilated pair
+# (w, r) whose segments fit a slice (w <= T) is computed locally. A longer
+# segment spans G = w / T ranks: for each head offset o every rank packs its
+# kept K/V rows (positions = o mod r, the kv heads of the query heads o, o + r,
+# ...: 1/r of its rows), the G ranks all-gather them, and each rank's kept
+# queries attend all the segment's kept rows. In the backward the all-gather's
+# transpose, a reduce-scatter, brings every rank's contribution to the
+# gathered rows' dK/dV back to the rank that holds those rows.
+
+
+class TorchComm:
+    """The collectives of the LongNet schedule over torch.distributed groups
+    (NCCL on GPUs; gloo lacks the tensor forms, so there the same sums are
+    taken by all_gather / all_reduce)."""
+
+    def all_gather(self, recv, send, group):
+        """recv [G, *send.shape] <- every group member's send, in group-rank order."""
+        if dist.get_backend(group) == "nccl":
+            dist.all_gather_into_tensor(recv.view(-1), send.reshape(-1), group=group)
+        else:
+            dist.all_gather(list(recv.unbind(0)), send, group=group)
+
+    def reduce_scatter(self, recv, send, group):
+        """recv <- sum over the group of send[this member's group rank]."""
+        if dist.get_backend(group) == "nccl":
+            dist.reduce_scatter_tensor(recv.reshape(-1), send.reshape(-1), op=dist.ReduceOp.SUM, group=group)
+        else:
+            buf = send.clone()
+            dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=group)
+            recv.copy_(buf[dist.get_rank(group)])
+
+
+class LongNetMesh:
+    """Rank d of M holds positions [d T, (d + 1) T). For every gathered segment
+    length w (w > T) the M / G groups of G = w / T consecutive ranks; every
+    rank must construct this (torch.distributed.new_group is collective)."""
+
+    def __init__(self, S: int, pairs, rank: int | None = None, world: int | None = None, make_groups: bool = True):
+        self.rank = dist.get_rank() if rank is None else rank
+        self.M = dist.get_world_size() if world is None else world
+        if S % self.M != 0:
+            raise ValueError(f"S={S} is not a multiple of the world size {self.M}")
+        self.T = S // self.M
+        self.groups = {}
+        for w, r in pairs:
+            if w <= self.T:
+                if self.T % w != 0:
+                    raise ValueError(f"segment {w} does not divide the slice {self.T}")
+                continue
+            if w % self.T != 0 or S % w != 0:
+                raise ValueError(f"segment {w} is not a multiple of the slice {self.T} or does not divide S")
+            G = w // self.T
+            if G in self.groups:
+                continue
+            mine = None
+            for s in range(self.M // G):  # every rank creates every group, in the same order
+                ranks = list(range(s * G, (s + 1) * G))
+                grp = dist.new_group(ranks) if make_groups else ranks
+                if self.rank in ranks:
+                    mine = grp
+            self.groups[G] = mine
+
+    def seg_rank(self, w: int) -> int:
+        return self.rank % (w // self.T)
+
+
+def longnet_rows(T, w, r, o, g):
+    """(lp0, k_lo, n_rows, n_kept): rank g's kept rows of offset o in a segment
+    of w = G T tokens (the plain arithmetic of usp_longnet_rows)."""
+    a = g * T
+    p0 = a + (o - a) % r
+    n_rows = (a + T - p0 + r - 1) // r if p0 < a + T else 0
+    return p0 - a, (p0 - o) // r, n_rows, (w - o + r - 1) // r
+
+
+def _n_sel(Hq, r, o):
+    return (Hq - o + r - 1) // r
+
+
+def _gather_kept(k, v, w, r, o, Hq, lm: LongNetMesh, ops, comm):
+    """The kept K/V rows of offset o of the whole segment on every rank of it:
+    kc, vc [B, n_kept, n_sel, D] (head j = the kv head of query head o + j r)."""
+    B, T, Hkv, D = k.shape
+    Gq = Hq // Hkv
+    G = w // T
+    g = lm.seg_rank(w)
+    ns = _n_sel(Hq, r, o)
+    shares = [longnet_rows(T, w, r, o, x) for x in range(G)]
+    n_max = max(s[2] for s in shares)
+    n_kept = shares[0][3]
+    lp0, _, n_rows, _ = shares[g]
+    send = torch.empty((2, B, n_max, ns, D), dtype=k.dtype, device=k.device)
+    jobs = [dict(src=x, dst=send[c], dtype=ops.BF16, n_b=B, n_k=n_rows, n_j=ns, D=D,
+                 s_b=T * Hkv * D, s_k=Hkv * D, s_h=D, s_k0=lp0, s_kstep=r, s_h0=o, s_hstep=r, s_hdiv=Gq,
+                 d_b=n_max * ns * D, d_k=ns * D, d_h=D) for c, x in enumerate((k, v))]
+    ops.rows_copy(jobs)
+    recv = torch.empty((G,) + tuple(send.shape), dtype=k.dtype, device=k.device)
+    comm.all_gather(recv, send, lm.groups[G])
+    kc = torch.empty((B, n_kept, ns, D), dtype=k.dtype, device=k.device)
+    vc = torch.empty_like(kc)
+    jobs = []
+    for x, (_, k_lo, nr, _) in enumerate(shares):
+        for c, dst in enumerate((kc, vc)):
+            jobs.append(dict(src=recv[x, c], dst=dst, dtype=ops.BF16, n_b=B, n_k=nr, n_j=ns, D=D,
+                             s_b=n_max * ns * D, s_k=ns * D, s_h=D, d_b=n_kept * ns * D, d_k=ns * D, d_h=D,
+                             d_k0=k_lo))
+    for x in range(0, len(jobs), 16):
+        ops.rows_copy(jobs[x:x + 16])
+    return kc, vc, shares, n_max
+
+
+def longnet_attn_fwd(q, k, v, pairs, causal, lm: LongNetMesh, ops, comm=None):
+    """LongNet dilated attention of this rank's slice q [B, T, Hq, D], k, v
+    [B, T, Hkv, D]: returns (O bf16 [B, T, Hq, D], LSE fp32 [B, T, Hq]), equal to
+    rows [d T, (d + 1) T) of dilated attention over the whole sequence."""
+    comm = TorchComm() if comm is None else comm
+    Hq = q.shape[2]
+    ops.fwd_begin()
+    for w, r in pairs:
+        if w <= lm.T:
+            ops.fwd_local(q, k, v, causal, w, r)
+            continue
+        for o in range(min(r, Hq)):
+            kc, vc, _, _ = _gather_kept(k, v, w, r, o, Hq, lm, ops, comm)
+            ops.fwd_cross(q, kc, vc, causal, w, r, o, lm.seg_rank(w))
+    return ops.fwd_end()
+
+
+def longnet_attn_bwd(q, k, v, out, lse, dO, pairs, causal, lm: LongNetMesh, ops, comm=None):
+    """Backward of longnet_attn_fwd on this rank: (dQ bf16, dK fp32, dV fp32) of
+    its own slice. Gathered pairs gather the kept K/V rows again, compute this
+    rank's queries' share of their gradients and reduce-scatter them home."""
+    comm = TorchComm() if comm is None else comm
+    B, T, Hkv, D = k.shape
+    Hq = q.shape[2]
+    Gq = Hq // Hkv
+    dK = torch.empty((B, T, Hkv, D), dtype=torch.float32, device=k.device)
+    dV = torch.empty_like(dK)
+    ops.bwd_begin(out, lse, dO, dK, dV)
+    for w, r in pairs:
+        if w <= T:
+            ops.bwd_local(q, k, v, dO, lse, dK, dV, causal, w, r)
+            continue
+        G = w // T
+        for o in range(min(r, Hq)):
+            kc, vc, shares, n_max = _gather_kept(k, v, w, r, o, Hq, lm, ops, comm)
+            ns = kc.shape[2]
+            n_kept = kc.shape[1]
+            dkc = torch.empty(kc.shape, dtype=torch.float32, device=k.device)
+            dvc = torch.empty_like(dkc)
+            ops.bwd_cross(q, kc, vc, dO, lse, dkc, dvc, causal, w, r, o, lm.seg_rank(w))
+            send = torch.empty((G, 2, B, n_max, ns, D), dtype=torch.float32, device=k.device)
+            jobs = []
+            for x, (_, k_lo, nr, _) in enumerate(shares):
+                for c, src in enumerate((dkc, dvc)):
+                    jobs.append(dict(src=src, dst=send[x, c], dtype=ops.F32, n_b=B, n_k=nr, n_j=ns, D=D,
+                                     s_b=n_kept * ns * D, s_k=ns * D, s_h=D, s_k0=k_lo,
+                                     d_b=n_max * ns * D, d_k=ns * D, d_h=D))
+            for x in range(0, len(jobs), 16):
+                ops.rows_copy(jobs[x:x + 16])
+            recv = torch.empty((2, B, n_max, ns, D), dtype=torch.float32, device=k.device)
+            comm.reduce_scatter(recv, send, lm.groups[G])
+            lp0, _, nr, _ = shares[lm.seg_rank(w)]
+            ops.rows_copy([dict(src=recv[c], dst=dst, dtype=ops.F32, add=1, n_b=B, n_k=nr, n_j=ns, D=D,
+                                s_b=n_max * ns * D, s_k=ns * D, s_h=D,
+                                d_b=T * Hkv * D, d_k=Hkv * D, d_h=D, d_k0=lp0, d_kstep=r, d_h0=o, d_hstep=r,
+                                d_hdiv=Gq) for c, dst in enumerate((dK, dV))])
+    dq = ops.bwd_end()
+    return dq, dK, dV
+
+
+class CudaLongNetOps:
+    """The per-rank LongNet compute in libusp.so kernels."""
+
+    def __init__(self, B, T, Hq, Hkv, D, pairs, stream=None, device="cuda"):
+        from . import binding as B_
+        self.B_ = B_
+        self.BF16, self.F32 = B_.USP_BF16, B_.USP_F32
+        self.shape = (B, T, Hq, Hkv, D)
+        self.stream = stream
+        self.ws_f = torch.zeros(B_.usp_longnet_workspace_size(B, T, Hq, D, pairs, 0), dtype=torch.uint8,
+                                device=device)
+        self.ws_b = torch.zeros(B_.usp_longnet_workspace_size(B, T, Hq, D, pairs, 1), dtype=torch.uint8,
+                                device=device)
+        self.device = device
+
+    def rows_copy(self, jobs):
+        self.B_.usp_rows_copy(jobs, self.stream)
+
+    def fwd_begin(self):
+        B, T, Hq, Hkv, D = self.shape
+        self.B_.usp_longnet_fwd_begin(B, T, Hq, D, self.ws_f, self.ws_f.numel(), self.stream)
+
+    def fwd_local(self, q, k, v, causal, w, r):
+        B, T, Hq, Hkv, D = self.shape
+        self.B_.usp_longnet_fwd_local(q, k, v, B, T, Hq, Hkv, D, causal, w, r, self.ws_f, self.ws_f.numel(),
+                                      self.stream)
+
+    def fwd_cross(self, q, kc, vc, causal, w, r, o, g):
+        B, T, Hq, Hkv, D = self.shape
+        self.B_.usp_longnet_fwd_cross(q, kc, vc, B, T, Hq, Hkv, D, causal, w, r, o, g, self.ws_f, self.ws_f.numel(),
+                                      self.stream)
+
+    def fwd_end(self):
+        B, T, Hq, Hkv, D = self.shape
+        out = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=self.device)
+        lse = torch.empty((B, T, Hq), dtype=torch.float32, device=self.device)
+        self.B_.usp_longnet_fwd_end(out, lse, B, T, Hq, D, self.ws_f, self.ws_f.numel(), self.stream)
+        return out, lse
+
+    def bwd_begin(self, out, lse, dO, dK, dV):
+        B, T, Hq, Hkv, D = self.shape
+        self.B_.usp_longnet_bwd_begin(out, lse, dO, dK, dV, B, T, Hq, Hkv, D, self.ws_b, self.ws_b.numel(),
+                                      self.stream)
+
+    def bwd_local(self, q, k, v, dO, lse, dK, dV, causal, w, r):
+        B, T, Hq, Hkv, D = self.shape
+        self.B_.usp_longnet_bwd_local(q, k, v, dO, lse, dK, dV, B, T, Hq, Hkv, D, causal, w, r, self.ws_b,
+                                      self.ws_b.numel(), self.stream)
+
+    def bwd_cross(self, q, kc, vc, dO, lse, dkc, dvc, causal, w, r, o, g):
+        B, T, Hq, Hkv, D = self.shape
+        self.B_.usp_longnet_bwd_cross(q, kc, vc, dO, lse, dkc, dvc, B, T, Hq, Hkv, D, causal, w, r, o, g, self.ws_b,
+                                      self.ws_b.numel(), self.stream)
+
+    def bwd_end(self):
+        B, T, Hq, Hkv, D = self.shape
+        dq = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=self.device)
+        self.B_.usp_longnet_bwd_end(dq, B, T, Hq, D, self.ws_b, self.ws_b.numel(), self.stream)
+        return dq
+
+    def check(self):
+        for ws in (self.ws_f, self.ws_b):
+            rc, site = self.B_.usp_workspace_status(ws, self.stream)
+            if rc != self.B_.USP_OK:
+                raise self.B_.UspError(rc, f"device wait timed out (site {site:#x})")

@@ -33,6 +33,25 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(B_.SIGNATURES), "binding must mirror the header"
 
 
+def declared_arities():
+    """usp_* name -> number of parameters in its include/usp.h prototype."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(usp_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_arities_match_the_header():
+    """Every ctypes signature takes exactly the prototype's parameters (a missing
+    or extra argument would shift every later one)."""
+    ar = declared_arities()
+    assert set(ar) == set(B_.SIGNATURES)
+    for name, (_, args) in B_.SIGNATURES.items():
+        assert len(args) == ar[name], (name, len(args), ar[name])
+
+
 def test_version_and_empty_error():
     assert B_.usp_version() >= 100
     assert isinstance(B_.usp_last_error(), str)
