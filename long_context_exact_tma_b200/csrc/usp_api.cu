@@ -168,6 +168,55 @@ int make_tmap_strided_h(CUtensorMap* m, const void* base, int D, int H, long lon
   return USP_OK;
 }
 unsigned long long current_wait_ns() { return g_wait_ns; }
+
+namespace {
+struct SidePool {
+  int dev = -1;
+  cudaStream_t s[kSideStreams];
+  cudaEvent_t fork;
+  cudaEvent_t join[kSideStreams];
+};
+thread_local SidePool t_side;
+
+cudaError_t side_pool(SidePool** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  SidePool& p = t_side;
+  if (p.dev != dev) {  // first use on this device by this thread
+    for (int i = 0; i < kSideStreams && e == cudaSuccess; ++i) {
+      e = cudaStreamCreateWithFlags(&p.s[i], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.join[i], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    p.dev = dev;
+  }
+  *out = &p;
+  return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t side_fork(cudaStream_t main, int n, cudaStream_t* out) {
+  SidePool* p = nullptr;
+  cudaError_t e = side_pool(&p);
+  if (e == cudaSuccess) e = cudaEventRecord(p->fork, main);
+  for (int i = 0; i < n && i < kSideStreams && e == cudaSuccess; ++i) {
+    e = cudaStreamWaitEvent(p->s[i], p->fork, 0);
+    out[i] = p->s[i];
+  }
+  return e;
+}
+
+cudaError_t side_join(cudaStream_t main, int n) {
+  SidePool* p = nullptr;
+  cudaError_t e = side_pool(&p);
+  for (int i = 0; i < n && i < kSideStreams && e == cudaSuccess; ++i) {
+    e = cudaEventRecord(p->join[i], p->s[i]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(main, p->join[i], 0);
+  }
+  return e;
+}
 }  // namespace usp
 
 namespace {

@@ -50,7 +50,17 @@ int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S,
   L.step = -1;
   const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;  // bytes per token row
   const int n_seg = S / wp;
-  for (int off = 0; off < rp && off < Hq; ++off) {
+  // the offsets write disjoint heads of the running result: their (often small)
+  // launches run side by side
+  const int n_off = rp < Hq ? rp : Hq;
+  const int n_st = n_off > 1 ? (n_off < kSideStreams ? n_off : kSideStreams) : 0;
+  cudaStream_t side[kSideStreams];
+  if (n_st) {
+    const cudaError_t e = side_fork(st, n_st, side);
+    if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "side streams: %s", cudaGetErrorString(e));
+  }
+  int rc = USP_OK;
+  for (int off = 0; off < n_off && rc == USP_OK; ++off) {
     const int kept = (wp - off + rp - 1) / rp;  // rows of a segment at offset off
     g.L = kept;
     g.c = kept;  // unused in the sub-problem mode
@@ -70,19 +80,23 @@ int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S,
     sb.o_run = o_run;
     sb.lse_run = lse_run;
     sub_defaults(sb, Hkv);
-    int rc = make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, kept, sb.n_prob,
-                               rp * tokq, wp * tokq);
+    rc = make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, kept, sb.n_prob, rp * tokq,
+                           wp * tokq);
     if (rc == USP_OK)
       rc = make_tmap_strided(&L.tm_k, static_cast<const uint8_t*>(k) + off * tokkv, D, Hkv, kept, sb.n_prob,
                              rp * tokkv, wp * tokkv);
     if (rc == USP_OK)
       rc = make_tmap_strided(&L.tm_v, static_cast<const uint8_t*>(v) + off * tokkv, D, Hkv, kept, sb.n_prob,
                              rp * tokkv, wp * tokkv);
-    if (rc != USP_OK) return rc;
-    const cudaError_t e = launch_attn_fwd(L, st);
-    if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated attention launch: %s", cudaGetErrorString(e));
+    if (rc != USP_OK) break;
+    const cudaError_t e = launch_attn_fwd(L, n_st ? side[off % n_st] : st);
+    if (e != cudaSuccess) rc = record_error(USP_ERR_CUDA, "dilated attention launch: %s", cudaGetErrorString(e));
   }
-  return USP_OK;
+  if (n_st) {
+    const cudaError_t e = side_join(st, n_st);
+    if (e != cudaSuccess && rc == USP_OK) rc = record_error(USP_ERR_CUDA, "side streams: %s", cudaGetErrorString(e));
+  }
+  return rc;
 }
 
 }  // namespace usp
@@ -153,8 +167,9 @@ DilatedLaunchShape launch_shape(int S, int Hq, int w, int r, int off) {
 
 namespace usp {
 
-size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r) {
-  size_t tbl = 0;  // the largest per-launch table: n_prob * n_heads * Lp floats
+// Floats of one row-table slot: the largest launch's n_prob * n_heads * Lp.
+size_t slot_floats(int B, int S, int Hq, int w, int r) {
+  size_t tbl = 0;
   for (int off = 0; off < r && off < Hq; ++off) {
     const DilatedLaunchShape sh = launch_shape(S, Hq, w, r, off);
     const size_t Lp = static_cast<size_t>((sh.kept + 127) / 128 * 128);
@@ -162,6 +177,10 @@ size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r) {
     if (n > tbl) tbl = n;
   }
   return tbl;
+}
+
+size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r) {
+  return kSideStreams * slot_floats(B, S, Hq, w, r);
 }
 
 int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO, const float* lse,
@@ -183,8 +202,23 @@ int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO
   L.dq = nullptr;
   L.dq_acc = dq_acc;
   const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;
-  for (int off = 0; off < rp && off < Hq; ++off) {
+  // With Hq == Hkv the offsets write disjoint dK/dV heads as well as dQ heads:
+  // side streams, each with its own row-table slot.
+  const int n_off = rp < Hq ? rp : Hq;
+  const int n_st = (n_off > 1 && Hq == Hkv) ? (n_off < kSideStreams ? n_off : kSideStreams) : 0;
+  const size_t slot = slot_floats(B, S, Hq, wp, rp);
+  cudaStream_t side[kSideStreams];
+  if (n_st) {
+    const cudaError_t e = side_fork(st, n_st, side);
+    if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "side streams: %s", cudaGetErrorString(e));
+  }
+  int rc = USP_OK;
+  for (int off = 0; off < n_off && rc == USP_OK; ++off) {
     const DilatedLaunchShape sh = launch_shape(S, Hq, wp, rp, off);
+    const int ks = n_st ? off % n_st : 0;  // stream and row-table slot
+    cudaStream_t os = n_st ? side[ks] : st;
+    L.lse2 = lse2_t + ks * slot;
+    L.delta = delta_t + ks * slot;
     FwdSub& sb = L.sub;
     sb.active = 1;
     sb.n_prob = B * sh.n_seg;
@@ -202,8 +236,8 @@ int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO
     g.L = sh.kept;
     g.c = sh.kept;
     L.Lp = (sh.kept + 127) / 128 * 128;
-    int rc = make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, sh.kept, sb.n_prob,
-                               rp * tokq, wp * tokq);
+    rc = make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, sh.kept, sb.n_prob,
+                           rp * tokq, wp * tokq);
     if (rc == USP_OK)
       rc = make_tmap_strided(&L.tm_do, static_cast<const uint8_t*>(dO) + off * tokq, D, Hq, sh.kept, sb.n_prob,
                              rp * tokq, wp * tokq);
@@ -213,13 +247,17 @@ int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO
     if (rc == USP_OK)
       rc = make_tmap_strided(&L.tm_v, static_cast<const uint8_t*>(v) + off * tokkv, D, Hkv, sh.kept, sb.n_prob,
                              rp * tokkv, wp * tokkv);
-    if (rc != USP_OK) return rc;
-    cudaError_t e = launch_dilated_tables(lse, delta_all, lse2_t, delta_t, sb, L.Lp, st);
-    if (e == cudaSuccess) e = launch_attn_bwd(L, st);
-    if (e == cudaSuccess) e = launch_attn_bwd_dq(L, st);
-    if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated backward launch: %s", cudaGetErrorString(e));
+    if (rc != USP_OK) break;
+    cudaError_t e = launch_dilated_tables(lse, delta_all, lse2_t + ks * slot, delta_t + ks * slot, sb, L.Lp, os);
+    if (e == cudaSuccess) e = launch_attn_bwd(L, os);
+    if (e == cudaSuccess) e = launch_attn_bwd_dq(L, os);
+    if (e != cudaSuccess) rc = record_error(USP_ERR_CUDA, "dilated backward launch: %s", cudaGetErrorString(e));
   }
-  return USP_OK;
+  if (n_st) {
+    const cudaError_t e = side_join(st, n_st);
+    if (e != cudaSuccess && rc == USP_OK) rc = record_error(USP_ERR_CUDA, "side streams: %s", cudaGetErrorString(e));
+  }
+  return rc;
 }
 
 }  // namespace usp

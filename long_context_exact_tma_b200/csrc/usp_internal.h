@@ -18,6 +18,15 @@ void note_launch();
 // The calling thread's bounded-wait limit (usp_set_wait_limit_ns).
 unsigned long long current_wait_ns();
 
+// Streams of the calling thread on the current device for launches that may
+// run at the same time: side_fork makes n (<= kSideStreams) of them wait for
+// the work issued so far on `main` and returns them; side_join makes `main`
+// wait for everything issued on them since. Created on first use, kept for the
+// thread's life (one set per thread, so concurrent callers never share an event).
+constexpr int kSideStreams = 4;
+cudaError_t side_fork(cudaStream_t main, int n, cudaStream_t* out);
+cudaError_t side_join(cudaStream_t main, int n);
+
 struct AttnGeom;
 // The shape checks of the attention calls; fills g; usp_status (message recorded).
 int validate_geom(int B, int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, AttnGeom* g);
@@ -176,7 +185,9 @@ cudaError_t launch_attn_bwd_dq(const BwdLaunch& a, cudaStream_t stream);  // dQ 
 // folds the pair's result into the running fp32 (O, LSE); the backward adds the
 // pair's dQ (into the fp32 dq_acc), dK and dV (fp32), with the final LSE and
 // Delta of every row and two row-table buffers of dilated_pair_table_floats
-// floats each. usp_status.
+// floats each (kSideStreams slots: the offsets of a pair write disjoint heads,
+// so their launches run on side streams at the same time; in the backward only
+// when Hq == Hkv, whose offsets also write disjoint kv heads). usp_status.
 int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S, int Hq, int Hkv, int D, int causal,
                       int w, int r, float* o_run, float* lse_run, int* status, cudaStream_t st);
 size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r);
