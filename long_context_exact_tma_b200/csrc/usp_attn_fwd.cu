@@ -341,56 +341,133 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         __syncwarp();
         mbar_arrive_w(&bars->desc_full[t]);
       };
-      bool ok = mbar_wait_w(&bars->k_full[0], 0, w, kSiteK);
-      const bool have = ok && bars->step[0][0] >= 0;
-      bool issued_any = false;
-      if (ok && !have) {
-        publish(0, nullptr);
-        publish(1, nullptr);
-      }
-      if (have) ok = mbar_wait_w(&bars->q_full, 0, w, kSiteQ);
-      if (ok && have) {
-        tc_fence_after();
-        publish(0, bars->step[0]);
-        publish(1, bars->step[0]);
-        issue_s(0, 0);
-        issue_s(1, 0);
-        umma_commit_w(&bars->k_empty[0]);
-        issued_any = true;
-      }
-      // Per key tile `it`, per query tile t in turn: O_t += P_t V, then S_t of
-      // tile it+1 (which overwrites P_t, so it waits for that PV to land). The
-      // softmax of one query tile thus overlaps the other tile's PV and S.
-      for (int it = 0; ok && have; ++it) {
-        const int s = it % C::kVSt;
-        const int s1 = (it + 1) % C::kKSt;
-        if (!mbar_wait_w(&bars->v_full[s], (it / C::kVSt) & 1, w, kSiteV)) { ok = false; break; }
-        const uint64_t vd = dV0 + ((s * C::kTileBytes) >> 4);
-        bool next = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!mbar_wait_w(&bars->p_full[t], it & 1, w, kSiteP)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-          umma_commit_w(&bars->pv_done[t]);
-          if (t == 1) umma_commit_w(&bars->v_empty[s]);
-          if (t == 0) {
-            if (!mbar_wait_w(&bars->k_full[s1], ((it + 1) / C::kKSt) & 1, w, kSiteK)) { ok = false; break; }
-            next = bars->step[(it + 1) & 3][0] >= 0;
-          }
-          if (next) {
-            if (!mbar_wait_w(&bars->pv_done[t], it & 1, w, kSitePvDone)) { ok = false; break; }
-            tc_fence_after();
-            publish(t, bars->step[(it + 1) & 3]);
-            issue_s(t, s1);
-            if (t == 1) umma_commit_w(&bars->k_empty[s1]);
-          } else {
-            publish(t, nullptr);
-          }
+      bool ok = true, issued_any = false;
+      if constexpr (kMask) {
+        // A query tile whose kind for a key tile is skip gets neither S nor PV of
+        // it, and its softmax warps never see the tile (the walk only holds tiles
+        // that at least one of the two query tiles attends). Each query tile counts
+        // its own products: npv[t] PV issued; the parities of its barriers follow.
+        auto attends = [](const int* slot, int t) { return ((slot[3] >> (4 * t)) & 15) != kSkip; };
+        int npv[2] = {0, 0};
+        bool pv_wait[2] = {false, false};  // a PV_t issued whose completion has not been waited for
+        ok = mbar_wait_w(&bars->k_full[0], 0, w, kSiteK);
+        const bool have = ok && bars->step[0][0] >= 0;
+        if (ok && !have) {
+          publish(0, nullptr);
+          publish(1, nullptr);
         }
-        if (!ok || !next) break;
+        if (have) ok = mbar_wait_w(&bars->q_full, 0, w, kSiteQ);
+        if (ok && have) {
+          tc_fence_after();
+          const int* sl = bars->step[0];
+          for (int t = 0; t < 2; ++t) {
+            if (!attends(sl, t)) continue;
+            publish(t, sl);
+            issue_s(t, 0);
+          }
+          umma_commit_w(&bars->k_empty[0]);
+          issued_any = true;
+        }
+        // Per key tile `it`, per query tile t in turn: O_t += P_t V, then S_t of
+        // tile it+1 (which overwrites P_t, so it waits for that PV to land). The
+        // softmax of one query tile thus overlaps the other tile's PV and S.
+        for (int it = 0; ok && have; ++it) {
+          const int s = it % C::kVSt;
+          const int s1 = (it + 1) % C::kKSt;
+          const int* cur = bars->step[it & 3];
+          const bool att1 = attends(cur, 1);
+          if (!mbar_wait_w(&bars->v_full[s], (it / C::kVSt) & 1, w, kSiteV)) { ok = false; break; }
+          const uint64_t vd = dV0 + ((s * C::kTileBytes) >> 4);
+          bool next = false;
+          const int* nxt = nullptr;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (attends(cur, t)) {
+              if (!mbar_wait_w(&bars->p_full[t], npv[t] & 1, w, kSiteP)) { ok = false; break; }
+              tc_fence_after();
+  #pragma unroll
+              for (int kk = 0; kk < kBN / 16; ++kk)
+                umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                                   (npv[t] > 0 || kk > 0) ? 1u : 0u);
+              umma_commit_w(&bars->pv_done[t]);
+              ++npv[t];
+              pv_wait[t] = true;
+              if (t == 1 || !att1) umma_commit_w(&bars->v_empty[s]);  // the tile's last PV
+            }
+            if (t == 0) {
+              if (!mbar_wait_w(&bars->k_full[s1], ((it + 1) / C::kKSt) & 1, w, kSiteK)) { ok = false; break; }
+              nxt = bars->step[(it + 1) & 3];
+              next = nxt[0] >= 0;
+            }
+            if (next) {
+              if (attends(nxt, t)) {
+                if (pv_wait[t]) {
+                  if (!mbar_wait_w(&bars->pv_done[t], (npv[t] - 1) & 1, w, kSitePvDone)) { ok = false; break; }
+                  pv_wait[t] = false;
+                }
+                tc_fence_after();
+                publish(t, nxt);
+                issue_s(t, s1);
+              }
+              if (t == 1) umma_commit_w(&bars->k_empty[s1]);  // after the tile's S
+            } else {
+              publish(t, nullptr);
+            }
+          }
+          if (!ok || !next) break;
+        }
+      } else {
+        // (no skip tiles to speak of without a mask: the plain loop, which
+        // measured faster than the counting one above on dense causal work)
+        ok = mbar_wait_w(&bars->k_full[0], 0, w, kSiteK);
+        const bool have = ok && bars->step[0][0] >= 0;
+        if (ok && !have) {
+          publish(0, nullptr);
+          publish(1, nullptr);
+        }
+        if (have) ok = mbar_wait_w(&bars->q_full, 0, w, kSiteQ);
+        if (ok && have) {
+          tc_fence_after();
+          publish(0, bars->step[0]);
+          publish(1, bars->step[0]);
+          issue_s(0, 0);
+          issue_s(1, 0);
+          umma_commit_w(&bars->k_empty[0]);
+          issued_any = true;
+        }
+        // Per key tile `it`, per query tile t in turn: O_t += P_t V, then S_t of
+        // tile it+1 (which overwrites P_t, so it waits for that PV to land). The
+        // softmax of one query tile thus overlaps the other tile's PV and S.
+        for (int it = 0; ok && have; ++it) {
+          const int s = it % C::kVSt;
+          const int s1 = (it + 1) % C::kKSt;
+          if (!mbar_wait_w(&bars->v_full[s], (it / C::kVSt) & 1, w, kSiteV)) { ok = false; break; }
+          const uint64_t vd = dV0 + ((s * C::kTileBytes) >> 4);
+          bool next = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!mbar_wait_w(&bars->p_full[t], it & 1, w, kSiteP)) { ok = false; break; }
+            tc_fence_after();
+  #pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                                 (it > 0 || kk > 0) ? 1u : 0u);
+            umma_commit_w(&bars->pv_done[t]);
+            if (t == 1) umma_commit_w(&bars->v_empty[s]);
+            if (t == 0) {
+              if (!mbar_wait_w(&bars->k_full[s1], ((it + 1) / C::kKSt) & 1, w, kSiteK)) { ok = false; break; }
+              next = bars->step[(it + 1) & 3][0] >= 0;
+            }
+            if (next) {
+              if (!mbar_wait_w(&bars->pv_done[t], it & 1, w, kSitePvDone)) { ok = false; break; }
+              tc_fence_after();
+              publish(t, bars->step[(it + 1) & 3]);
+              issue_s(t, s1);
+              if (t == 1) umma_commit_w(&bars->k_empty[s1]);
+            } else {
+              publish(t, nullptr);
+            }
+          }
+          if (!ok || !next) break;
+        }
       }
       if (!ok && issued_any) {
         umma_commit_w(&bars->drain);
