@@ -457,6 +457,7 @@ def per_workload(dev, peak_tf, peak_hbm):
         del rm, hs
         torch.cuda.empty_cache()
     res.update(variants_per_workload(dev, peak_tf))
+    res.update(rank_per_workload(dev, peak_tf))
     return res
 
 
@@ -519,6 +520,153 @@ def variants_per_workload(dev, peak_tf):
         "bwd": {"TFLOP/s": round(2.5 * fl / ms_b / 1e9, 1), "frac_of_peak": round(2.5 * fl / ms_b / 1e9 / peak_tf, 4),
                 "ms": round(ms_b, 3)}}
     del qh, kh, vh, doh, o, l, bmd
+    torch.cuda.empty_cache()
+    return res
+
+
+def rank_per_workload(dev, peak_tf):
+    """Event-timed per-rank compute of the two multi-GPU layouts, on one GPU
+    (the collectives between the calls are not part of it):
+      - one rank of a real USP mesh: ring rank 0 of the S=16K ring-8 workload
+        runs its 8 ring steps (usp_ring_fwd_step, each partial folded by
+        usp_lse_merge) and the backward steps (usp_ring_bwd_prepare +
+        usp_ring_bwd_step) against 8 resident K/V blocks;
+      - rank 0 of LongNet's distributed layout over 4 ranks on the S=32K
+        dilated schedule: its local pairs and, for the gathered pairs, the cross
+        attention of its kept rows against the segment's kept K/V rows (gathered
+        beforehand by usp_rows_copy from the whole sequence, as the all-gather
+        would deliver them), forward and backward.
+    FLOPs are those of the rank's visible (query, key) pairs."""
+    from long_context_exact_tma_b200 import binding as B_
+    from long_context_exact_tma_b200 import dist as udist
+    from usp_inputs import normal_bf16
+    res = {}
+    # -- one rank of the USP mesh (ring 8, S=16K)
+    w = dict(WORKLOADS[2])
+    B, S, Hq, Hkv, D, P_u, P_r = w["B"], w["S"], w["Hq"], w["Hkv"], w["D"], w["P_u"], w["P_r"]
+    causal, L = w["causal"], w["S"] // w["P_r"]
+    P, c = P_u * P_r, S // (2 * P_u * P_r)
+    q = normal_bf16(950, (B, L, Hq, D), device=dev)
+    do = normal_bf16(951, (B, L, Hq, D), device=dev)
+    ks = [normal_bf16(960 + j, (B, L, Hkv, D), device=dev) for j in range(P_r)]
+    vs = [normal_bf16(980 + j, (B, L, Hkv, D), device=dev) for j in range(P_r)]
+    pos0 = [x for r_ in (0, 2 * P - 1) for x in range(r_ * c, (r_ + 1) * c)]  # ring rank 0's zigzag positions
+    vis = sum(p + 1 for p in pos0) if causal else len(pos0) * S
+    fl = 4.0 * D * B * Hq * vis
+    rows = B * L * Hq
+    wsf = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 0), dtype=torch.uint8,
+                      device=dev)
+    wsb = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 1), dtype=torch.uint8,
+                      device=dev)
+    o_parts = torch.empty((2, rows, D), dtype=torch.float32, device=dev)
+    l_parts = torch.empty((2, rows), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, L, Hq), dtype=torch.float32, device=dev)
+
+    def ring_fwd():
+        for t in range(P_r):
+            j = (0 - t) % P_r
+            B_.usp_ring_fwd_step(q, ks[j], vs[j], o_parts[0 if t == 0 else 1], l_parts[0 if t == 0 else 1], B, S, Hq,
+                                 Hkv, D, causal, P_u, P_r, 0, 0, t, wsf, wsf.numel())
+            if t > 0:
+                B_.usp_lse_merge(o_parts, l_parts, 2, rows, D, o_parts[0], B_.USP_F32, l_parts[0])
+        B_.usp_lse_merge(o_parts[:1], l_parts[:1], 1, rows, D, out, B_.USP_BF16, lse)
+
+    ring_fwd()
+    dq_acc = torch.zeros((B, L, Hq, D), dtype=torch.float32, device=dev)
+    dq = torch.empty_like(q)
+    dk = torch.zeros((B, L, Hkv, D), dtype=torch.float32, device=dev)
+    dv = torch.zeros_like(dk)
+
+    def ring_bwd():
+        B_.usp_ring_bwd_prepare(out, lse, do, B, S, Hq, Hkv, D, causal, P_u, P_r, wsb, wsb.numel())
+        for t in range(P_r):
+            j = (0 - t) % P_r
+            B_.usp_ring_bwd_step(q, ks[j], vs[j], do, dq_acc, dq if t == P_r - 1 else None, dk, dv, B, S, Hq, Hkv, D,
+                                 causal, P_u, P_r, 0, 0, t, wsb, wsb.numel())
+
+    ms_f, ms_b = _time_pair(ring_fwd, ring_bwd, reps=10)
+    for ws in (wsf, wsb):
+        rc, site = B_.usp_workspace_status(ws)
+        if rc != B_.USP_OK:
+            raise B_.UspError(rc, f"device wait timed out (site {site:#x})")
+    res["usp_rank_s16k_ring8"] = {
+        "shape": "ring rank 0 of the S=16K ring-8 workload: 8 ring steps against resident K/V blocks (no NCCL)",
+        "fwd": {"TFLOP/s": round(fl / ms_f / 1e9, 1), "frac_of_peak": round(fl / ms_f / 1e9 / peak_tf, 4),
+                "ms": round(ms_f, 3)},
+        "bwd": {"TFLOP/s": round(2.5 * fl / ms_b / 1e9, 1), "frac_of_peak": round(2.5 * fl / ms_b / 1e9 / peak_tf, 4),
+                "ms": round(ms_b, 3)}}
+    del q, do, ks, vs, o_parts, l_parts, out, lse, dq_acc, dq, dk, dv, wsf, wsb
+    # -- rank 0 of LongNet's distributed layout, 4 ranks, S=32K
+    B, S, H, D, M = 1, 32768, 16, 128, 4
+    T = S // M
+    pairs = [(2048, 1), (4096, 2), (8192, 4), (16384, 6), (32768, 12)]
+    qg, kg, vg, dog = (normal_bf16(900 + x, (B, S, H, D), device=dev) for x in range(4))
+    q, k, v, do = (x[:, :T].contiguous() for x in (qg, kg, vg, dog))
+    ops = udist.CudaLongNetOps(B, T, H, H, D, pairs, device=dev)
+    gathered = {}
+    vis = 0
+    for w_, r in pairs:
+        for h in range(H):
+            o = h % r
+            if w_ <= T:  # every segment of the slice, causal among its kept rows
+                kept = (w_ - o + r - 1) // r
+                vis += (T // w_) * kept * (kept + 1) // 2
+            else:  # rank 0 holds the first kept rows of its segment
+                _, k_lo, n_rows, _ = udist.longnet_rows(T, w_, r, o, 0)
+                vis += sum(k_lo + x + 1 for x in range(n_rows))
+        if w_ <= T:
+            continue
+        for o in range(min(r, H)):
+            ns = (H - o + r - 1) // r
+            n_kept = (w_ - o + r - 1) // r
+            kc = torch.empty((B, n_kept, ns, D), dtype=torch.bfloat16, device=dev)
+            vc = torch.empty_like(kc)
+            # the segment's kept rows of the kv heads of query heads o, o + r, ..., in kept order
+            B_.usp_rows_copy([dict(src=x, dst=y, dtype=B_.USP_BF16, n_b=B, n_k=n_kept, n_j=ns, D=D, s_b=S * H * D,
+                                   s_k=H * D, s_h=D, s_k0=o, s_kstep=r, s_h0=o, s_hstep=r, d_b=n_kept * ns * D,
+                                   d_k=ns * D, d_h=D) for x, y in ((kg, kc), (vg, vc))])
+            gathered[(w_, r, o)] = (kc, vc, torch.empty(kc.shape, dtype=torch.float32, device=dev),
+                                    torch.empty(kc.shape, dtype=torch.float32, device=dev))
+    fl = 4.0 * D * B * vis
+    state = {}
+
+    def ln_fwd():
+        ops.fwd_begin()
+        for w_, r in pairs:
+            if w_ <= T:
+                ops.fwd_local(q, k, v, True, w_, r)
+            else:
+                for o in range(min(r, H)):
+                    kc, vc, _, _ = gathered[(w_, r, o)]
+                    ops.fwd_cross(q, kc, vc, True, w_, r, o, 0)
+        state["out"], state["lse"] = ops.fwd_end()
+
+    ln_fwd()
+    dK = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
+    dV = torch.empty_like(dK)
+
+    def ln_bwd():
+        ops.bwd_begin(state["out"], state["lse"], do, dK, dV)
+        for w_, r in pairs:
+            if w_ <= T:
+                ops.bwd_local(q, k, v, do, state["lse"], dK, dV, True, w_, r)
+            else:
+                for o in range(min(r, H)):
+                    kc, vc, dkc, dvc = gathered[(w_, r, o)]
+                    ops.bwd_cross(q, kc, vc, do, state["lse"], dkc, dvc, True, w_, r, o, 0)
+        ops.bwd_end()
+
+    ms_f, ms_b = _time_pair(ln_fwd, ln_bwd, reps=5)
+    ops.check()
+    res["longnet_rank_s32k_4ranks"] = {
+        "shape": "rank 0 of 4 (T=8192) on the S=32K dilated schedule H=16 D=128 causal; gathered pairs "
+                 "(16384,6) (32768,12) from pre-gathered kept K/V rows (no NCCL)",
+        "fwd": {"TFLOP/s": round(fl / ms_f / 1e9, 1), "frac_of_peak": round(fl / ms_f / 1e9 / peak_tf, 4),
+                "ms": round(ms_f, 3)},
+        "bwd": {"TFLOP/s": round(2.5 * fl / ms_b / 1e9, 1), "frac_of_peak": round(2.5 * fl / ms_b / 1e9 / peak_tf, 4),
+                "ms": round(ms_b, 3)}}
+    del qg, kg, vg, dog, q, k, v, do, gathered, dK, dV, state, ops
     torch.cuda.empty_cache()
     return res
 
