@@ -528,8 +528,8 @@ def rank_per_workload(dev, peak_tf):
     """Event-timed per-rank compute of the two multi-GPU layouts, on one GPU
     (the collectives between the calls are not part of it):
       - one rank of a real USP mesh: ring rank 0 of the S=16K ring-8 workload
-        runs its 8 ring steps (usp_ring_fwd_step, each partial folded by
-        usp_lse_merge) and the backward steps (usp_ring_bwd_prepare +
+        runs its 8 ring steps (usp_ring_fwd_accumulate: each step's partial
+        folded into a running one in the kernel) and the backward steps (usp_ring_bwd_prepare +
         usp_ring_bwd_step) against 8 resident K/V blocks;
       - rank 0 of LongNet's distributed layout over 4 ranks on the S=32K
         dilated schedule: its local pairs and, for the gathered pairs, the cross
@@ -563,13 +563,11 @@ def rank_per_workload(dev, peak_tf):
     out = torch.empty_like(q)
     lse = torch.empty((B, L, Hq), dtype=torch.float32, device=dev)
 
-    def ring_fwd():
+    def ring_fwd():  # each step folded into the running partial in the kernel's epilogue
         for t in range(P_r):
             j = (0 - t) % P_r
-            B_.usp_ring_fwd_step(q, ks[j], vs[j], o_parts[0 if t == 0 else 1], l_parts[0 if t == 0 else 1], B, S, Hq,
-                                 Hkv, D, causal, P_u, P_r, 0, 0, t, wsf, wsf.numel())
-            if t > 0:
-                B_.usp_lse_merge(o_parts, l_parts, 2, rows, D, o_parts[0], B_.USP_F32, l_parts[0])
+            B_.usp_ring_fwd_accumulate(q, ks[j], vs[j], o_parts[0], l_parts[0], B, S, Hq, Hkv, D, causal, P_u, P_r,
+                                       0, 0, t, wsf, wsf.numel())
         B_.usp_lse_merge(o_parts[:1], l_parts[:1], 1, rows, D, out, B_.USP_BF16, lse)
 
     ring_fwd()

@@ -265,6 +265,13 @@ int usp_attn_bwd_masked(const void* q, const void* k, const void* v, const void*
  * (rows that see no key of the block: LSE = -inf, O = 0). Fold the partials
  * with usp_lse_merge (in place into a running fp32 result). Workspace 256 B.
  *
+ * usp_ring_fwd_accumulate: the same step, folded into a running fp32 result
+ * instead: step t = 0 writes o_run / lse_run ([B][L][Hq/P_u][D], [B][L][Hq/P_u])
+ * like usp_ring_fwd_step; every later step merges its partial into them by the
+ * log-sum-exp merge in the kernel's epilogue (one buffer, no merge launch).
+ * Call it for t = 0, 1, ... in order; usp_lse_merge with n_parts = 1 then
+ * writes the bf16 O and the LSE.
+ *
  * usp_ring_bwd_prepare: the per-head -LSE*log2(e) and -Delta tables of the
  * rank's rows from its final out, lse and dO (workspace of
  * usp_ring_workspace_size(..., bwd = 1)).
@@ -283,6 +290,9 @@ size_t usp_ring_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal,
 int usp_ring_fwd_step(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int S,
                       int Hq, int Hkv, int D, int causal, int P_u, int P_r, int i, int u, int t, void* workspace,
                       size_t ws_bytes, void* stream);
+int usp_ring_fwd_accumulate(const void* q, const void* k, const void* v, float* o_run, float* lse_run, int B, int S,
+                            int Hq, int Hkv, int D, int causal, int P_u, int P_r, int i, int u, int t,
+                            void* workspace, size_t ws_bytes, void* stream);
 int usp_ring_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,
                          int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream);
 int usp_ring_bwd_step(const void* q, const void* k, const void* v, const void* dO, float* dq_acc, void* dq_out,

@@ -79,6 +79,7 @@ SIGNATURES = {
     "usp_ulysses_pack": (_I, [_I, ctypes.POINTER(PermuteJob), _I, _I, _I, _I, _P]),
     "usp_ring_workspace_size": (_SZ, [_I] * 9),
     "usp_ring_fwd_step": (_I, [_P] * 5 + [_I] * 11 + [_P, _SZ, _P]),
+    "usp_ring_fwd_accumulate": (_I, [_P] * 5 + [_I] * 11 + [_P, _SZ, _P]),
     "usp_ring_bwd_prepare": (_I, [_P] * 3 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_ring_bwd_step": (_I, [_P] * 8 + [_I] * 11 + [_P, _SZ, _P]),
     "usp_dilated_workspace_size": (_SZ, [_I] * 4),
@@ -217,6 +218,13 @@ def usp_ring_fwd_step(q, k, v, o_part, lse_part, B, S, Hq, Hkv, D, causal, P_u, 
                       stream=None, check=True):
     rc = lib().usp_ring_fwd_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, S, Hq, Hkv, D,
                                  int(causal), P_u, P_r, i, u, t, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_ring_fwd_accumulate(q, k, v, o_run, lse_run, B, S, Hq, Hkv, D, causal, P_u, P_r, i, u, t, workspace,
+                            ws_bytes, stream=None, check=True):
+    rc = lib().usp_ring_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o_run), _ptr(lse_run), B, S, Hq, Hkv, D,
+                                       int(causal), P_u, P_r, i, u, t, _ptr(workspace), ws_bytes, _stream(stream))
     return _check(rc) if check else rc
 
 

@@ -78,6 +78,7 @@ struct FwdArgs {
   unsigned long long wait_ns;
   FwdSub sub;  // sub-problem mode (kSub): see usp_internal.h
   int loc_i, loc_u;  // local mode: the one rank (ring i, Ulysses u) this launch computes
+  int fold;          // step >= 0: fold into o_part / lse_part instead of writing them
 };
 
 struct FwdBars {
@@ -677,6 +678,23 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         if (store) a.sub.lse_run[ridx] = lse_new;
       } else {
       const size_t row_idx = (static_cast<size_t>(rank * g.B + b) * g.L + (store ? tau_q : 0)) * g.Hq_l + h;
+      // fp32 partial of a ring step: written (weight 1/l), or folded into the
+      // running partial already there by the log-sum-exp merge
+      float w_old = 0.f, w_new = inv_l, lse_out = lse_val;
+      if (a.step >= 0 && a.fold && store) {
+        const float lse_old = a.lse_part[row_idx];
+        const float mx = fmaxf(lse_old, lse_val);
+        w_new = 0.f;
+        lse_out = -INFINITY;
+        if (mx != -INFINITY) {
+          const float e_old = ex2_approx((lse_old - mx) * 1.4426950408889634f);
+          const float e_new = ex2_approx((lse_val - mx) * 1.4426950408889634f);
+          const float inv = 1.f / (e_old + e_new);
+          w_old = e_old * inv;
+          w_new = e_new * inv * inv_l;
+          lse_out = mx + __logf(e_old + e_new);
+        }
+      }
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -703,9 +721,15 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           } else {
             float4* dst = reinterpret_cast<float4*>(a.o_part + row_idx * D + c0);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(__uint_as_float(o[q * 4 + 0]) * inv_l, __uint_as_float(o[q * 4 + 1]) * inv_l,
-                                   __uint_as_float(o[q * 4 + 2]) * inv_l, __uint_as_float(o[q * 4 + 3]) * inv_l);
+            for (int q = 0; q < 8; ++q) {
+              float4 nv = make_float4(__uint_as_float(o[q * 4 + 0]) * w_new, __uint_as_float(o[q * 4 + 1]) * w_new,
+                                      __uint_as_float(o[q * 4 + 2]) * w_new, __uint_as_float(o[q * 4 + 3]) * w_new);
+              if (a.fold) {
+                const float4 ov = dst[q];
+                nv = make_float4(nv.x + ov.x * w_old, nv.y + ov.y * w_old, nv.z + ov.z * w_old, nv.w + ov.w * w_old);
+              }
+              dst[q] = nv;
+            }
           }
         }
       }
@@ -713,7 +737,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         if (a.step < 0)
           a.lse[row_idx] = lse_val;
         else
-          a.lse_part[row_idx] = lse_val;
+          a.lse_part[row_idx] = lse_out;
       }
       }  // USP epilogue
     }
@@ -761,6 +785,7 @@ cudaError_t launch_fwd_d(const FwdLaunch& L, cudaStream_t stream) {
   } else if (kMode == kModeLocal) {
     a.loc_i = L.loc_i;
     a.loc_u = L.loc_u;
+    a.fold = L.fold;
     blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * a.g.B * a.g.Hq_l;
   } else {
     blocks = static_cast<long long>((a.g.n_qtiles + 1) / 2) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hq_l;

@@ -141,6 +141,7 @@ struct FwdLaunch {
   MaskArgs mask;      // masked variant when mask.bm or mask.cu is set
   int local;          // local mode: one rank (loc_i, loc_u) of a real mesh, its own buffers (B in dim 4)
   int loc_i, loc_u;
+  int fold;           // stepwise / local: fold into o_part / lse_part (log-sum-exp merge) instead of writing
 };
 cudaError_t launch_attn_fwd(const FwdLaunch& a, cudaStream_t stream);
 

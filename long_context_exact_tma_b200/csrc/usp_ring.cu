@@ -81,9 +81,13 @@ size_t usp_ring_workspace_size(int B, int S, int Hq, int Hkv, int D, int causal,
   return bwd ? ring_bwd_ws(g) : static_cast<size_t>(usp::kStatusBytes);
 }
 
-int usp_ring_fwd_step(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int S,
-                      int Hq, int Hkv, int D, int causal, int P_u, int P_r, int i, int u, int t, void* workspace,
-                      size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int ring_fwd(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int S, int Hq,
+             int Hkv, int D, int causal, int P_u, int P_r, int i, int u, int t, void* workspace, size_t ws_bytes,
+             void* stream, bool fold) {
   usp::AttnGeom g{};
   int rc = usp::validate_geom(B, S, Hq, Hkv, D, causal, P_u, P_r, &g);
   if (rc != USP_OK) return rc;
@@ -107,9 +111,28 @@ int usp_ring_fwd_step(const void* q, const void* k, const void* v, float* o_part
   L.local = 1;
   L.loc_i = i;
   L.loc_u = u;
+  L.fold = fold ? 1 : 0;
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
   if (e == cudaSuccess) e = usp::launch_attn_fwd(L, st);
   return e == cudaSuccess ? USP_OK : record_error(USP_ERR_CUDA, "ring step launch: %s", cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+int usp_ring_fwd_step(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int B, int S,
+                      int Hq, int Hkv, int D, int causal, int P_u, int P_r, int i, int u, int t, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  return ring_fwd(q, k, v, o_part, lse_part, B, S, Hq, Hkv, D, causal, P_u, P_r, i, u, t, workspace, ws_bytes,
+                  stream, false);
+}
+
+int usp_ring_fwd_accumulate(const void* q, const void* k, const void* v, float* o_run, float* lse_run, int B, int S,
+                            int Hq, int Hkv, int D, int causal, int P_u, int P_r, int i, int u, int t,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  return ring_fwd(q, k, v, o_run, lse_run, B, S, Hq, Hkv, D, causal, P_u, P_r, i, u, t, workspace, ws_bytes, stream,
+                  t > 0);
 }
 
 int usp_ring_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,

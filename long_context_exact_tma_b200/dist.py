@@ -18,7 +18,7 @@ The backward passes K/V around the ring again, the dK/dV of each block
 travelling with it and arriving back at their owner after P_r hops.
 
 Every step of the compute runs in libusp.so (usp_ulysses_pack,
-usp_ring_fwd_step / usp_lse_merge, usp_ring_bwd_prepare / usp_ring_bwd_step);
+usp_ring_fwd_accumulate / usp_lse_merge, usp_ring_bwd_prepare / usp_ring_bwd_step);
 the exchanges are torch.distributed collectives (NCCL on GPUs): an equal-split
 all_to_all_single per group and batched isend/irecv to the ring neighbours,
 with the next K/V block in flight while the current one is computed. The
@@ -104,6 +104,12 @@ class CudaOps:
         self.B_.usp_ring_fwd_step(q, k, v, o_part, lse_part, g.B, g.S, g.Hq, g.Hkv, g.D, g.causal, g.P_u, g.P_r, m.i,
                                   m.u, t, self.ws_f, self.ws_f.numel(), self.stream)
 
+    def fwd_acc(self, q, k, v, o_run, lse_run, t):
+        """Step t folded into the running fp32 result (written at t = 0)."""
+        g, m = self.geo, self.mesh
+        self.B_.usp_ring_fwd_accumulate(q, k, v, o_run, lse_run, g.B, g.S, g.Hq, g.Hkv, g.D, g.causal, g.P_u, g.P_r,
+                                        m.i, m.u, t, self.ws_f, self.ws_f.numel(), self.stream)
+
     def merge(self, o_parts, lse_parts, n, out, lse_out):
         """n partials o_parts [n, rows, D], lse_parts [n, rows] -> out (fp32 or bf16), lse_out."""
         rows, D = o_parts.shape[1], o_parts.shape[2]
@@ -179,26 +185,23 @@ def ring_attn_fwd(q, k, v, geo: Geometry, mesh: Mesh, ops):
     rows = q.shape[0] * q.shape[1] * q.shape[2]
     D = q.shape[3]
     dev = q.device
-    # slot 0: running merge of the steps done; slot 1: the current step's partial
-    o_parts = torch.empty((2, rows, D), dtype=torch.float32, device=dev)
-    l_parts = torch.empty((2, rows), dtype=torch.float32, device=dev)
+    # the running fp32 result: step 0 writes it, every later step is folded into it
+    o_run = torch.empty((1, rows, D), dtype=torch.float32, device=dev)
+    l_run = torch.empty((1, rows), dtype=torch.float32, device=dev)
     # the caller's k, v are only ever sent; blocks are received into two buffers of our own
     bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(geo.P_r - 1, 2))]
     cur = (k, v)
     for t in range(geo.P_r):
         nxt = bufs[t % 2] if t < geo.P_r - 1 else None
         reqs = _exchange(cur, nxt, mesh.ring_next, mesh.ring_prev) if nxt is not None else []
-        slot = 0 if t == 0 else 1
-        ops.fwd_step(q, cur[0], cur[1], o_parts[slot], l_parts[slot], t)
-        if t > 0:
-            ops.merge(o_parts, l_parts, 2, o_parts[0], l_parts[0])
+        ops.fwd_acc(q, cur[0], cur[1], o_run[0], l_run[0], t)
         for r in reqs:
             r.wait()
         if nxt is not None:
             cur = nxt
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-    ops.merge(o_parts[:1], l_parts[:1], 1, out.view(rows, D), lse.view(rows))
+    ops.merge(o_run, l_run, 1, out.view(rows, D), lse.view(rows))
     return out, lse
 
 

@@ -69,6 +69,14 @@ class TorchOps:
         o_part.copy_(o.reshape(o_part.shape))
         lse_part.copy_(lse.permute(0, 2, 1).reshape(lse_part.shape))
 
+    def fwd_acc(self, q, k, v, o_run, lse_run, t):
+        if t == 0:
+            self.fwd_step(q, k, v, o_run, lse_run, t)
+            return
+        o_t, l_t = torch.empty_like(o_run), torch.empty_like(lse_run)
+        self.fwd_step(q, k, v, o_t, l_t, t)
+        self.merge(torch.stack([o_run, o_t]), torch.stack([lse_run, l_t]), 2, o_run, lse_run)
+
     def merge(self, o_parts, lse_parts, n, out, lse_out):
         lp = lse_parts[:n].double()
         m = lp.max(0).values

@@ -62,8 +62,10 @@ def test_ulysses_pack_around_all_to_all_bit_exact(cuda):
                 assert torch.equal(out, rm[i * P_u + u])
 
 
-def _ring_all_ranks(spec, hs, do_hs):
-    """Run every rank's ring schedule with the per-rank calls (one GPU, ranks in turn)."""
+def _ring_all_ranks(spec, hs, do_hs, accumulate=False):
+    """Run every rank's ring schedule with the per-rank calls (one GPU, ranks in turn):
+    each step's partial merged by usp_lse_merge, or (accumulate) folded into one
+    running partial by usp_ring_fwd_accumulate."""
     B, S, Hq, Hkv, D = (spec[k] for k in ("B", "S", "Hq", "Hkv", "D"))
     P_u, P_r, causal = spec["P_u"], spec["P_r"], spec["causal"]
     geo = (B, S, Hq, Hkv, D, causal, P_u, P_r)
@@ -80,6 +82,10 @@ def _ring_all_ranks(spec, hs, do_hs):
             l_parts = torch.empty((2, rows), dtype=torch.float32, device=dev)
             for t in range(P_r):
                 j = (i - t) % P_r
+                if accumulate:
+                    B_.usp_ring_fwd_accumulate(q[i, u], k[j, u], v[j, u], o_parts[0], l_parts[0], *geo, i, u, t,
+                                               ws_f, ws_f.numel())
+                    continue
                 s = 0 if t == 0 else 1
                 B_.usp_ring_fwd_step(q[i, u], k[j, u], v[j, u], o_parts[s], l_parts[s], *geo, i, u, t, ws_f,
                                      ws_f.numel())
@@ -104,13 +110,15 @@ def _ring_all_ranks(spec, hs, do_hs):
     return out, lse, dq, dk, dv
 
 
+@pytest.mark.parametrize("accumulate", [False, True], ids=["merged", "accumulated"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_ring_steps_of_every_rank_match_oracle(cuda, name):
+def test_ring_steps_of_every_rank_match_oracle(cuda, name, accumulate):
     spec = CASES[name]
     t = inputs(spec, which=("q", "k", "v", "do"))
     P_u, P_r = spec["P_u"], spec["P_r"]
     hs = {n: oracle.to_head_sharded(t[n].cpu(), P_u, P_r).to(cuda) for n in ("q", "k", "v", "do")}
-    out, lse, dq, dk, dv = _ring_all_ranks(spec, hs, hs["do"])
+    out, lse, dq, dk, dv = _ring_all_ranks(spec, hs, hs["do"], accumulate)
+    name = f"{name}/accumulated" if accumulate else name
     to_g = lambda x: oracle.from_head_sharded(x.cpu(), P_u, P_r)  # noqa: E731
     tc = {n: t[n].cpu() for n in ("q", "k", "v", "do")}
     o_g = to_g(out)
