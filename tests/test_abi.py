@@ -198,3 +198,69 @@ def test_masked_rejects_unaligned_chunks_and_bad_docs():
     assert rc == B_.USP_ERR_INVALID_ARG
     rc = L.usp_attn_bwd_masked(*([FAKE] * 9), 1, 768, 4, 4, 128, 1, 2, 2, m, FAKE, 1 << 30, None)
     assert rc == B_.USP_ERR_UNSUPPORTED
+
+
+def test_rows_copy_rejects_bad_jobs():
+    """Validation of usp_rows_copy before any launch (no GPU needed)."""
+    L = B_.lib()
+    good = dict(src=FAKE, dst=FAKE, dtype=B_.USP_BF16, n_b=1, n_k=4, n_j=2, D=128, s_b=0, s_k=256, s_h=128,
+                d_b=0, d_k=256, d_h=128)
+
+    def call(**kw):
+        j = dict(good)
+        j.update(kw)
+        arr = (B_.RowsJob * 1)()
+        f = dict(add=0, s_k0=0, s_kstep=1, s_h0=0, s_hstep=1, s_hdiv=1, d_k0=0, d_kstep=1, d_h0=0, d_hstep=1,
+                 d_hdiv=1)
+        f.update(j)
+        arr[0] = B_.RowsJob(**f)
+        return L.usp_rows_copy(arr, 1, None)
+    assert call(dtype=5) == B_.USP_ERR_INVALID_ARG                 # unknown dtype
+    assert call(add=1) == B_.USP_ERR_INVALID_ARG                   # add needs fp32
+    assert call(D=12) == B_.USP_ERR_INVALID_ARG                    # 24-byte rows
+    assert call(s_hdiv=0) == B_.USP_ERR_INVALID_ARG
+    assert call(d_kstep=-1) == B_.USP_ERR_INVALID_ARG
+    assert call(src=None) == B_.USP_ERR_INVALID_ARG
+    assert call(dst=FAKE + 8) == B_.USP_ERR_INVALID_ARG            # unaligned
+    assert call(s_k=100) == B_.USP_ERR_INVALID_ARG                 # rows not 16-byte aligned
+    assert call(n_k=0) == B_.USP_OK                                 # nothing to move, nothing launched
+    assert L.usp_rows_copy(None, 1, None) == B_.USP_ERR_INVALID_ARG
+    arr = (B_.RowsJob * 17)()
+    assert L.usp_rows_copy(arr, 17, None) == B_.USP_ERR_INVALID_ARG
+
+
+def test_longnet_rejects_bad_arguments():
+    import ctypes
+    L = B_.lib()
+    ws = 1 << 30
+    # local pairs need w <= T and T % w == 0; gathered ones w > T, w % T == 0
+    assert L.usp_longnet_fwd_local(FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 2048, 2, FAKE, ws, None) \
+        == B_.USP_ERR_UNSUPPORTED
+    assert L.usp_longnet_fwd_local(FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 384, 2, FAKE, ws, None) \
+        == B_.USP_ERR_UNSUPPORTED
+    assert L.usp_longnet_fwd_cross(FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 512, 2, 0, 0, FAKE, ws, None) \
+        == B_.USP_ERR_UNSUPPORTED
+    assert L.usp_longnet_fwd_cross(FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 3072, 2, 2, 0, FAKE, ws, None) \
+        == B_.USP_ERR_INVALID_ARG                                   # offset >= r
+    assert L.usp_longnet_fwd_cross(FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 3072, 2, 0, 3, FAKE, ws, None) \
+        == B_.USP_ERR_INVALID_ARG                                   # rank outside the segment of 3
+    assert L.usp_longnet_fwd_cross(FAKE, FAKE, FAKE, 1, 1024, 4, 4, 96, 1, 3072, 2, 0, 0, FAKE, ws, None) \
+        == B_.USP_ERR_UNSUPPORTED                                   # D
+    assert L.usp_longnet_fwd_begin(1, 1024, 4, 128, FAKE, 100, None) == B_.USP_ERR_WORKSPACE
+    assert L.usp_longnet_rows(1024, 1536, 2, 0, 0, None, None, None, None) == B_.USP_ERR_INVALID_ARG
+    w = (ctypes.c_int * 2)(512, 4096)
+    r = (ctypes.c_int * 2)(1, 3)
+    n = B_.usp_longnet_workspace_size(1, 1024, 4, 128, [(512, 1), (4096, 3)], 1)
+    assert n > 256 and B_.usp_longnet_workspace_size(1, 1024, 4, 128, [(768, 1)], 1) == 0
+    assert L.usp_longnet_workspace_size(1, 1024, 4, 128, 2, w, r, 0) == 256 + 1024 * 4 * (4 * 128 + 4)
+    assert L.usp_longnet_bwd_local(*([FAKE] * 7), 1, 1024, 4, 4, 128, 1, 512, 1, FAKE, 1000, None) \
+        == B_.USP_ERR_WORKSPACE
+
+
+def test_ring_accumulate_rejects_bad_arguments():
+    L = B_.lib()
+    # rank outside the 1 x 4 mesh, then a step past the ring
+    assert L.usp_ring_fwd_accumulate(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 1, 4, 4, 0, 0, FAKE, 256,
+                                     None) == B_.USP_ERR_INVALID_ARG
+    assert L.usp_ring_fwd_accumulate(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1024, 4, 4, 128, 1, 1, 4, 0, 0, 4, FAKE, 256,
+                                     None) == B_.USP_ERR_INVALID_ARG
