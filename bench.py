@@ -527,10 +527,11 @@ def variants_per_workload(dev, peak_tf):
 def rank_per_workload(dev, peak_tf):
     """Event-timed per-rank compute of the two multi-GPU layouts, on one GPU
     (the collectives between the calls are not part of it):
-      - one rank of a real USP mesh: ring rank 0 of the S=16K ring-8 workload
-        runs its 8 ring steps (usp_ring_fwd_accumulate: each step's partial
-        folded into a running one in the kernel) and the backward steps (usp_ring_bwd_prepare +
-        usp_ring_bwd_step) against 8 resident K/V blocks;
+      - one rank of a real USP mesh, rank (0, 0) of the S=16K ring-8 and of the
+        S=128K USP 4x2 workloads: its ring steps (usp_ring_fwd_accumulate: each
+        step's partial folded into a running one in the kernel) and the backward
+        steps (usp_ring_bwd_prepare + usp_ring_bwd_step) against resident K/V
+        blocks;
       - rank 0 of LongNet's distributed layout over 4 ranks on the S=32K
         dilated schedule: its local pairs and, for the gathered pairs, the cross
         attention of its kept rows against the segment's kept K/V rows (gathered
@@ -541,60 +542,65 @@ def rank_per_workload(dev, peak_tf):
     from long_context_exact_tma_b200 import dist as udist
     from usp_inputs import normal_bf16
     res = {}
-    # -- one rank of the USP mesh (ring 8, S=16K)
-    w = dict(WORKLOADS[2])
-    B, S, Hq, Hkv, D, P_u, P_r = w["B"], w["S"], w["Hq"], w["Hkv"], w["D"], w["P_u"], w["P_r"]
-    causal, L = w["causal"], w["S"] // w["P_r"]
-    P, c = P_u * P_r, S // (2 * P_u * P_r)
-    q = normal_bf16(950, (B, L, Hq, D), device=dev)
-    do = normal_bf16(951, (B, L, Hq, D), device=dev)
-    ks = [normal_bf16(960 + j, (B, L, Hkv, D), device=dev) for j in range(P_r)]
-    vs = [normal_bf16(980 + j, (B, L, Hkv, D), device=dev) for j in range(P_r)]
-    pos0 = [x for r_ in (0, 2 * P - 1) for x in range(r_ * c, (r_ + 1) * c)]  # ring rank 0's zigzag positions
-    vis = sum(p + 1 for p in pos0) if causal else len(pos0) * S
-    fl = 4.0 * D * B * Hq * vis
-    rows = B * L * Hq
-    wsf = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 0), dtype=torch.uint8,
-                      device=dev)
-    wsb = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 1), dtype=torch.uint8,
-                      device=dev)
-    o_parts = torch.empty((2, rows, D), dtype=torch.float32, device=dev)
-    l_parts = torch.empty((2, rows), dtype=torch.float32, device=dev)
-    out = torch.empty_like(q)
-    lse = torch.empty((B, L, Hq), dtype=torch.float32, device=dev)
+    # -- one rank of the USP mesh: ring 8 at S=16K (2048 rows a rank) and USP 4x2 at S=128K (64K rows)
+    for cfg, key in ((2, "usp_rank_s16k_ring8"), (3, "usp_rank_s128k_usp4x2")):
+        w = dict(WORKLOADS[cfg])
+        B, S, Hq, Hkv, D, P_u, P_r = w["B"], w["S"], w["Hq"], w["Hkv"], w["D"], w["P_u"], w["P_r"]
+        causal, L = w["causal"], w["S"] // w["P_r"]
+        P, c = P_u * P_r, S // (2 * P_u * P_r)
+        Hl, Hkl = Hq // P_u, Hkv // P_u
+        q = normal_bf16(950, (B, L, Hl, D), device=dev)
+        do = normal_bf16(951, (B, L, Hl, D), device=dev)
+        ks = [normal_bf16(960 + j, (B, L, Hkl, D), device=dev) for j in range(P_r)]
+        vs = [normal_bf16(980 + j, (B, L, Hkl, D), device=dev) for j in range(P_r)]
+        # rank (i=0, u=0) holds, after the all-to-all, the zigzag chunks of ranks 0 .. P_u-1
+        pos0 = [x for rr in range(P_u) for ch in (rr, 2 * P - 1 - rr) for x in range(ch * c, (ch + 1) * c)]
+        vis = sum(p + 1 for p in pos0) if causal else len(pos0) * S
+        fl = 4.0 * D * B * Hl * vis
+        rows = B * L * Hl
+        wsf = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 0), dtype=torch.uint8,
+                          device=dev)
+        wsb = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 1), dtype=torch.uint8,
+                          device=dev)
+        o_run = torch.empty((1, rows, D), dtype=torch.float32, device=dev)
+        l_run = torch.empty((1, rows), dtype=torch.float32, device=dev)
+        out = torch.empty_like(q)
+        lse = torch.empty((B, L, Hl), dtype=torch.float32, device=dev)
 
-    def ring_fwd():  # each step folded into the running partial in the kernel's epilogue
-        for t in range(P_r):
-            j = (0 - t) % P_r
-            B_.usp_ring_fwd_accumulate(q, ks[j], vs[j], o_parts[0], l_parts[0], B, S, Hq, Hkv, D, causal, P_u, P_r,
-                                       0, 0, t, wsf, wsf.numel())
-        B_.usp_lse_merge(o_parts[:1], l_parts[:1], 1, rows, D, out, B_.USP_BF16, lse)
+        def ring_fwd():  # each step folded into the running partial in the kernel's epilogue
+            for t in range(P_r):
+                j = (0 - t) % P_r
+                B_.usp_ring_fwd_accumulate(q, ks[j], vs[j], o_run[0], l_run[0], B, S, Hq, Hkv, D, causal, P_u, P_r,
+                                           0, 0, t, wsf, wsf.numel())
+            B_.usp_lse_merge(o_run, l_run, 1, rows, D, out, B_.USP_BF16, lse)
 
-    ring_fwd()
-    dq_acc = torch.zeros((B, L, Hq, D), dtype=torch.float32, device=dev)
-    dq = torch.empty_like(q)
-    dk = torch.zeros((B, L, Hkv, D), dtype=torch.float32, device=dev)
-    dv = torch.zeros_like(dk)
+        ring_fwd()
+        dq_acc = torch.zeros((B, L, Hl, D), dtype=torch.float32, device=dev)
+        dq = torch.empty_like(q)
+        dk = torch.zeros((B, L, Hkl, D), dtype=torch.float32, device=dev)
+        dv = torch.zeros_like(dk)
 
-    def ring_bwd():
-        B_.usp_ring_bwd_prepare(out, lse, do, B, S, Hq, Hkv, D, causal, P_u, P_r, wsb, wsb.numel())
-        for t in range(P_r):
-            j = (0 - t) % P_r
-            B_.usp_ring_bwd_step(q, ks[j], vs[j], do, dq_acc, dq if t == P_r - 1 else None, dk, dv, B, S, Hq, Hkv, D,
-                                 causal, P_u, P_r, 0, 0, t, wsb, wsb.numel())
+        def ring_bwd():
+            B_.usp_ring_bwd_prepare(out, lse, do, B, S, Hq, Hkv, D, causal, P_u, P_r, wsb, wsb.numel())
+            for t in range(P_r):
+                j = (0 - t) % P_r
+                B_.usp_ring_bwd_step(q, ks[j], vs[j], do, dq_acc, dq if t == P_r - 1 else None, dk, dv, B, S, Hq,
+                                     Hkv, D, causal, P_u, P_r, 0, 0, t, wsb, wsb.numel())
 
-    ms_f, ms_b = _time_pair(ring_fwd, ring_bwd, reps=10)
-    for ws in (wsf, wsb):
-        rc, site = B_.usp_workspace_status(ws)
-        if rc != B_.USP_OK:
-            raise B_.UspError(rc, f"device wait timed out (site {site:#x})")
-    res["usp_rank_s16k_ring8"] = {
-        "shape": "ring rank 0 of the S=16K ring-8 workload: 8 ring steps against resident K/V blocks (no NCCL)",
-        "fwd": {"TFLOP/s": round(fl / ms_f / 1e9, 1), "frac_of_peak": round(fl / ms_f / 1e9 / peak_tf, 4),
-                "ms": round(ms_f, 3)},
-        "bwd": {"TFLOP/s": round(2.5 * fl / ms_b / 1e9, 1), "frac_of_peak": round(2.5 * fl / ms_b / 1e9 / peak_tf, 4),
-                "ms": round(ms_b, 3)}}
-    del q, do, ks, vs, o_parts, l_parts, out, lse, dq_acc, dq, dk, dv, wsf, wsb
+        ms_f, ms_b = _time_pair(ring_fwd, ring_bwd, reps=10 if cfg == 2 else 2)
+        for ws in (wsf, wsb):
+            rc, site = B_.usp_workspace_status(ws)
+            if rc != B_.USP_OK:
+                raise B_.UspError(rc, f"device wait timed out (site {site:#x})")
+        res[key] = {
+            "shape": f"rank (0, 0) of the {w['name']} mesh: its {P_r} ring steps against resident K/V blocks "
+                     f"({L} rows, {Hl} heads; no NCCL)",
+            "fwd": {"TFLOP/s": round(fl / ms_f / 1e9, 1), "frac_of_peak": round(fl / ms_f / 1e9 / peak_tf, 4),
+                    "ms": round(ms_f, 3)},
+            "bwd": {"TFLOP/s": round(2.5 * fl / ms_b / 1e9, 1),
+                    "frac_of_peak": round(2.5 * fl / ms_b / 1e9 / peak_tf, 4), "ms": round(ms_b, 3)}}
+        del q, do, ks, vs, o_run, l_run, out, lse, dq_acc, dq, dk, dv, wsf, wsb
+        torch.cuda.empty_cache()
     # -- rank 0 of LongNet's distributed layout, 4 ranks, S=32K
     B, S, H, D, M = 1, 32768, 16, 128, 4
     T = S // M
