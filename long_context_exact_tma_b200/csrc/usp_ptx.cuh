@@ -66,29 +66,36 @@ struct WaitCtl {
 // the abort flag and records `site` in the status word).
 // The status word (a global load of several hundred cycles) and the timer are
 // read only every 32nd round, so that a phase completing is seen within one
-// try_wait and not after a global round trip.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w, int site) {
-  const uint32_t a = smem_addr(bar);
-  if (mbar_try_wait(a, parity)) return true;
+// try_wait and not after a global round trip. Only the first try_wait is
+// inlined at each wait site; the polling loop is one out-of-line function, so
+// the many wait sites of a warp-specialised kernel keep its hot loops small
+// (the warps of all roles share each SM sub-partition's instruction cache).
+static __device__ __noinline__ bool mbar_wait_poll(uint32_t a, uint32_t parity, volatile int* abort_flag, int* status,
+                                                   uint64_t limit_ns, int site) {
   uint64_t t0 = 0;
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(a, parity)) return true;
-    if (*w.abort_flag) return false;
+    if (*abort_flag) return false;
     if ((n & 31u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(w.status) != 0) {  // another CTA already gave up
-        *w.abort_flag = 1;
+      if (*reinterpret_cast<volatile int*>(status) != 0) {  // another CTA already gave up
+        *abort_flag = 1;
         return false;
       }
       const uint64_t now = global_timer_ns();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > w.limit_ns) {
-        *w.abort_flag = 1;
-        atomicCAS(w.status, 0, site);
+      } else if (now - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicCAS(status, 0, site);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w, int site) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  return mbar_wait_poll(a, parity, w.abort_flag, w.status, w.limit_ns, site);
 }
 
 // Drain wait used after an abort: ignores the abort flag, gives up after limit_ns.
