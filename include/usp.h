@@ -374,10 +374,10 @@ size_t usp_dilated_workspace_size(int B, int S, int Hq, int D);
  *   out, lse   the forward's outputs;  dO [B][S][Hq][D] bf16
  *   dQ         [B][S][Hq][D] bf16;  dK, dV [B][S][Hkv][D] fp32 (overwritten)
  *   workspace  usp_dilated_bwd_workspace_size(B, S, Hq, D, n_pairs, w, r)
- *              bytes (status, Delta of every row, an fp32 dQ, and four slots
- *              of the row tables of the largest launch: with Hq == Hkv the
- *              head offsets of a pair run on up to four streams at once, the
- *              forward's too); 0 for an unsupported shape.
+ *              bytes (status, Delta of every row, an fp32 dQ, and one slot of
+ *              the row tables of the largest launch per head offset, up to
+ *              16: with Hq == Hkv the head offsets of a pair run on up to 16
+ *              streams at once, the forward's too); 0 for an unsupported shape.
  */
 size_t usp_dilated_bwd_workspace_size(int B, int S, int Hq, int D, int n_pairs, const int* w, const int* r);
 int usp_dilated_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,

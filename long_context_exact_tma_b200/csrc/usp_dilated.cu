@@ -180,7 +180,8 @@ size_t slot_floats(int B, int S, int Hq, int w, int r) {
 }
 
 size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r) {
-  return kSideStreams * slot_floats(B, S, Hq, w, r);
+  const int n_off = r < Hq ? r : Hq;  // launches of the pair, at most kSideStreams of them at a time
+  return static_cast<size_t>(n_off < kSideStreams ? n_off : kSideStreams) * slot_floats(B, S, Hq, w, r);
 }
 
 int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO, const float* lse,

@@ -23,7 +23,7 @@ unsigned long long current_wait_ns();
 // the work issued so far on `main` and returns them; side_join makes `main`
 // wait for everything issued on them since. Created on first use, kept for the
 // thread's life (one set per thread, so concurrent callers never share an event).
-constexpr int kSideStreams = 4;
+constexpr int kSideStreams = 16;
 cudaError_t side_fork(cudaStream_t main, int n, cudaStream_t* out);
 cudaError_t side_join(cudaStream_t main, int n);
 
