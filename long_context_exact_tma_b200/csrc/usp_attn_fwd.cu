@@ -20,7 +20,9 @@
 //               of waiting behind the previous tile's PV.
 //   warp 1      TMEM allocator and UMMA issuer (one thread), per key tile and
 //               query tile t = 0, 1 in turn:
-//                 O_t += P_t V    (M=128 N=D; A = P_t read from TMEM)
+//                 O_t += P_t V    (M=128 N=D; A = P_t read from TMEM; in two
+//                                 halves of 64 keys, the first as soon as
+//                                 softmax t has written that half of P_t)
 //                 S_t  = Q_t K^T  of the next key tile (M=128 N=128, fp32 in TMEM;
 //                                 it overwrites P_t, so it waits for that PV)
 //               so the tensor core runs tile 1's PV and S while softmax 0 works
@@ -85,6 +87,7 @@ struct FwdBars {
   uint64_t q_full;
   uint64_t k_full[3], v_full[3], k_empty[3], v_empty[3];
   uint64_t s_full[2], p_full[2], pv_done[2], desc_full[2];
+  uint64_t p_half[2];  // P_t of the tile's first 64 keys is in TMEM (the first half of PV_t may start)
   uint64_t drain;
   // Key-tile descriptors published by the producer with k_full of that tile:
   // {1, or -1 = no more tiles; ring rank j of the key owner; key tile n;
@@ -197,6 +200,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_full[t], 4);  // one arrival per softmax warp
+      mbar_init(&bars->p_half[t], 4);
       mbar_init(&bars->pv_done[t], 1);
       mbar_init(&bars->desc_full[t], 1);
     }
@@ -383,12 +387,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           const int* nxt = nullptr;
           for (int t = 0; t < 2 && ok; ++t) {
             if (attends(cur, t)) {
+              // PV in two halves of 64 keys: the first as soon as their P is in TMEM
+              if (!mbar_wait_w(&bars->p_half[t], npv[t] & 1, w, kSiteP)) { ok = false; break; }
+              tc_fence_after();
+  #pragma unroll
+              for (int kk = 0; kk < kBN / 32; ++kk)
+                umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                                   (npv[t] > 0 || kk > 0) ? 1u : 0u);
               if (!mbar_wait_w(&bars->p_full[t], npv[t] & 1, w, kSiteP)) { ok = false; break; }
               tc_fence_after();
   #pragma unroll
-              for (int kk = 0; kk < kBN / 16; ++kk)
-                umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
-                                   (npv[t] > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+                umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
               umma_commit_w(&bars->pv_done[t]);
               ++npv[t];
               pv_wait[t] = true;
@@ -445,12 +455,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           const uint64_t vd = dV0 + ((s * C::kTileBytes) >> 4);
           bool next = false;
           for (int t = 0; t < 2 && ok; ++t) {
+            // PV in two halves of 64 keys: the first as soon as their P is in TMEM
+            if (!mbar_wait_w(&bars->p_half[t], it & 1, w, kSiteP)) { ok = false; break; }
+            tc_fence_after();
+  #pragma unroll
+            for (int kk = 0; kk < kBN / 32; ++kk)
+              umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
+                                 (it > 0 || kk > 0) ? 1u : 0u);
             if (!mbar_wait_w(&bars->p_full[t], it & 1, w, kSiteP)) { ok = false; break; }
             tc_fence_after();
   #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-              umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV,
-                                 (it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+              umma_bf16_tmem_a_w(tmem + col_o(t), tmem + col_s(t) + kk * 8, vd + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
             umma_commit_w(&bars->pv_done[t]);
             if (t == 1) umma_commit_w(&bars->v_empty[s]);
             if (t == 0) {
@@ -601,13 +617,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       };
       emit(r0, 0);
       emit(r1, 16);
-      emit(r2, 32);
-      emit(r3, 48);
-      const float rs = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) + (acc[3].x + acc[3].y);
-      const float rsb =
-          (accb[0].x + accb[0].y) + (accb[1].x + accb[1].y) + (accb[2].x + accb[2].y) + (accb[3].x + accb[3].y);
       // The PV UMMA of the previous tile has completed (S_t is only issued after
-      // it), so O_t can be rescaled in place.
+      // it), so O_t can be rescaled in place -- before the first half of P is
+      // handed over, since the first half of PV_t starts on it.
       if (it > 0 && __any_sync(0xffffffffu, bump)) {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -620,6 +632,14 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           tmem_st32(trow + cO + c0, o);
         }
       }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive_warp(&bars->p_half[t]);
+      emit(r2, 32);
+      emit(r3, 48);
+      const float rs = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) + (acc[3].x + acc[3].y);
+      const float rsb =
+          (accb[0].x + accb[0].y) + (accb[1].x + accb[1].y) + (accb[2].x + accb[2].y) + (accb[3].x + accb[3].y);
       l_run = l_run * alpha + rs;
       lb_run = lb_run * alpha + rsb;
       tmem_st_wait();
