@@ -644,6 +644,7 @@ def rank_per_workload(dev, peak_tf):
                 for o in range(min(r, H)):
                     kc, vc, _, _ = gathered[(w_, r, o)]
                     ops.fwd_cross(q, kc, vc, True, w_, r, o, 0)
+                ops.cross_join()
         state["out"], state["lse"] = ops.fwd_end()
 
     ln_fwd()
@@ -659,6 +660,7 @@ def rank_per_workload(dev, peak_tf):
                 for o in range(min(r, H)):
                     kc, vc, dkc, dvc = gathered[(w_, r, o)]
                     ops.bwd_cross(q, kc, vc, do, state["lse"], dkc, dvc, True, w_, r, o, 0)
+                ops.cross_join()
         ops.bwd_end()
 
     ms_f, ms_b = _time_pair(ln_fwd, ln_bwd, reps=5)

@@ -454,6 +454,12 @@ int usp_rows_copy(const usp_rows_job* jobs, int n_jobs, void* stream);
  * fp32 (overwritten), which the caller reduce-scatters over the segment and
  * adds at its own kept rows (usp_rows_copy with add); usp_longnet_bwd_end
  * writes dQ [B][T][Hq][D] bf16.
+ * Concurrency: the offsets of one gathered pair write disjoint heads (and,
+ * backward, their own dkc/dvc and the row-table slot o mod 16 of the
+ * workspace), so their usp_longnet_fwd_cross / usp_longnet_bwd_cross calls may
+ * run on different streams at the same time, as long as offsets that share a
+ * slot (o mod 16) share a stream; calls of different pairs, and the local
+ * calls, must not overlap each other.
  * Workspace: usp_longnet_workspace_size(B, T, Hq, D, n_pairs, w, r, bwd) for
  * the pairs that will be passed (0 for an unsupported shape). D in {64, 128},
  * Hq % Hkv == 0, 1 <= r <= w.

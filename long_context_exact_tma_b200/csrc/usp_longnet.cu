@@ -71,9 +71,8 @@ size_t fwd_ws(long long B, long long T, long long Hq, long long D) {
   return static_cast<size_t>(usp::kStatusBytes) + static_cast<size_t>(B * T * Hq) * (4 * D + 4);
 }
 
-// The largest row table of a pair's launches on this rank (floats).
-size_t pair_table(int B, int T, int Hq, int w, int r) {
-  if (w <= T) return usp::dilated_pair_table_floats(B, T, Hq, w, r);
+// The largest row table of one offset's cross launch of a gathered pair (floats).
+size_t cross_slot_floats(int B, int T, int Hq, int r) {
   size_t tbl = 0;
   for (int o = 0; o < r && o < Hq; ++o) {
     const size_t Lp = static_cast<size_t>(((T + r - 1) / r + 127) / 128 * 128);  // n_rows <= ceil(T / r)
@@ -81,6 +80,16 @@ size_t pair_table(int B, int T, int Hq, int w, int r) {
     if (n > tbl) tbl = n;
   }
   return tbl;
+}
+
+// The row tables a pair's launches on this rank need (floats): for a gathered
+// pair one slot per head offset, up to usp::kSideStreams (offset o uses slot
+// o mod kSideStreams, so the offsets' cross backwards may run concurrently).
+size_t pair_table(int B, int T, int Hq, int w, int r) {
+  if (w <= T) return usp::dilated_pair_table_floats(B, T, Hq, w, r);
+  const int n_off = r < Hq ? r : Hq;
+  const int slots = n_off < usp::kSideStreams ? n_off : usp::kSideStreams;
+  return static_cast<size_t>(slots) * cross_slot_floats(B, T, Hq, r);
 }
 
 // Delta takes whole 16-byte groups, so the fp32 dQ after it stays aligned.
@@ -334,8 +343,11 @@ int usp_longnet_bwd_cross(const void* q, const void* kc, const void* vc, const v
   L.status = static_cast<int*>(workspace);
   L.wait_ns = usp::current_wait_ns();
   L.Lp = (x.n_rows + 127) / 128 * 128;
-  L.lse2 = p.lse2_t;
-  L.delta = p.delta_t;
+  const size_t slot = static_cast<size_t>(o % usp::kSideStreams) * cross_slot_floats(B, T, Hq, r);
+  float* const lse2_t = p.lse2_t + slot;  // this offset's row-table slot
+  float* const delta_t = p.delta_t + slot;
+  L.lse2 = lse2_t;
+  L.delta = delta_t;
   L.dk = dkc;
   L.dv = dvc;
   L.dq = nullptr;
@@ -345,7 +357,7 @@ int usp_longnet_bwd_cross(const void* q, const void* kc, const void* vc, const v
   if (rc == USP_OK) rc = gathered_map(&L.tm_k, kc, x, D, n_sel, B);
   if (rc == USP_OK) rc = gathered_map(&L.tm_v, vc, x, D, n_sel, B);
   if (rc != USP_OK) return rc;
-  e = usp::launch_dilated_tables(lse, p.delta, p.lse2_t, p.delta_t, L.sub, L.Lp, st);
+  e = usp::launch_dilated_tables(lse, p.delta, lse2_t, delta_t, L.sub, L.Lp, st);
   if (e == cudaSuccess) e = usp::launch_attn_bwd(L, st);
   if (e == cudaSuccess) e = usp::launch_attn_bwd_dq(L, st);
   return e == cudaSuccess ? USP_OK : record_error(USP_ERR_CUDA, "cross backward launch: %s", cudaGetErrorString(e));

@@ -380,9 +380,11 @@ def longnet_attn_fwd(q, k, v, pairs, causal, lm: LongNetMesh, ops, comm=None):
         if w <= lm.T:
             ops.fwd_local(q, k, v, causal, w, r)
             continue
+        # the offsets write disjoint heads: ops may run their cross attentions side by side
         for o in range(min(r, Hq)):
             kc, vc, _, _ = _gather_kept(k, v, w, r, o, Hq, lm, ops, comm)
             ops.fwd_cross(q, kc, vc, causal, w, r, o, lm.seg_rank(w))
+        ops.cross_join()
     return ops.fwd_end()
 
 
@@ -402,13 +404,19 @@ def longnet_attn_bwd(q, k, v, out, lse, dO, pairs, causal, lm: LongNetMesh, ops,
             ops.bwd_local(q, k, v, dO, lse, dK, dV, causal, w, r)
             continue
         G = w // T
+        # every offset's cross backward first (ops may run them side by side: disjoint
+        # heads, their own dkc / dvc), then their gradients home
+        pending = []
         for o in range(min(r, Hq)):
             kc, vc, shares, n_max = _gather_kept(k, v, w, r, o, Hq, lm, ops, comm)
-            ns = kc.shape[2]
-            n_kept = kc.shape[1]
             dkc = torch.empty(kc.shape, dtype=torch.float32, device=k.device)
             dvc = torch.empty_like(dkc)
             ops.bwd_cross(q, kc, vc, dO, lse, dkc, dvc, causal, w, r, o, lm.seg_rank(w))
+            pending.append((o, shares, n_max, dkc, dvc))
+        ops.cross_join()
+        for o, shares, n_max, dkc, dvc in pending:
+            ns = dkc.shape[2]
+            n_kept = dkc.shape[1]
             send = torch.empty((G, 2, B, n_max, ns, D), dtype=torch.float32, device=k.device)
             jobs = []
             for x, (_, k_lo, nr, _) in enumerate(shares):
@@ -430,7 +438,12 @@ def longnet_attn_bwd(q, k, v, out, lse, dO, pairs, causal, lm: LongNetMesh, ops,
 
 
 class CudaLongNetOps:
-    """The per-rank LongNet compute in libusp.so kernels."""
+    """The per-rank LongNet compute in libusp.so kernels. The cross attentions of
+    one gathered pair's head offsets run on side streams (offset o on stream
+    o mod min(16, offsets): the library's row-table slot of a cross backward is o
+    mod 16); cross_join makes the main stream wait for them."""
+
+    N_SIDE = 16
 
     def __init__(self, B, T, Hq, Hkv, D, pairs, stream=None, device="cuda"):
         from . import binding as B_
@@ -438,6 +451,8 @@ class CudaLongNetOps:
         self.BF16, self.F32 = B_.USP_BF16, B_.USP_F32
         self.shape = (B, T, Hq, Hkv, D)
         self.stream = stream
+        self._side = None
+        self._used = []
         self.ws_f = torch.zeros(B_.usp_longnet_workspace_size(B, T, Hq, D, pairs, 0), dtype=torch.uint8,
                                 device=device)
         self.ws_b = torch.zeros(B_.usp_longnet_workspace_size(B, T, Hq, D, pairs, 1), dtype=torch.uint8,
@@ -456,10 +471,37 @@ class CudaLongNetOps:
         self.B_.usp_longnet_fwd_local(q, k, v, B, T, Hq, Hkv, D, causal, w, r, self.ws_f, self.ws_f.numel(),
                                       self.stream)
 
+    def _main(self):
+        return self.stream if self.stream is not None else torch.cuda.current_stream(self.device)
+
+    def _side_for(self, o, r, tensors):
+        """The side stream of offset o, after everything issued so far on the main
+        stream; the given tensors are kept from reuse until its work is done."""
+        if self._side is None:
+            self._side = [torch.cuda.Stream(device=self.device) for _ in range(self.N_SIDE)]
+        s = self._side[o % min(self.N_SIDE, r, self.shape[2])]
+        ev = torch.cuda.Event()
+        ev.record(self._main())
+        s.wait_event(ev)
+        for t in tensors:
+            t.record_stream(s)
+        if s not in self._used:
+            self._used.append(s)
+        return s
+
+    def cross_join(self):
+        main = self._main()
+        for s in self._used:
+            ev = torch.cuda.Event()
+            ev.record(s)
+            main.wait_event(ev)
+        self._used = []
+
     def fwd_cross(self, q, kc, vc, causal, w, r, o, g):
         B, T, Hq, Hkv, D = self.shape
+        s = self._side_for(o, r, (q, kc, vc))
         self.B_.usp_longnet_fwd_cross(q, kc, vc, B, T, Hq, Hkv, D, causal, w, r, o, g, self.ws_f, self.ws_f.numel(),
-                                      self.stream)
+                                      s)
 
     def fwd_end(self):
         B, T, Hq, Hkv, D = self.shape
@@ -480,8 +522,9 @@ class CudaLongNetOps:
 
     def bwd_cross(self, q, kc, vc, dO, lse, dkc, dvc, causal, w, r, o, g):
         B, T, Hq, Hkv, D = self.shape
+        s = self._side_for(o, r, (q, kc, vc, dO, lse, dkc, dvc))
         self.B_.usp_longnet_bwd_cross(q, kc, vc, dO, lse, dkc, dvc, B, T, Hq, Hkv, D, causal, w, r, o, g, self.ws_b,
-                                      self.ws_b.numel(), self.stream)
+                                      self.ws_b.numel(), s)
 
     def bwd_end(self):
         B, T, Hq, Hkv, D = self.shape

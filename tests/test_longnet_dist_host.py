@@ -107,6 +107,9 @@ class TorchLongNetOps:
                                     causal)
                 self._fold(b, rows, h, O, L)
 
+    def cross_join(self):
+        pass
+
     def fwd_end(self):
         return self.o.clone(), self.l.clone()
 
