@@ -202,12 +202,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   // Work item: CTAs of one (b, Ulysses rank, kv-head) run together; inside it,
   // key tiles in increasing original position (the causally heaviest first).
   int gl, u, b, j, n, prob = 0;
-  if constexpr (kSub) {  // work item: (problem, kv-head, key tile)
+  if constexpr (kSub) {  // work item: (problem, kv-head of the launch, key tile)
     int wi = blockIdx.x;
     n = wi % g.n_ktiles;
     wi /= g.n_ktiles;
-    gl = wi % g.Hkv_l;
-    prob = wi / g.Hkv_l;
+    gl = a.sub.kv0 + (wi % a.sub.n_kv) * a.sub.kv_step;
+    prob = wi / a.sub.n_kv;
     u = b = j = 0;
   } else if constexpr (kLocal) {
     int wi = blockIdx.x;
@@ -618,6 +618,13 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   a.loc_j = L.loc_j;
   a.sub = L.sub;
   if (kSub) {  // one-rank geometry of every problem (see the forward's sub-problem mode)
+    if (a.sub.n_kv <= 0) {  // every kv head
+      a.sub.kv0 = 0;
+      a.sub.kv_step = 1;
+      a.sub.n_kv = a.g.Hkv_l;
+    }
+    if (a.sub.kv0 < 0 || a.sub.kv_step < 1 || a.sub.kv0 + (a.sub.n_kv - 1) * a.sub.kv_step >= a.g.Hkv_l)
+      return cudaErrorInvalidValue;
     a.g.P_u = a.g.P_r = a.g.P = a.g.n_ranks = 1;
     a.g.L = L.sub.L;
     a.g.c = kBN;
@@ -626,7 +633,7 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
     a.g.n_qtiles = (L.sub.Lq + kBM - 1) / kBM;
     a.g.n_ktiles = (L.sub.L + kBN - 1) / kBN;
   }
-  const long long blocks = kSub     ? static_cast<long long>(a.g.n_ktiles) * a.g.Hkv_l * L.sub.n_prob
+  const long long blocks = kSub     ? static_cast<long long>(a.g.n_ktiles) * a.sub.n_kv * L.sub.n_prob
                            : kLocal ? static_cast<long long>(a.g.n_ktiles) * a.g.B * a.g.Hkv_l
                                     : static_cast<long long>(a.g.n_ktiles) * a.g.P_r * a.g.P_u * a.g.B * a.g.Hkv_l;
   if (blocks <= 0) return cudaSuccess;

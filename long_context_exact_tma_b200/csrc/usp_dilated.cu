@@ -234,6 +234,11 @@ int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO
     sb.S = S;
     sb.Hq = Hq;
     sub_defaults(sb, Hkv);
+    if (rp % g.G == 0) {  // the offset's query heads o + j r sit in the kv heads o/G + j r/G, one each
+      sb.kv0 = off / g.G;
+      sb.kv_step = rp / g.G;
+      sb.n_kv = sh.n_heads;
+    }
     g.L = sh.kept;
     g.c = sh.kept;
     L.Lp = (sh.kept + 127) / 128 * 128;

@@ -114,6 +114,8 @@ struct FwdSub {
   int Lq, q_off;
   int out_h0, out_hstep;
   int kS, kw, koff, kstep, kH;
+  // kv heads the dK/dV launch walks: kv0 + x * kv_step for x < n_kv (n_kv = 0: all)
+  int kv0, kv_step, n_kv;
 };
 inline void sub_defaults(FwdSub& sb, int Hkv) {
   sb.Lq = sb.L;
@@ -125,6 +127,9 @@ inline void sub_defaults(FwdSub& sb, int Hkv) {
   sb.koff = sb.off;
   sb.kstep = sb.r;
   sb.kH = Hkv;
+  sb.kv0 = 0;
+  sb.kv_step = 1;
+  sb.n_kv = 0;
 }
 
 struct FwdLaunch {

@@ -83,6 +83,8 @@ BWD_CASES = {
     "longnet_scaled_s768": (1, 768, 4, 4, 128, True, [(64, 1), (128, 2), (256, 4), (384, 6), (768, 12)]),
     "noncausal_gqa_d64": (2, 512, 8, 2, 64, False, [(128, 1), (256, 3), (512, 8)]),
     "tiny_segments_gqa": (1, 384, 4, 2, 128, True, [(96, 1), (192, 5), (384, 7)]),
+    # r a multiple of the group size: each dK/dV launch walks only its offset's kv heads
+    "gqa_r_multiple_of_group": (1, 512, 8, 4, 128, True, [(128, 2), (256, 4), (512, 8)]),
 }
 
 
