@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
                             static_cast<size_t>(store ? tau_q : 0) * a.sub.r;
         const size_t ridx = orow * a.sub.Hq + (a.sub.out_h0 + h * a.sub.out_hstep);
         float lse_old = -INFINITY;
-        if (store) lse_old = a.sub.lse_run[ridx];
+        if (store && !a.sub.first) lse_old = a.sub.lse_run[ridx];
         const float mx = fmaxf(lse_old, lse_val);
         float w_old = 0.f, w_new = 0.f, lse_new = -INFINITY;
         if (mx != -INFINITY) {
@@ -687,7 +687,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
             float4* dst = reinterpret_cast<float4*>(a.sub.o_run + ridx * D + c0);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              const float4 ov = dst[q];
+              const float4 ov = a.sub.first ? make_float4(0.f, 0.f, 0.f, 0.f) : dst[q];
               dst[q] = make_float4(ov.x * w_old + __uint_as_float(o[q * 4 + 0]) * w_new,
                                    ov.y * w_old + __uint_as_float(o[q * 4 + 1]) * w_new,
                                    ov.z * w_old + __uint_as_float(o[q * 4 + 2]) * w_new,

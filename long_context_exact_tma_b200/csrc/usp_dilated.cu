@@ -37,7 +37,8 @@ extern "C" size_t usp_dilated_workspace_size(int B, int S, int Hq, int D) {
 namespace usp {
 
 int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S, int Hq, int Hkv, int D, int causal,
-                      int wp, int rp, float* o_run, float* lse_run, int* status, cudaStream_t st) {
+                      int wp, int rp, float* o_run, float* lse_run, int* status, cudaStream_t st, int first) {
+  if (first && rp != 1) return record_error(USP_ERR_INVALID_ARG, "only a pair with r = 1 covers every row");
   FwdLaunch L{};
   AttnGeom& g = L.g;
   g.B = B; g.S = S; g.Hq = Hq; g.Hkv = Hkv; g.D = D; g.causal = causal;
@@ -80,6 +81,7 @@ int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S,
     sb.o_run = o_run;
     sb.lse_run = lse_run;
     sub_defaults(sb, Hkv);
+    sb.first = first;
     rc = make_tmap_strided(&L.tm_q, static_cast<const uint8_t*>(q) + off * tokq, D, Hq, kept, sb.n_prob, rp * tokq,
                            wp * tokq);
     if (rc == USP_OK)
@@ -127,11 +129,23 @@ extern "C" int usp_dilated_attn_fwd(const void* q, const void* k, const void* v,
   const long long rows = static_cast<long long>(B) * S * Hq;
   float* o_run = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + usp::kStatusBytes);
   float* lse_run = o_run + rows * D;
+  // A pair with r = 1 covers every row and head: run first, it writes the running
+  // result, which then needs no initialisation (the log-sum-exp merge of the pairs
+  // does not depend on their order).
+  int p1 = -1;
+  for (int p = 0; p < n_pairs && p1 < 0; ++p)
+    if (r[p] == 1) p1 = p;
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
-  if (e == cudaSuccess) e = usp::launch_fill_running(o_run, lse_run, rows, D, st);
+  if (e == cudaSuccess && p1 < 0) e = usp::launch_fill_running(o_run, lse_run, rows, D, st);
   if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "running-result init: %s", cudaGetErrorString(e));
 
+  if (p1 >= 0) {
+    const int rc = usp::dilated_fold_pair(q, k, v, B, S, Hq, Hkv, D, causal, w[p1], 1, o_run, lse_run,
+                                          static_cast<int*>(workspace), st, 1);
+    if (rc != USP_OK) return rc;
+  }
   for (int p = 0; p < n_pairs; ++p) {
+    if (p == p1) continue;
     const int rc = usp::dilated_fold_pair(q, k, v, B, S, Hq, Hkv, D, causal, w[p], r[p], o_run, lse_run,
                                           static_cast<int*>(workspace), st);
     if (rc != USP_OK) return rc;

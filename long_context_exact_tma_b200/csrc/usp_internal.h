@@ -116,6 +116,9 @@ struct FwdSub {
   int kS, kw, koff, kstep, kH;
   // kv heads the dK/dV launch walks: kv0 + x * kv_step for x < n_kv (n_kv = 0: all)
   int kv0, kv_step, n_kv;
+  // forward: the launch's rows hold nothing yet (a pair with r = 1 run first): write
+  // the running (O, LSE) instead of folding into it, without reading it
+  int first;
 };
 inline void sub_defaults(FwdSub& sb, int Hkv) {
   sb.Lq = sb.L;
@@ -130,6 +133,7 @@ inline void sub_defaults(FwdSub& sb, int Hkv) {
   sb.kv0 = 0;
   sb.kv_step = 1;
   sb.n_kv = 0;
+  sb.first = 0;
 }
 
 struct FwdLaunch {
@@ -193,9 +197,11 @@ cudaError_t launch_attn_bwd_dq(const BwdLaunch& a, cudaStream_t stream);  // dQ 
 // Delta of every row and two row-table buffers of dilated_pair_table_floats
 // floats each (kSideStreams slots: the offsets of a pair write disjoint heads,
 // so their launches run on side streams at the same time; in the backward only
-// when Hq == Hkv, whose offsets also write disjoint kv heads). usp_status.
+// when Hq == Hkv, whose offsets also write disjoint kv heads). With `first` (only
+// for r = 1, whose launch covers every row and head) the forward writes the
+// running result instead of folding, so it needs no initialisation. usp_status.
 int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S, int Hq, int Hkv, int D, int causal,
-                      int w, int r, float* o_run, float* lse_run, int* status, cudaStream_t st);
+                      int w, int r, float* o_run, float* lse_run, int* status, cudaStream_t st, int first = 0);
 size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r);
 int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO, const float* lse,
                      const float* delta_all, float* dq_acc, float* dK, float* dV, float* lse2_t, float* delta_t, int B,

@@ -24,6 +24,8 @@ CASES = {
     "single_pair_full": (1, 1024, 2, 2, 128, True, [(1024, 1)]),
     "tiny_segments": (1, 768, 4, 2, 128, True, [(96, 1), (192, 5), (768, 7)]),
     "sparse_rows_only": (1, 1536, 6, 6, 64, True, [(1536, 4), (512, 2)]),
+    # the r = 1 pair (which writes the running result) listed last, with GQA
+    "r1_pair_listed_last": (1, 1024, 4, 2, 128, True, [(512, 2), (1024, 3), (256, 1)]),
 }
 
 
