@@ -573,7 +573,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
                                     __uint_as_float(rk[4 * q + 2]) * g.scale, __uint_as_float(rk[4 * q + 3]) * g.scale);
             float4 nv = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
                                     __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
-            if constexpr (kLocal || kSub) {  // add (travelling ring gradients; the pairs' sum)
+            // add (travelling ring gradients; the pairs' sum, but for a dilated pair with r = 1
+            // run first, which writes)
+            if (kLocal || (kSub && !a.sub.first)) {
               const float4 ok_ = dkp[q], ov = dvp[q];
               nk = make_float4(nk.x + ok_.x, nk.y + ok_.y, nk.z + ok_.z, nk.w + ok_.w);
               nv = make_float4(nv.x + ov.x, nv.y + ov.y, nv.z + ov.z, nv.w + ov.w);

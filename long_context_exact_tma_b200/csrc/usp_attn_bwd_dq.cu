@@ -494,7 +494,8 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
           const float4* acc = reinterpret_cast<const float4*>(a.dq_acc + qr * D + c0);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 ov = acc[q];
+            // (a dilated pair with r = 1 run first writes the accumulator: nothing to read)
+            const float4 ov = (kSub && a.sub.first) ? make_float4(0.f, 0.f, 0.f, 0.f) : acc[q];
             o[q * 4 + 0] = __float_as_uint(ov.x + __uint_as_float(o[q * 4 + 0]) * g.scale);
             o[q * 4 + 1] = __float_as_uint(ov.y + __uint_as_float(o[q * 4 + 1]) * g.scale);
             o[q * 4 + 2] = __float_as_uint(ov.z + __uint_as_float(o[q * 4 + 2]) * g.scale);

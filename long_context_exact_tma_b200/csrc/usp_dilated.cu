@@ -200,7 +200,9 @@ size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r) {
 
 int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO, const float* lse,
                      const float* delta_all, float* dq_acc, float* dK, float* dV, float* lse2_t, float* delta_t, int B,
-                     int S, int Hq, int Hkv, int D, int causal, int wp, int rp, int* status, cudaStream_t st) {
+                     int S, int Hq, int Hkv, int D, int causal, int wp, int rp, int* status, cudaStream_t st,
+                     int first) {
+  if (first && rp != 1) return record_error(USP_ERR_INVALID_ARG, "only a pair with r = 1 covers every row");
   BwdLaunch L{};
   AttnGeom& g = L.g;
   g.B = B; g.S = S; g.Hq = Hq; g.Hkv = Hkv; g.D = D; g.causal = causal;
@@ -248,6 +250,7 @@ int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO
     sb.S = S;
     sb.Hq = Hq;
     sub_defaults(sb, Hkv);
+    sb.first = first;  // write dQ, dK, dV instead of adding (r = 1 only: every row and head)
     if (rp % g.G == 0) {  // the offset's query heads o + j r sit in the kv heads o/G + j r/G, one each
       sb.kv0 = off / g.G;
       sb.kv_step = rp / g.G;
@@ -349,14 +352,27 @@ extern "C" int usp_dilated_attn_bwd(const void* q, const void* k, const void* v,
   float* dq_acc = delta_all + rows;
   float* lse2_t = dq_acc + rows * D;
   float* delta_t = lse2_t + tbl;
+  // As in the forward, a pair with r = 1 (every row and head) runs first and writes dQ's
+  // accumulator, dK and dV, which then need no zeroing.
+  int p1 = -1;
+  for (int p = 0; p < n_pairs && p1 < 0; ++p)
+    if (r[p] == 1) p1 = p;
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dq_acc, 0, rows * D * sizeof(float), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dK, 0, kv_elems * sizeof(float), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, kv_elems * sizeof(float), st);
+  if (p1 < 0) {
+    if (e == cudaSuccess) e = cudaMemsetAsync(dq_acc, 0, rows * D * sizeof(float), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dK, 0, kv_elems * sizeof(float), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, kv_elems * sizeof(float), st);
+  }
   if (e == cudaSuccess) e = usp::launch_bwd_preprocess(out, dO, delta_all, rows, D, st);
   if (e != cudaSuccess) return record_error(USP_ERR_CUDA, "dilated backward init: %s", cudaGetErrorString(e));
 
+  if (p1 >= 0) {
+    rc = usp::dilated_bwd_pair(q, k, v, dO, lse, delta_all, dq_acc, dK, dV, lse2_t, delta_t, B, S, Hq, Hkv, D,
+                               causal, w[p1], 1, static_cast<int*>(workspace), st, 1);
+    if (rc != USP_OK) return rc;
+  }
   for (int p = 0; p < n_pairs; ++p) {
+    if (p == p1) continue;
     rc = usp::dilated_bwd_pair(q, k, v, dO, lse, delta_all, dq_acc, dK, dV, lse2_t, delta_t, B, S, Hq, Hkv, D,
                                causal, w[p], r[p], static_cast<int*>(workspace), st);
     if (rc != USP_OK) return rc;

@@ -205,6 +205,7 @@ int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S,
 size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r);
 int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO, const float* lse,
                      const float* delta_all, float* dq_acc, float* dK, float* dV, float* lse2_t, float* delta_t, int B,
-                     int S, int Hq, int Hkv, int D, int causal, int w, int r, int* status, cudaStream_t st);
+                     int S, int Hq, int Hkv, int D, int causal, int w, int r, int* status, cudaStream_t st,
+                     int first = 0);
 
 }  // namespace usp

@@ -87,6 +87,9 @@ BWD_CASES = {
     "tiny_segments_gqa": (1, 384, 4, 2, 128, True, [(96, 1), (192, 5), (384, 7)]),
     # r a multiple of the group size: each dK/dV launch walks only its offset's kv heads
     "gqa_r_multiple_of_group": (1, 512, 8, 4, 128, True, [(128, 2), (256, 4), (512, 8)]),
+    # no r = 1 pair (the gradients start from zero) / the r = 1 pair (which writes them) listed last
+    "no_r1_pair": (1, 512, 4, 4, 128, True, [(256, 2), (512, 4)]),
+    "r1_pair_listed_last_gqa": (1, 512, 4, 2, 128, True, [(256, 2), (512, 3), (128, 1)]),
 }
 
 
