@@ -119,70 +119,55 @@ __global__ void __launch_bounds__(256) lse_merge_small_kernel(const float* o_par
 }
 
 // One warp per row; 4 bf16 (8 bytes) per lane per pass.
+// dO_r . O_r of one row of D bf16 (16-byte read-only loads: when the rows of a
+// warp's threads lie apart, the second half of each 32-byte sector comes from L1).
+__device__ __forceinline__ float row_dot_bf16(const __nv_bfloat16* a, const __nv_bfloat16* b, int D) {
+  const uint4* pa = reinterpret_cast<const uint4*>(a);
+  const uint4* pb = reinterpret_cast<const uint4*>(b);
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 x = __ldg(pa + c), y = __ldg(pb + c);
+    const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+    const __nv_bfloat162* y2 = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 fx = __bfloat1622float2(x2[k]);
+      const float2 fy = __bfloat1622float2(y2[k]);
+      acc0 = fmaf(fx.x, fy.x, acc0);
+      acc1 = fmaf(fx.y, fy.y, acc1);
+    }
+  }
+  return acc0 + acc1;
+}
+
+// Delta_r = dO_r . O_r, thread per row.
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ out,
                                                              const __nv_bfloat16* __restrict__ dO,
                                                              float* __restrict__ delta, long long rows, int D) {
-  const int lane = threadIdx.x & 31;
-  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
-       r += n_warps) {
-    float acc = 0.f;
-    for (int d4 = lane; d4 * 4 < D; d4 += 32) {
-      const uint2 a = __ldcs(reinterpret_cast<const uint2*>(out + r * D) + d4);
-      const uint2 b = __ldcs(reinterpret_cast<const uint2*>(dO + r * D) + d4);
-      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float2 fa = __bfloat1622float2(a2[k]);
-        const float2 fb = __bfloat1622float2(b2[k]);
-        acc = fmaf(fa.x, fb.x, acc);
-        acc = fmaf(fa.y, fb.y, acc);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) delta[r] = acc;
-  }
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; r < rows; r += stride)
+    delta[r] = row_dot_bf16(out + r * D, dO + r * D, D);
 }
 
-// -Delta and -LSE*log2(e) of every row (the negated forms the backward adds),
-// written per head: row (rb, tau, h) of the head-sharded layout goes to
-// [rb*Hl + h][tau] of a [n_rb*Hl][Lp] table.
+// The per-head tables of the backward kernels, thread per row: consecutive threads
+// take consecutive rows tau of one (rank-batch, head), so their -Delta and
+// -LSE*log2(e) entries are written side by side.
 __global__ void __launch_bounds__(256) bwd_prep_rows_kernel(const __nv_bfloat16* __restrict__ out,
                                                             const __nv_bfloat16* __restrict__ dO,
                                                             const float* __restrict__ lse,
                                                             float* __restrict__ delta_t, float* __restrict__ lse2_t,
                                                             long long rows, int L, int Hl, int D, int Lp) {
-  const int lane = threadIdx.x & 31;
-  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
-       r += n_warps) {
-    float acc = 0.f;
-    for (int d4 = lane; d4 * 4 < D; d4 += 32) {
-      const uint2 x = __ldcs(reinterpret_cast<const uint2*>(out + r * D) + d4);
-      const uint2 y = __ldcs(reinterpret_cast<const uint2*>(dO + r * D) + d4);
-      const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
-      const __nv_bfloat162* y2 = reinterpret_cast<const __nv_bfloat162*>(&y);
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float2 fx = __bfloat1622float2(x2[k]);
-        const float2 fy = __bfloat1622float2(y2[k]);
-        acc = fmaf(fx.x, fy.x, acc);
-        acc = fmaf(fx.y, fy.y, acc);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      const long long h = r % Hl, rt = r / Hl, tau = rt % L, rb = rt / L;
-      const long long dst = (rb * Hl + h) * Lp + tau;
-      delta_t[dst] = -acc;
-      // a row that saw no key (LSE = -inf, O = 0; masked attention) must give
-      // P = 0, as the padding rows do, not exp2(+inf)
-      const float l = lse[r];
-      lse2_t[dst] = l == -INFINITY ? -INFINITY : -l * 1.4426950408889634f;
-    }
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < rows; x += stride) {
+    const long long tau = x % L, hb = x / L;  // hb = rank-batch * Hl + head
+    const long long r = ((hb / Hl) * L + tau) * Hl + hb % Hl;
+    const long long dst = hb * Lp + tau;
+    delta_t[dst] = -row_dot_bf16(out + r * D, dO + r * D, D);
+    // a row that saw no key (LSE = -inf, O = 0; masked attention) must give
+    // P = 0, as the padding rows do, not exp2(+inf)
+    const float l = lse[r];
+    lse2_t[dst] = l == -INFINITY ? -INFINITY : -l * 1.4426950408889634f;
   }
   // Padding rows [L, Lp) of every head: LSE = +inf and Delta = 0, so a padded
   // query contributes exactly zero (P = exp2(s - inf) = 0) whatever the workspace held.
@@ -309,7 +294,7 @@ cudaError_t launch_lse_merge(const float* o_parts, const float* lse_parts, int n
 cudaError_t launch_bwd_preprocess(const void* out, const void* dO, float* delta, long long rows, int D,
                                   cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
-  bwd_preprocess_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
+  bwd_preprocess_kernel<<<grid_for(256, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
                                                                static_cast<const __nv_bfloat16*>(dO), delta,
                                                                rows, D);
   note_launch();
@@ -320,7 +305,7 @@ cudaError_t launch_bwd_prep_rows(const void* out, const void* dO, const float* l
                                  int n_rb, int L, int Hl, int D, int Lp, cudaStream_t stream) {
   const long long rows = static_cast<long long>(n_rb) * L * Hl;
   if (rows == 0) return cudaSuccess;
-  bwd_prep_rows_kernel<<<grid_for(8, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
+  bwd_prep_rows_kernel<<<grid_for(256, rows), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(out),
                                                               static_cast<const __nv_bfloat16*>(dO), lse, delta_t,
                                                               lse2_t, rows, L, Hl, D, Lp);
   note_launch();
