@@ -450,7 +450,8 @@ class CudaLongNetOps:
         self.B_ = B_
         self.BF16, self.F32 = B_.USP_BF16, B_.USP_F32
         self.shape = (B, T, Hq, Hkv, D)
-        self.stream = stream
+        # (a raw cudaStream_t handle is wrapped, so that events can be recorded on it)
+        self.stream = torch.cuda.ExternalStream(stream, device=device) if isinstance(stream, int) else stream
         self._side = None
         self._used = []
         self.ws_f = torch.zeros(B_.usp_longnet_workspace_size(B, T, Hq, D, pairs, 0), dtype=torch.uint8,
