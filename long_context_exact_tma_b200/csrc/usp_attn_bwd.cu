@@ -539,7 +539,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     // ------------------------------------------------------------ dK, dV epilogue
     // the last step's dK/dV UMMAs (and every earlier one) have landed once its ds_used arrives
     if (ok && k >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars->ds_used, (k - 1) & 1, w, kSiteBEpi));
-    if (ok) {
+    // adding the gradients of a key tile that no query saw changes nothing: no read, no write
+    const bool noop = k == 0 && (kLocal || (kSub && !a.sub.first));
+    if (ok && !noop) {
       tc_fence_after();
       const bool store = tau_k < g.L;
       size_t kr;

@@ -466,7 +466,10 @@ __global__ void __launch_bounds__(kThreadsDq, 1)
     // ------------------------------------------------------------ epilogue: dQ rows
     if (ok && it >= 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_done[(it - 1) & 1], ((it - 1) >> 1) & 1, w, kSiteQEpi));
-    if (ok) {
+    // adding the dQ of a query tile that saw no key changes nothing (unless this call
+    // writes the bf16 result, or is a dilated pair that writes the accumulator)
+    const bool noop = it == 0 && (kLocal || kSub) && a.dq == nullptr && !(kSub && a.sub.first);
+    if (ok && !noop) {
       tc_fence_after();
       const bool store = tau_q < g.Lq;
       size_t qr;

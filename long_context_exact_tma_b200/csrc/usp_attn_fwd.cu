@@ -648,7 +648,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     }
     // ------------------------------------------------------------ epilogue
     if (ok && it >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars->pv_done[t], (it - 1) & 1, w, kSiteO));
-    if (ok) {
+    // folding a tile that saw no key changes nothing (its weight is 0): no read, no write
+    const bool noop = it == 0 && (kSub ? !a.sub.first : (a.step >= 0 && a.fold));
+    if (ok && !noop) {
       tc_fence_after();
       const bool store = tau_q < g.Lq;
       const float inv_l = lb_run > 0.f ? 1.f / lb_run : 0.f;
