@@ -118,7 +118,6 @@ __global__ void __launch_bounds__(256) lse_merge_small_kernel(const float* o_par
   }
 }
 
-// One warp per row; 4 bf16 (8 bytes) per lane per pass.
 // dO_r . O_r of one row of D bf16 (16-byte read-only loads: when the rows of a
 // warp's threads lie apart, the second half of each 32-byte sector comes from L1).
 __device__ __forceinline__ float row_dot_bf16(const __nv_bfloat16* a, const __nv_bfloat16* b, int D) {
