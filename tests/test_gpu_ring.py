@@ -13,7 +13,7 @@ import oracle
 from long_context_exact_tma_b200 import api
 from long_context_exact_tma_b200 import binding as B_
 
-from helpers import GRAD_REL_L2, GRAD_STATS, assert_fwd_ok, compare_fwd, inputs, make_spec, rel_l2
+from helpers import GRAD_REL_L2, GRAD_STATS, assert_fwd_ok, compare_fwd, fwd_stats, inputs, make_spec, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -128,3 +128,64 @@ def test_ring_steps_of_every_rank_match_oracle(cuda, name, accumulate):
     errs = {n: rel_l2(to_g(g).double().numpy(), ref[n]) for n, g in (("dq", dq), ("dk", dk), ("dv", dv))}
     GRAD_STATS.append((f"ring_steps/{name}", errs))
     assert all(e <= GRAD_REL_L2 for e in errs.values()), errs
+
+
+def test_rank_full_size_s128k_usp4x2_sampled(cuda):
+    """Rank (0, 0) of the S=128K GQA USP 4x2 mesh in the launch configuration of
+    its per-rank measurement: its 2 forward ring steps folded by
+    usp_ring_fwd_accumulate into one running partial, then its 2 backward steps.
+    O, LSE and dQ of sampled rows of the rank (complete after every ring step)
+    against the oracle over the whole sequence."""
+    from usp_inputs import WORKLOADS
+    spec = dict(WORKLOADS[3])
+    B, S, Hq, Hkv, D, P_u, P_r = (spec[n] for n in ("B", "S", "Hq", "Hkv", "D", "P_u", "P_r"))
+    causal, L, Hl = spec["causal"], S // P_r, Hq // P_u
+    t = inputs(spec, which=("q", "k", "v", "do"))
+    hs = {n: api.to_head_sharded(t[n], P_u, P_r) for n in ("q", "k", "v", "do")}
+    tc = {n: x.cpu() for n, x in t.items() if n in ("q", "k", "v", "do")}
+    del t
+    q, do = hs["q"][0, 0].contiguous(), hs["do"][0, 0].contiguous()
+    ks = [hs["k"][j, 0].contiguous() for j in range(P_r)]
+    vs = [hs["v"][j, 0].contiguous() for j in range(P_r)]
+    del hs
+    torch.cuda.empty_cache()
+    rows = B * L * Hl
+    wsf = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 0), dtype=torch.uint8,
+                      device=cuda)
+    wsb = torch.zeros(B_.usp_ring_workspace_size(B, S, Hq, Hkv, D, causal, P_u, P_r, 1), dtype=torch.uint8,
+                      device=cuda)
+    o_run = torch.empty((1, rows, D), dtype=torch.float32, device=cuda)
+    l_run = torch.empty((1, rows), dtype=torch.float32, device=cuda)
+    for s in range(P_r):
+        B_.usp_ring_fwd_accumulate(q, ks[(0 - s) % P_r], vs[(0 - s) % P_r], o_run[0], l_run[0], B, S, Hq, Hkv, D,
+                                   causal, P_u, P_r, 0, 0, s, wsf, wsf.numel())
+    out = torch.empty_like(q)
+    lse = torch.empty((B, L, Hl), dtype=torch.float32, device=cuda)
+    B_.usp_lse_merge(o_run, l_run, 1, rows, D, out, B_.USP_BF16, lse)
+    dq_acc = torch.zeros((B, L, Hl, D), dtype=torch.float32, device=cuda)
+    dq = torch.empty_like(q)
+    dk = torch.zeros((B, L, Hkv // P_u, D), dtype=torch.float32, device=cuda)
+    dv = torch.zeros_like(dk)
+    B_.usp_ring_bwd_prepare(out, lse, do, B, S, Hq, Hkv, D, causal, P_u, P_r, wsb, wsb.numel())
+    for s in range(P_r):
+        B_.usp_ring_bwd_step(q, ks[(0 - s) % P_r], vs[(0 - s) % P_r], do, dq_acc, dq if s == P_r - 1 else None, dk,
+                             dv, B, S, Hq, Hkv, D, causal, P_u, P_r, 0, 0, s, wsb, wsb.numel())
+    torch.cuda.synchronize()
+    for ws in (wsf, wsb):
+        assert B_.usp_workspace_status(ws)[0] == B_.USP_OK
+    # the rank's rows in original positions, through the oracle's own layout map
+    pos = torch.arange(S, dtype=torch.float32).view(1, S, 1, 1).expand(B, S, P_u, 1).contiguous()
+    pos0 = oracle.to_head_sharded(pos, P_u, P_r)[0, 0, 0, :, 0, 0].long().numpy()
+    rng = np.random.default_rng(33)
+    loc = [(int(rng.integers(B)), int(rng.integers(Hl)), int(rng.integers(L))) for _ in range(40)]
+    loc += [(0, 0, 0), (B - 1, Hl - 1, L - 1)]
+    glob = [(b, h, int(pos0[x])) for b, h, x in loc]  # rank (i, u) = (0, 0): local head = global head
+    o_ref, lse_ref = oracle.attn_fwd_rows(tc["q"], tc["k"], tc["v"], causal, glob)
+    o_g = np.stack([out[b, x, h].float().cpu().numpy() for b, h, x in loc])
+    l_g = np.array([float(lse[b, x, h]) for b, h, x in loc])
+    assert_fwd_ok(fwd_stats(o_g, l_g, o_ref, lse_ref, name="ring_rank/s128k_usp4x2/sampled"))
+    dq_ref, _, _ = oracle.attn_dq_rows(tc["q"], tc["k"], tc["v"], tc["do"], causal, glob)
+    dq_g = np.stack([dq[b, x, h].double().cpu().numpy() for b, h, x in loc])
+    err = rel_l2(dq_g, dq_ref)
+    GRAD_STATS.append(("ring_rank/s128k_usp4x2/sampled", {"dq": err}))
+    assert err <= GRAD_REL_L2, err
