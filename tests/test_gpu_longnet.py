@@ -148,3 +148,42 @@ def test_rows_copy_bit_exact(cuda):
             ref[:, lp0 + r * k, j // (H // Hkv)] += add[:, k, j]
     torch.cuda.synchronize()
     assert torch.equal(acc, ref)
+
+
+def test_longnet_rank_full_size_s32k_sampled(cuda):
+    """Rank 0 of 4 on the S=32K LongNet schedule in the launch configuration of
+    its per-rank measurement: local pairs on its slice, and for the gathered
+    pairs every head offset's cross attention (on side streams) against the
+    segment's kept K/V rows gathered from the whole sequence. O and LSE of
+    sampled rows of the slice against the oracle's dilated attention."""
+    from long_context_exact_tma_b200 import binding as B_
+    B, S, H, D, M = 1, 32768, 16, 128, 4
+    T = S // M
+    pairs = [(2048, 1), (4096, 2), (8192, 4), (16384, 6), (32768, 12)]
+    qg, kg, vg = (normal_bf16(900 + x, (B, S, H, D), device=cuda) for x in range(3))
+    q, k, v = (x[:, :T].contiguous() for x in (qg, kg, vg))
+    ops = udist.CudaLongNetOps(B, T, H, H, D, pairs, device=cuda)
+    ops.fwd_begin()
+    for w, r in pairs:
+        if w <= T:
+            ops.fwd_local(q, k, v, True, w, r)
+            continue
+        for o in range(min(r, H)):
+            ns = (H - o + r - 1) // r
+            n_kept = (w - o + r - 1) // r
+            kc = torch.empty((B, n_kept, ns, D), dtype=torch.bfloat16, device=cuda)
+            vc = torch.empty_like(kc)
+            B_.usp_rows_copy([dict(src=x, dst=y, dtype=B_.USP_BF16, n_b=B, n_k=n_kept, n_j=ns, D=D, s_b=S * H * D,
+                                   s_k=H * D, s_h=D, s_k0=o, s_kstep=r, s_h0=o, s_hstep=r, d_b=n_kept * ns * D,
+                                   d_k=ns * D, d_h=D) for x, y in ((kg, kc), (vg, vc))])
+            ops.fwd_cross(q, kc, vc, True, w, r, o, 0)
+        ops.cross_join()
+    out, lse = ops.fwd_end()
+    torch.cuda.synchronize()
+    ops.check()
+    rng = np.random.default_rng(34)
+    rows = [(0, int(rng.integers(H)), int(rng.integers(T))) for _ in range(40)] + [(0, 0, 0), (0, H - 1, T - 1)]
+    o_ref, l_ref = oracle.dilated_fwd_rows(qg.cpu(), kg.cpu(), vg.cpu(), True, pairs, rows)
+    o_g = np.stack([out[b, i, h].float().cpu().numpy() for b, h, i in rows])
+    l_g = np.array([float(lse[b, i, h]) for b, h, i in rows])
+    assert_fwd_ok(fwd_stats(o_g, l_g, o_ref, l_ref, name="longnet_rank/s32k_rank0_of_4/sampled"))
