@@ -128,3 +128,20 @@ def rel_l2(x, ref):
     x = np.asarray(x, np.float64)
     ref = np.asarray(ref, np.float64)
     return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def sum_invariants(dk, dv, do, G):
+    """sum_j dK_j = 0 and sum_j dV_j = sum over the group of sum_i dO_i, per (b, kv-head).
+
+    The dV invariant compares the vector sum_j dV_j with its reference sum_i dO_i
+    by relative L2 against that reference (the relative L2 of the readings, over
+    the compared elements). The dK invariant's reference is 0, so its error is
+    measured against the size of dK itself, ||dK||_F."""
+    dk = dk.double()
+    dv = dv.double()
+    B, S, Hkv, D = dk.shape
+    sk = dk.sum(1)
+    nk = dk.pow(2).sum(1).sum(-1).sqrt()
+    dsum = do.double().sum(1).view(B, Hkv, G, D).sum(2)
+    sv = dv.sum(1) - dsum
+    return (sk.norm(dim=-1) / nk).max().item(), (sv.norm(dim=-1) / dsum.norm(dim=-1)).max().item()

@@ -9,7 +9,7 @@ import oracle
 from long_context_exact_tma_b200 import api
 from usp_inputs import WORKLOADS
 
-from helpers import GRAD_REL_L2, GRAD_STATS, head_shard_cpu, inputs, make_spec, rel_l2, unshard_cpu
+from helpers import GRAD_REL_L2, GRAD_STATS, head_shard_cpu, inputs, make_spec, rel_l2, unshard_cpu, sum_invariants
 
 pytestmark = pytest.mark.gpu
 
@@ -72,23 +72,6 @@ def test_bwd_small_full_tensors(cuda, name):
     assert all(e <= GRAD_REL_L2 for e in errs.values()), errs
 
 
-def _sum_invariants(dk, dv, do, G):
-    """sum_j dK_j = 0 and sum_j dV_j = sum over the group of sum_i dO_i, per (b, kv-head).
-
-    The dV invariant compares the vector sum_j dV_j with its reference sum_i dO_i
-    by relative L2 against that reference (the relative L2 of the readings, over
-    the compared elements). The dK invariant's reference is 0, so its error is
-    measured against the size of dK itself, ||dK||_F."""
-    dk = dk.double()
-    dv = dv.double()
-    B, S, Hkv, D = dk.shape
-    sk = dk.sum(1)
-    nk = dk.pow(2).sum(1).sum(-1).sqrt()
-    dsum = do.double().sum(1).view(B, Hkv, G, D).sum(2)
-    sv = dv.sum(1) - dsum
-    return (sk.norm(dim=-1) / nk).max().item(), (sv.norm(dim=-1) / dsum.norm(dim=-1)).max().item()
-
-
 @pytest.mark.parametrize("cfg", [1, 3, 4, 5])
 def test_bwd_full_size_sampled(cuda, cfg):
     spec = dict(WORKLOADS[cfg])
@@ -109,7 +92,7 @@ def test_bwd_full_size_sampled(cuda, cfg):
     dq_g = dq.double().numpy()[idx[:, 0], idx[:, 2], idx[:, 1]]
     errs = {"dq_rows": rel_l2(dq_g, dq_ref)}
     # size-independent invariants of dK, dV
-    ek, ev = _sum_invariants(dk, dv, tc["do"], G)
+    ek, ev = sum_invariants(dk, dv, tc["do"], G)
     errs.update(sum_dk=ek, sum_dv=ev)
     GRAD_STATS.append((spec["name"], errs))
     if causal:

@@ -106,3 +106,22 @@ def test_dilated_backward_full_tensors(cuda, name):
     errs = {n: rel_l2(g.double().cpu().numpy(), ref[n]) for n, g in (("dq", dq), ("dk", dk), ("dv", dv))}
     GRAD_STATS.append((f"dilated/{name}", errs))
     assert all(e <= GRAD_REL_L2 for e in errs.values()), errs
+
+
+def test_dilated_backward_longnet_s32k_invariants(cuda):
+    """The LongNet schedule at S=32K (the bench's dilated workload), backward at
+    full size through size-independent properties. The backward uses the merged
+    LSE, so a query's weights over all its pairs' keys sum to 1 (keys counted
+    once per pair): per head sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i. A kv
+    head or a pair's rows left out, or counted twice, breaks them."""
+    from helpers import GRAD_REL_L2, GRAD_STATS, sum_invariants
+    B, S, H, D = 1, 32768, 16, 128
+    q, k, v = _inputs(B, S, H, H, D, 820, cuda)
+    do = normal_bf16(821, (B, S, H, D), device=cuda)
+    o, lse = api.dilated_attn_fwd(q, k, v, True, LONGNET_PAIRS, check_status=True)
+    dq, dk, dv = api.dilated_attn_bwd(q, k, v, o, lse, do, True, LONGNET_PAIRS, check_status=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(dq.float()).all() and torch.isfinite(dk).all() and torch.isfinite(dv).all()
+    ek, ev = sum_invariants(dk.cpu(), dv.cpu(), do.cpu(), 1)
+    GRAD_STATS.append(("dilated/longnet_s32k/invariants", {"sum_dk": ek, "sum_dv": ev}))
+    assert ek <= GRAD_REL_L2 and ev <= GRAD_REL_L2, (ek, ev)
