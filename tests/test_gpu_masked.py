@@ -98,3 +98,42 @@ def test_masked_sampled_rows_s16k_ring8(cuda):
     empty = np.isneginf(l_ref)
     assert np.array_equal(np.isneginf(lg), empty) and np.all(og[empty] == 0)
     assert_fwd_ok(fwd_stats(og[~empty], lg[~empty], o_ref[~empty], l_ref[~empty], name="masked/s16k_ring8/sampled"))
+
+
+def test_block_sparse_bench_config_s16k(cuda):
+    """The block-sparse line's configuration: the S=16K ring-8 workload (32 heads)
+    with its seeded half-dense 128x128 block mask, causal. Forward on sampled rows
+    against the oracle; backward at full size through sum_j dK_j = 0 and
+    sum_j dV_j = sum_i dO_i per head, the latter over the rows that see a key."""
+    from helpers import sum_invariants
+    from usp_inputs import WORKLOADS
+    spec = dict(WORKLOADS[2])
+    B, S, Hq, Hkv, P_u, P_r = (spec[n] for n in ("B", "S", "Hq", "Hkv", "P_u", "P_r"))
+    nb = S // 128
+    bm = (np.random.default_rng(17).random((B, Hq, nb, nb)) < 0.5).astype(np.uint8)
+    t = inputs(spec, which=("q", "k", "v", "do"))
+    qh, kh, vh, doh = (api.to_head_sharded(t[n], P_u, P_r) for n in ("q", "k", "v", "do"))
+    tc = {n: t[n].cpu() for n in ("q", "k", "v", "do")}
+    del t
+    bmd = torch.tensor(bm, device=cuda)
+    out, lse = api.attn_fwd_masked(qh, kh, vh, True, P_u, P_r, block_mask=bmd, check_status=True)
+    dq, dk, dv = api.attn_bwd_masked(qh, kh, vh, out, lse, doh, True, P_u, P_r, block_mask=bmd, check_status=True)
+    torch.cuda.synchronize()
+    o, l = unshard_cpu(out, spec), lse_to_global(lse, spec)
+    rng = np.random.default_rng(12)
+    rows = [(0, int(rng.integers(Hq)), int(rng.integers(S))) for _ in range(64)] + [(0, 0, 0), (0, Hq - 1, S - 1)]
+    o_ref, l_ref = oracle.masked_fwd_rows(tc["q"], tc["k"], tc["v"], True, rows, block_mask=bm, block=128)
+    idx = np.array(rows)
+    og = o.float().numpy()[idx[:, 0], idx[:, 2], idx[:, 1]]
+    lg = l.numpy()[idx[:, 0], idx[:, 2], idx[:, 1]]
+    empty = np.isneginf(l_ref)
+    assert np.array_equal(np.isneginf(lg), empty) and np.all(og[empty] == 0)
+    assert_fwd_ok(fwd_stats(og[~empty], lg[~empty], o_ref[~empty], l_ref[~empty], name="masked/bench_s16k/sampled"))
+    # a row sees a key iff one of its query block's blocks up to the diagonal is kept
+    sees = np.cumsum(bm, axis=-1)[..., np.arange(nb), np.arange(nb)] > 0  # [B, Hq, nb]
+    row_sees = torch.tensor(np.repeat(sees, 128, axis=-1)).permute(0, 2, 1)  # [B, S, Hq]
+    do_seen = tc["do"].double() * row_sees.unsqueeze(-1)
+    ek, ev = sum_invariants(unshard_cpu(dk, spec), unshard_cpu(dv, spec), do_seen, Hq // Hkv)
+    GRAD_STATS.append(("masked/bench_s16k/invariants", {"sum_dk": ek, "sum_dv": ev}))
+    assert torch.isfinite(dq.float()).all()
+    assert ek <= GRAD_REL_L2 and ev <= GRAD_REL_L2, (ek, ev)
