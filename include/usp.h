@@ -376,8 +376,9 @@ size_t usp_dilated_workspace_size(int B, int S, int Hq, int D);
  *   workspace  usp_dilated_bwd_workspace_size(B, S, Hq, D, n_pairs, w, r)
  *              bytes (status, Delta of every row, an fp32 dQ, and one slot of
  *              the row tables of the largest launch per head offset, up to
- *              16: with Hq == Hkv the head offsets of a pair run on up to 16
- *              streams at once, the forward's too); 0 for an unsupported shape.
+ *              16: the head offsets of a pair write disjoint rows and run on
+ *              up to 16 streams at once, the forward's too); 0 for an
+ *              unsupported shape.
  */
 size_t usp_dilated_bwd_workspace_size(int B, int S, int Hq, int D, int n_pairs, const int* w, const int* r);
 int usp_dilated_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,

@@ -219,10 +219,11 @@ int dilated_bwd_pair(const void* q, const void* k, const void* v, const void* dO
   L.dq = nullptr;
   L.dq_acc = dq_acc;
   const unsigned long long tokq = 2ull * Hq * D, tokkv = 2ull * Hkv * D;
-  // With Hq == Hkv the offsets write disjoint dK/dV heads as well as dQ heads:
-  // side streams, each with its own row-table slot.
+  // Offset o's launches write dQ, dK and dV only at the rows o + tau r of each
+  // segment (whatever the kv heads they walk), so the offsets' writes are
+  // disjoint: side streams, each with its own row-table slot.
   const int n_off = rp < Hq ? rp : Hq;
-  const int n_st = (n_off > 1 && Hq == Hkv) ? (n_off < kSideStreams ? n_off : kSideStreams) : 0;
+  const int n_st = n_off > 1 ? (n_off < kSideStreams ? n_off : kSideStreams) : 0;
   const size_t slot = slot_floats(B, S, Hq, wp, rp);
   cudaStream_t side[kSideStreams];
   if (n_st) {

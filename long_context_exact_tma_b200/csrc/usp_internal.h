@@ -195,11 +195,11 @@ cudaError_t launch_attn_bwd_dq(const BwdLaunch& a, cudaStream_t stream);  // dQ 
 // folds the pair's result into the running fp32 (O, LSE); the backward adds the
 // pair's dQ (into the fp32 dq_acc), dK and dV (fp32), with the final LSE and
 // Delta of every row and two row-table buffers of dilated_pair_table_floats
-// floats each (kSideStreams slots: the offsets of a pair write disjoint heads,
-// so their launches run on side streams at the same time; in the backward only
-// when Hq == Hkv, whose offsets also write disjoint kv heads). With `first` (only
-// for r = 1, whose launch covers every row and head) the forward writes the
-// running result instead of folding, so it needs no initialisation. usp_status.
+// floats each (kSideStreams slots: the offsets of a pair write disjoint rows,
+// o + tau r of each segment, so their launches run on side streams at the same
+// time). With `first` (only for r = 1, whose launch covers every row and head)
+// the forward writes the running result instead of folding, so it needs no
+// initialisation. usp_status.
 int dilated_fold_pair(const void* q, const void* k, const void* v, int B, int S, int Hq, int Hkv, int D, int causal,
                       int w, int r, float* o_run, float* lse_run, int* status, cudaStream_t st, int first = 0);
 size_t dilated_pair_table_floats(int B, int S, int Hq, int w, int r);

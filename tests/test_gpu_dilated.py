@@ -108,20 +108,23 @@ def test_dilated_backward_full_tensors(cuda, name):
     assert all(e <= GRAD_REL_L2 for e in errs.values()), errs
 
 
-def test_dilated_backward_longnet_s32k_invariants(cuda):
-    """The LongNet schedule at S=32K (the bench's dilated workload), backward at
-    full size through size-independent properties. The backward uses the merged
-    LSE, so a query's weights over all its pairs' keys sum to 1 (keys counted
-    once per pair): per head sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i. A kv
-    head or a pair's rows left out, or counted twice, breaks them."""
+@pytest.mark.parametrize("Hkv", [16, 4])
+def test_dilated_backward_longnet_s32k_invariants(cuda, Hkv):
+    """The LongNet schedule at S=32K (the bench's dilated workload, and its GQA
+    form with 4 query heads per kv head), backward at full size through
+    size-independent properties. The backward uses the merged LSE, so a query's
+    weights over all its pairs' keys sum to 1 (keys counted once per pair): per
+    kv head sum_j dK_j = 0 and sum_j dV_j = the sum of dO_i over the group's
+    query heads. A kv head or a pair's rows left out, counted twice, or an add
+    lost between the head offsets' launches (which run side by side) breaks them."""
     from helpers import GRAD_REL_L2, GRAD_STATS, sum_invariants
     B, S, H, D = 1, 32768, 16, 128
-    q, k, v = _inputs(B, S, H, H, D, 820, cuda)
+    q, k, v = _inputs(B, S, H, Hkv, D, 820, cuda)
     do = normal_bf16(821, (B, S, H, D), device=cuda)
     o, lse = api.dilated_attn_fwd(q, k, v, True, LONGNET_PAIRS, check_status=True)
     dq, dk, dv = api.dilated_attn_bwd(q, k, v, o, lse, do, True, LONGNET_PAIRS, check_status=True)
     torch.cuda.synchronize()
     assert torch.isfinite(dq.float()).all() and torch.isfinite(dk).all() and torch.isfinite(dv).all()
-    ek, ev = sum_invariants(dk.cpu(), dv.cpu(), do.cpu(), 1)
-    GRAD_STATS.append(("dilated/longnet_s32k/invariants", {"sum_dk": ek, "sum_dv": ev}))
+    ek, ev = sum_invariants(dk.cpu(), dv.cpu(), do.cpu(), H // Hkv)
+    GRAD_STATS.append((f"dilated/longnet_s32k_hkv{Hkv}/invariants", {"sum_dk": ek, "sum_dv": ev}))
     assert ek <= GRAD_REL_L2 and ev <= GRAD_REL_L2, (ek, ev)
