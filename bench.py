@@ -43,8 +43,8 @@ UNIT = "TFLOP/s"
 # dK/dV kernel on causal_fwd_s16k_ring8, from an ncu capture of that kernel.
 # Reported only while the kernel's sources hash to what was captured (else the
 # figure is stale: null).
-DKDV_TRAFFIC = {"workload": "causal_fwd_s16k_ring8", "bytes": 1033061376,
-                "sources_sha256": "ccd52666330460259699b1d9cd4c451dc2499691f7be82113d6552936d78842d"}
+DKDV_TRAFFIC = {"workload": "causal_fwd_s16k_ring8", "bytes": 781033728,
+                "sources_sha256": "efaf41de641c87d3408e1460971a064274774df578ded8a458e1663acd49aec7"}
 DKDV_SOURCES = ("usp_attn_bwd.cu", "usp_attn_common.cuh", "usp_ptx.cuh", "usp_internal.h")
 
 
@@ -192,12 +192,13 @@ class Step:
                    "do": torch.empty((P_r, P_u, B, L, Hq // P_u, D), dtype=bf, device=dev)}
         self.out = torch.empty_like(self.hs["q"])
         self.lse = torch.empty(self.hs["q"].shape[:-1], dtype=torch.float32, device=dev)
+        # gradients in the inputs' type (bf16, accumulated in fp32 on chip)
         self.dq = torch.empty_like(self.hs["q"])
-        self.dk = torch.empty(self.hs["k"].shape, dtype=torch.float32, device=dev)
-        self.dv = torch.empty(self.hs["v"].shape, dtype=torch.float32, device=dev)
+        self.dk = torch.empty_like(self.hs["k"])
+        self.dv = torch.empty_like(self.hs["v"])
         self.o_rm = torch.empty((P, B, S // P, Hq, D), dtype=bf, device=dev)
         self.dq_rm = torch.empty_like(self.o_rm)
-        self.dk_rm = torch.empty((P, B, S // P, Hkv, D), dtype=torch.float32, device=dev)
+        self.dk_rm = torch.empty((P, B, S // P, Hkv, D), dtype=bf, device=dev)
         self.dv_rm = torch.empty_like(self.dk_rm)
         self.ws_f = api.workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, w["causal"], P_u, P_r, 0, 0), dev)
         self.ws_b = api.workspace(B_.usp_attn_workspace_size(B, S, Hq, Hkv, D, w["causal"], P_u, P_r, 0, 1), dev)
@@ -243,8 +244,8 @@ class Step:
         B_.usp_attn_bwd_prepare(self.out, self.lse, self.hs["do"], *geo, ws_b, ws_b.numel(), st)
         if ev:
             ev["dkdv"][0].record(st)
-        B_.usp_attn_bwd_dkdv(self.hs["q"], self.hs["k"], self.hs["v"], self.hs["do"], self.dk, self.dv, *geo,
-                             ws_b, ws_b.numel(), st)
+        B_.usp_attn_bwd_dkdv_bf16(self.hs["q"], self.hs["k"], self.hs["v"], self.hs["do"], self.dk, self.dv, *geo,
+                                  ws_b, ws_b.numel(), st)
         if ev:
             ev["dkdv"][1].record(st)
         B_.usp_attn_bwd_dq(self.hs["q"], self.hs["k"], self.hs["v"], self.hs["do"], self.dq, *geo,
@@ -766,6 +767,7 @@ def bench_ours(args, w, world, rank, local):
                    "global_batch": w["B"] * world, "seq_len": w["S"],
                    "parallelism": f"{world} independent replicas x (USP {w['P_u']}x{w['P_r']} virtual ranks)",
                    "l2": l2_note(step, dev)},
+        "grad_dtype": "bf16 (dQ, dK, dV; fp32 accumulation on chip)",
         "pct_of_peak": round(100.0 * value / world / peak_tf, 2),
         "fwd_tflops": round(f_fwd / (fwd_ms / 1e3) / 1e12, 2),
         # the Ulysses seq->head all-to-all of Q, K, V (one launch): read + write of every element once
@@ -778,7 +780,7 @@ def bench_ours(args, w, world, rank, local):
                   "peak_source": f"{peak_src} hbm_gbs"},
         "exp_count_fwd": int(flops_fwd(w) / (4 * w["D"])),  # B*Hq*S^2 (/2 causal); the backward recomputes them
         "bwd_tflops": round(bwd_tf, 2),
-        "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel (key-major dK/dV; usp_attn_bwd_dkdv call)",
+        "roofline": {"bound": "tensor", "kernel": "attn_bwd_kernel (key-major dK/dV; usp_attn_bwd_dkdv_bf16 call)",
                      "achieved": round(dkdv_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(dkdv_tf / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "launch_ms": round(dkdv_ms, 4), "traffic": dkdv_traffic(w["name"])},

@@ -193,6 +193,9 @@ int usp_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
  *                         accumulated on chip and written once as bf16.
  * dkdv and dq read only the prepared workspace and the inputs, so they may run in
  * either order (or on two streams) after prepare.
+ * usp_attn_bwd_dkdv_bf16 is usp_attn_bwd_dkdv with dK and dV returned in the
+ * inputs' type, as dQ is: head-sharded bf16 [P_r][P_u][B][L][Hkv/P_u][D], each
+ * element the fp32 sum of usp_attn_bwd_dkdv rounded once to bf16 (nearest even).
  */
 int usp_attn_bwd_prepare(const void* out, const float* lse, const void* dO, int B, int S, int Hq, int Hkv, int D,
                          int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream);
@@ -201,6 +204,9 @@ int usp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* d
                       void* stream);
 int usp_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dQ, int B, int S, int Hq,
                     int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes, void* stream);
+int usp_attn_bwd_dkdv_bf16(const void* q, const void* k, const void* v, const void* dO, void* dK, void* dV, int B,
+                           int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, void* workspace,
+                           size_t ws_bytes, void* stream);
 
 /*
  * Sparse and variable-length attention under the Ulysses layout

@@ -143,10 +143,14 @@ def attn_fwd(q, k, v, causal: bool, P_u: int, P_r: int, mode: int = B_.USP_MODE_
 
 
 def attn_bwd(q, k, v, out, lse, dO, causal: bool, P_u: int, P_r: int, ws=None, dq=None, dk=None, dv=None,
-             stream=None, check_status: bool = False):
-    """Backward; returns (dQ bf16 like q, dK fp32 like k, dV fp32 like v). With
-    check_status=True the call synchronises and raises on a timed-out device wait."""
+             stream=None, check_status: bool = False, grad_dtype=torch.float32):
+    """Backward; returns (dQ bf16 like q, dK like k, dV like v), dK and dV in
+    grad_dtype: fp32 (usp_attn_bwd) or bf16 (usp_attn_bwd_prepare, _dkdv_bf16 and
+    _dq). With check_status=True the call synchronises and raises on a timed-out
+    device wait."""
     _require_cuda(q, k, v, out, lse, dO)
+    if grad_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("grad_dtype must be torch.float32 or torch.bfloat16")
     Pr, Pu, B, L, Hql, D = q.shape
     Hkv = k.shape[4] * P_u
     Hq = Hql * P_u
@@ -155,10 +159,18 @@ def attn_bwd(q, k, v, out, lse, dO, causal: bool, P_u: int, P_r: int, ws=None, d
     if ws is None:
         ws = workspace(need, q.device)
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty(k.shape, dtype=torch.float32, device=k.device) if dk is None else dk
-    dv = torch.empty(v.shape, dtype=torch.float32, device=v.device) if dv is None else dv
-    B_.usp_attn_bwd(q, k, v, out, lse, dO, dq, dk, dv, B, S, Hq, Hkv, D, causal, P_u, P_r, ws, ws.numel(),
-                    stream)
+    dk = torch.empty(k.shape, dtype=grad_dtype, device=k.device) if dk is None else dk
+    dv = torch.empty(v.shape, dtype=grad_dtype, device=v.device) if dv is None else dv
+    if dk.dtype != grad_dtype or dv.dtype != grad_dtype:
+        raise ValueError("dk and dv must have dtype grad_dtype")
+    if grad_dtype == torch.float32:
+        B_.usp_attn_bwd(q, k, v, out, lse, dO, dq, dk, dv, B, S, Hq, Hkv, D, causal, P_u, P_r, ws, ws.numel(),
+                        stream)
+    else:
+        geo = (B, S, Hq, Hkv, D, causal, P_u, P_r)
+        B_.usp_attn_bwd_prepare(out, lse, dO, *geo, ws, ws.numel(), stream)
+        B_.usp_attn_bwd_dkdv_bf16(q, k, v, dO, dk, dv, *geo, ws, ws.numel(), stream)
+        B_.usp_attn_bwd_dq(q, k, v, dO, dq, *geo, ws, ws.numel(), stream)
     if check_status:
         check_workspace(ws, stream)
     return dq, dk, dv

@@ -103,6 +103,7 @@ SIGNATURES = {
     "usp_attn_bwd_masked": (_I, [_P] * 9 + [_I] * 8 + [ctypes.POINTER(AttnMask), _P, _SZ, _P]),
     "usp_attn_bwd_prepare": (_I, [_P, _P, _P] + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_dkdv": (_I, [_P] * 6 + [_I] * 8 + [_P, _SZ, _P]),
+    "usp_attn_bwd_dkdv_bf16": (_I, [_P] * 6 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_dq": (_I, [_P] * 5 + [_I] * 8 + [_P, _SZ, _P]),
     "usp_attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 8 + [_P]),
     "usp_attn_bwd_noalloc_status": (_I, [_P, _P]),
@@ -403,6 +404,13 @@ def usp_attn_bwd_dkdv(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, w
                       check=True):
     rc = lib().usp_attn_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dK), _ptr(dV), B, S, Hq, Hkv, D,
                                  int(causal), P_u, P_r, _ptr(workspace), ws_bytes, _stream(stream))
+    return _check(rc) if check else rc
+
+
+def usp_attn_bwd_dkdv_bf16(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes,
+                           stream=None, check=True):
+    rc = lib().usp_attn_bwd_dkdv_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dK), _ptr(dV), B, S, Hq, Hkv, D,
+                                      int(causal), P_u, P_r, _ptr(workspace), ws_bytes, _stream(stream))
     return _check(rc) if check else rc
 
 

@@ -458,16 +458,22 @@ int bwd_launch_setup(const void* q, const void* k, const void* v, const void* dO
   return USP_OK;
 }
 
-int bwd_dkdv_impl(const void* q, const void* k, const void* v, const void* dO, float* dK, float* dV, int B, int S,
-                  int Hq, int Hkv, int D, int causal, int P_u, int P_r, const usp_attn_mask* mask, void* workspace,
-                  size_t ws_bytes, void* stream) {
+// dK, dV in fp32 (bf16 = 0) or, rounded once from the fp32 sums, in bf16 (bf16 = 1)
+int bwd_dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void* dK, void* dV, int bf16, int B,
+                  int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, const usp_attn_mask* mask,
+                  void* workspace, size_t ws_bytes, void* stream) {
   if (!dK || !dV) return fail(USP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(dK) || !aligned16(dV)) return fail(USP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   BwdLaunch L{};
   const int rc = bwd_launch_setup(q, k, v, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes, &L);
   if (rc != USP_OK) return rc;
-  L.dk = dK;
-  L.dv = dV;
+  if (bf16) {
+    L.dk_bf16 = dK;
+    L.dv_bf16 = dV;
+  } else {
+    L.dk = static_cast<float*>(dK);
+    L.dv = static_cast<float*>(dV);
+  }
   const cudaError_t e = launch_attn_bwd(L, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? USP_OK : cuda_fail(e, "attention backward (dK, dV) launch");
 }
@@ -500,7 +506,7 @@ int attn_bwd_impl(const void* q, const void* k, const void* v, const void* out, 
   if ((rc = usp_attn_bwd_prepare(out, lse, dO, B, S, Hq, Hkv, D, causal, P_u, P_r, workspace, ws_bytes, stream)) !=
       USP_OK)
     return rc;
-  if ((rc = bwd_dkdv_impl(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes,
+  if ((rc = bwd_dkdv_impl(q, k, v, dO, dK, dV, 0, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes,
                           stream)) != USP_OK)
     return rc;
   return bwd_dq_impl(q, k, v, dO, dQ, B, S, Hq, Hkv, D, causal, P_u, P_r, mask, workspace, ws_bytes, stream);
@@ -512,7 +518,14 @@ extern "C" {
 int usp_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, float* dK, float* dV, int B,
                       int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, void* workspace, size_t ws_bytes,
                       void* stream) {
-  return bwd_dkdv_impl(q, k, v, dO, dK, dV, B, S, Hq, Hkv, D, causal, P_u, P_r, nullptr, workspace, ws_bytes,
+  return bwd_dkdv_impl(q, k, v, dO, dK, dV, 0, B, S, Hq, Hkv, D, causal, P_u, P_r, nullptr, workspace, ws_bytes,
+                       stream);
+}
+
+int usp_attn_bwd_dkdv_bf16(const void* q, const void* k, const void* v, const void* dO, void* dK, void* dV, int B,
+                           int S, int Hq, int Hkv, int D, int causal, int P_u, int P_r, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  return bwd_dkdv_impl(q, k, v, dO, dK, dV, 1, B, S, Hq, Hkv, D, causal, P_u, P_r, nullptr, workspace, ws_bytes,
                        stream);
 }
 

@@ -66,6 +66,8 @@ struct BwdArgs {
   int Lp;
   float* dk;           // fp32 [n_ranks][B][L][Hkv_l][D]
   float* dv;
+  void* dk_bf16;       // mesh mode: when set, dK and dV are written here as bf16 instead
+  void* dv_bf16;
   int* status;
   unsigned long long wait_ns;
   int loc_i, loc_u, loc_j;  // local mode: query rank (i, u), KV block of ring rank j
@@ -566,7 +568,25 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) rk[c] = rv[c] = 0u;
         }
-        if (store) {
+        if (store && !kLocal && !kSub && a.dk_bf16 != nullptr) {
+          // the gradients in the inputs' type, rounded once from the fp32 sums
+          uint4* dkp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.dk_bf16) + kr * D + c0);
+          uint4* dvp = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.dv_bf16) + kr * D + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 hk, hv;
+            hk.x = pack_bf16x2(__uint_as_float(rk[8 * q + 0]) * g.scale, __uint_as_float(rk[8 * q + 1]) * g.scale);
+            hk.y = pack_bf16x2(__uint_as_float(rk[8 * q + 2]) * g.scale, __uint_as_float(rk[8 * q + 3]) * g.scale);
+            hk.z = pack_bf16x2(__uint_as_float(rk[8 * q + 4]) * g.scale, __uint_as_float(rk[8 * q + 5]) * g.scale);
+            hk.w = pack_bf16x2(__uint_as_float(rk[8 * q + 6]) * g.scale, __uint_as_float(rk[8 * q + 7]) * g.scale);
+            hv.x = pack_bf16x2(__uint_as_float(rv[8 * q + 0]), __uint_as_float(rv[8 * q + 1]));
+            hv.y = pack_bf16x2(__uint_as_float(rv[8 * q + 2]), __uint_as_float(rv[8 * q + 3]));
+            hv.z = pack_bf16x2(__uint_as_float(rv[8 * q + 4]), __uint_as_float(rv[8 * q + 5]));
+            hv.w = pack_bf16x2(__uint_as_float(rv[8 * q + 6]), __uint_as_float(rv[8 * q + 7]));
+            dkp[q] = hk;
+            dvp[q] = hv;
+          }
+        } else if (store) {
           float4* dkp = reinterpret_cast<float4*>(a.dk + kr * D + c0);
           float4* dvp = reinterpret_cast<float4*>(a.dv + kr * D + c0);
 #pragma unroll
@@ -615,6 +635,10 @@ cudaError_t launch_bwd_d(const BwdLaunch& L, cudaStream_t stream) {
   a.Lp = L.Lp;
   a.dk = L.dk;
   a.dv = L.dv;
+  a.dk_bf16 = L.dk_bf16;
+  a.dv_bf16 = L.dv_bf16;
+  if ((kLocal || kSub) && (L.dk_bf16 != nullptr || L.dv_bf16 != nullptr)) return cudaErrorInvalidValue;
+  if ((L.dk_bf16 == nullptr) != (L.dv_bf16 == nullptr)) return cudaErrorInvalidValue;
   a.status = L.status;
   a.wait_ns = L.wait_ns;
   a.loc_i = L.loc_i;

@@ -177,6 +177,8 @@ struct BwdLaunch {
   void* dq;            // bf16, q layout (written by the query-major kernel)
   float* dk;           // fp32, k layout
   float* dv;           // fp32, v layout
+  void* dk_bf16;       // mesh mode only: when set, dK and dV are written as bf16 here (k, v layout)
+  void* dv_bf16;       // instead of dk, dv
   int* status;
   unsigned long long wait_ns;
   MaskArgs mask;       // masked variant when mask.bm or mask.cu is set

@@ -155,3 +155,43 @@ def test_bwd_phases_compose_to_usp_attn_bwd(cuda):
     assert B_.usp_workspace_status(ws)[0] == 0
     for a_, b_ in zip(whole, (dq, dk, dv)):
         assert torch.equal(a_, b_)
+
+
+BF16_GRAD_CASES = ["tiny_causal_usp2x2", "gqa_usp2x2_unaligned", "d64_ragged_unaligned", "batch2_causal_ring4",
+                   "noncausal_usp2x2_gqa_d64"]
+
+
+def _bf16_vs_f32(spec, t, dev):
+    P_u, P_r, causal = spec["P_u"], spec["P_r"], spec["causal"]
+    q, k, v, do = (head_shard_cpu(t[n], spec).to(dev) for n in ("q", "k", "v", "do"))
+    out, lse = api.attn_fwd(q, k, v, causal, P_u, P_r, check_status=True)
+    g32 = api.attn_bwd(q, k, v, out, lse, do, causal, P_u, P_r, check_status=True)
+    g16 = api.attn_bwd(q, k, v, out, lse, do, causal, P_u, P_r, check_status=True, grad_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert g16[1].dtype == torch.bfloat16 and g16[2].dtype == torch.bfloat16
+    # the same fp32 sums, rounded once to the nearest bf16 (ties to even), as torch rounds
+    assert torch.equal(g16[0], g32[0])
+    assert torch.equal(g16[1], g32[1].to(torch.bfloat16))
+    assert torch.equal(g16[2], g32[2].to(torch.bfloat16))
+    return g16
+
+
+@pytest.mark.parametrize("name", BF16_GRAD_CASES)
+def test_bwd_bf16_grads_small(cuda, name):
+    """usp_attn_bwd_dkdv_bf16: dK, dV in bf16 are the fp32 call's values rounded to
+    bf16 element by element, and stay within the gradient bound of the oracle."""
+    spec = SMALL[name]
+    t = inputs(spec, which=("q", "k", "v", "do"))
+    dq, dk, dv = (unshard_cpu(x, spec) for x in _bf16_vs_f32(spec, t, cuda))
+    ref = oracle_grads({n: t[n].cpu() for n in ("q", "k", "v", "do")}, spec)
+    errs = {n: rel_l2(g.double().numpy(), ref[n]) for n, g in (("dq", dq), ("dk", dk), ("dv", dv))}
+    GRAD_STATS.append((f"bf16 grads/{name}", errs))
+    assert all(e <= GRAD_REL_L2 for e in errs.values()), errs
+
+
+def test_bwd_bf16_grads_s16k_ring8(cuda):
+    """The same element-wise rounding identity on the S=16K ring-8 workload, in
+    the launch configuration the bench step times."""
+    spec = dict(WORKLOADS[2])
+    t = inputs(spec, which=("q", "k", "v", "do"))
+    _bf16_vs_f32(spec, t, cuda)
