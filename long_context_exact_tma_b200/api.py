@@ -148,9 +148,9 @@ def attn_bwd(q, k, v, out, lse, dO, causal: bool, P_u: int, P_r: int, ws=None, d
     grad_dtype: fp32 (usp_attn_bwd) or bf16 (usp_attn_bwd_prepare, _dkdv_bf16 and
     _dq). With check_status=True the call synchronises and raises on a timed-out
     device wait."""
-    _require_cuda(q, k, v, out, lse, dO)
     if grad_dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("grad_dtype must be torch.float32 or torch.bfloat16")
+    _require_cuda(q, k, v, out, lse, dO)
     Pr, Pu, B, L, Hql, D = q.shape
     Hkv = k.shape[4] * P_u
     Hq = Hql * P_u

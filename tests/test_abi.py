@@ -114,6 +114,27 @@ def test_bwd_rejects_bad_arguments():
     assert L.usp_attn_bwd(*bad) == B_.USP_ERR_INVALID_ARG
 
 
+def test_bwd_dkdv_bf16_rejects_bad_arguments():
+    L = B_.lib()
+    args = [FAKE] * 6 + [1, 256, 2, 2, 64, 1, 2, 2, FAKE, 256, None]
+    assert L.usp_attn_bwd_dkdv_bf16(*args) == B_.USP_ERR_WORKSPACE  # needs the prepared tables
+    bad = list(args)
+    bad[10] = 48  # D
+    assert L.usp_attn_bwd_dkdv_bf16(*bad) == B_.USP_ERR_UNSUPPORTED
+    for i in (4, 5):  # dK, dV
+        bad = list(args)
+        bad[i] = None
+        assert L.usp_attn_bwd_dkdv_bf16(*bad) == B_.USP_ERR_INVALID_ARG
+
+
+def test_attn_bwd_rejects_other_gradient_types():
+    import torch
+    from long_context_exact_tma_b200 import api
+    x = torch.zeros(1)
+    with pytest.raises(ValueError):
+        api.attn_bwd(x, x, x, x, x, x, True, 1, 1, grad_dtype=torch.float16)
+
+
 @pytest.mark.parametrize("name", ["usp_zigzag_shard", "usp_zigzag_unshard", "usp_seq2head_permute",
                                   "usp_head2seq_permute"])
 def test_layout_rejects_bad_arguments(name):
