@@ -26,7 +26,9 @@
 //               Thread = key row, in two phases per step: P^T as bf16 over the S^T
 //               columns as soon as S^T lands (dV starts on it while dP^T is still
 //               in flight), then dS^T over the dP^T columns (dK starts on it). At
-//               the end dK and dV rows (fp32) are written out.
+//               the end dK and dV rows are written out in fp32 (added to the
+//               buffers in the local and sub-problem modes) or, in the mesh mode
+//               when asked, rounded once to bf16.
 // Every wait is bounded (usp_ptx.cuh).
 #include <math.h>
 
