@@ -156,3 +156,51 @@ def test_usp_mesh_schedule_on_gloo(P_u, P_r, causal):
     for rank, errs in res.items():
         # the partials and accumulators are fp32 buffers, as on the GPU: fp32 rounding only
         assert all(e < 1e-5 for e in errs.values()), (rank, errs)
+
+
+def _worker_peer_lost(rank, world, port, P_u, P_r, results):
+    """Rank 1 leaves between steps (before the step's first collective, none of
+    its work in flight); rank 0 runs the step and must get an error from the
+    process group within its timeout instead of waiting for ever."""
+    import datetime
+    import time
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import sys
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    from long_context_exact_tma_b200 import dist as udist
+    B, S, Hq, Hkv, D = 1, 2 * world * 6, 4, 2, 8
+    geo = udist.Geometry(B, S, Hq, Hkv, D, True, P_u, P_r)
+    mesh = udist.Mesh(P_u, P_r)
+    if rank == 1:
+        results[rank] = "left"
+        os._exit(0)  # gone without a goodbye: no destroy_process_group
+    T = S // world
+    x = {n: torch.zeros((B, T, h, D), dtype=torch.float64) for n, h in (("q", Hq), ("k", Hkv), ("v", Hkv))}
+    t0 = time.monotonic()
+    try:
+        udist.usp_attention(x["q"], x["k"], x["v"], geo, mesh, TorchOps(geo, mesh))
+        results[rank] = ("no error", time.monotonic() - t0)
+    except Exception as e:  # the process group's error for the lost peer
+        results[rank] = ("error", time.monotonic() - t0, type(e).__name__)
+    os._exit(0)
+
+
+@pytest.mark.timeout(180)
+@pytest.mark.parametrize("P_u,P_r", [(2, 1), (1, 2)])
+def test_usp_mesh_lost_peer_raises_instead_of_hanging(P_u, P_r):
+    """Failure detection on the host: a rank that leaves the mesh makes the
+    surviving rank's next collective (the Ulysses all-to-all, or the ring's
+    send/receive) end with an error within the process group's 5 s timeout."""
+    world = P_u * P_r
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_worker_peer_lost, args=(world, _free_port(), P_u, P_r, results), nprocs=world,
+                           start_method="spawn", join=True)
+        res = dict(results)
+    assert res.get(1) == "left"
+    status, elapsed = res[0][0], res[0][1]
+    assert status == "error", res[0]
+    assert elapsed < 60, res[0]
