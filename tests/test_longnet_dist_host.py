@@ -236,3 +236,48 @@ def test_longnet_rows_against_brute_force_and_the_library(T, w, r):
             assert kept[k_lo:k_lo + n_rows] == mine
             seen += mine
         assert seen == kept
+
+
+def _worker_peer_lost(rank, world, port, results):
+    """Rank 1 leaves between steps; rank 0 runs the forward, whose first gathered
+    pair all-gathers kept K/V rows over the segment, and must get an error from
+    the process group within its timeout instead of waiting for ever."""
+    import datetime
+    import time
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import sys
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    from long_context_exact_tma_b200 import dist as udist
+    _, T, Hq, Hkv, causal, pairs = CASES["w2_causal"]
+    B, D = 1, 8
+    lm = udist.LongNetMesh(world * T, pairs)
+    if rank == 1:
+        results[rank] = "left"
+        os._exit(0)  # gone without a goodbye: no destroy_process_group
+    q = torch.zeros((B, T, Hq, D), dtype=torch.float64)
+    kv = torch.zeros((B, T, Hkv, D), dtype=torch.float64)
+    t0 = time.monotonic()
+    try:
+        udist.longnet_attn_fwd(q, kv, kv, pairs, causal, lm, TorchLongNetOps(B, T, Hq, Hkv, D))
+        results[rank] = ("no error", time.monotonic() - t0)
+    except Exception as e:  # the process group's error for the lost peer
+        results[rank] = ("error", time.monotonic() - t0, type(e).__name__)
+    os._exit(0)
+
+
+@pytest.mark.timeout(180)
+def test_longnet_lost_peer_raises_instead_of_hanging():
+    """Failure detection on the host for LongNet's layout: with one rank gone, the
+    survivor's all-gather of a segment's kept rows ends with an error within the
+    process group's 5 s timeout."""
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_worker_peer_lost, args=(2, _free_port(), results), nprocs=2, join=True,
+                           start_method="spawn")
+        res = dict(results)
+    assert res.get(1) == "left"
+    assert res[0][0] == "error", res[0]
+    assert res[0][1] < 60, res[0]
