@@ -1,5 +1,6 @@
 """Host-side logic of bench.py on CPU: the max-over-ranks timing reduction with
-two gloo ranks (the data path has no collective), and the clock-sample summary."""
+two gloo ranks (the data path has no collective), the clock-sample summary, the
+FLOP convention and when the stored dK/dV DRAM figure is reported."""
 import os
 import socket
 
@@ -54,3 +55,14 @@ def test_flop_convention():
     assert bench.flops_fwd(w) == 4 * 32 * 16384 ** 2 * 128 / 2
     w["causal"] = False
     assert bench.flops_fwd(w) == 4 * 32 * 16384 ** 2 * 128
+
+
+def test_dkdv_traffic_is_reported_only_for_its_sources_and_workload(monkeypatch):
+    """The stored ncu DRAM figure of the dK/dV kernel is reported for the workload it
+    was captured on while the kernel's sources hash to what was captured, else null."""
+    rec = dict(bench.DKDV_TRAFFIC)
+    assert bench.dkdv_traffic("some_other_workload") is None
+    monkeypatch.setattr(bench, "DKDV_TRAFFIC", dict(rec, sources_sha256="0" * 64))
+    assert bench.dkdv_traffic(rec["workload"]) is None
+    monkeypatch.setattr(bench, "DKDV_TRAFFIC", dict(rec, sources_sha256=bench.dkdv_sources_sha256()))
+    assert bench.dkdv_traffic(rec["workload"]) == rec["bytes"]
